@@ -1,0 +1,214 @@
+/*
+ * kvq.h - C ABI of the rotated-angle KV-cache codec and of decode attention
+ * over the compressed cache, for NVIDIA B200 (sm_100a).
+ *
+ * Method: "TurboAngle: Near-Lossless KV Cache Compression via Uniform Angle
+ * Quantization", Abstract.  Each key or value head vector is multiplied by a
+ * seeded random +-1 diagonal D, transformed by the Fast Walsh-Hadamard
+ * transform H (scaled by 1/sqrt(d)), split into consecutive element pairs,
+ * and every pair is stored as a uniformly quantized angle plus a quantized
+ * norm: 8-bit linear norms for keys, 4-bit log-space norms for values, with
+ * the codebook size L chosen per layer and separately for K and V
+ * ("per-layer early-boost").  Decode attention reads the codes directly and
+ * never materialises a dequantized cache (the on-the-fly reconstruction
+ * principle of "OCTOPUS: Joint Triplet Quantization for KV Cache via
+ * Octahedral Parametrization", sections "TL;DR" and "Why it matters").
+ *
+ * The pages give the method in words only.  This header fixes every formula
+ * and byte the library uses; where the pages are silent the plainest reading
+ * is taken and marked "(reading)".
+ *
+ * ---------------------------------------------------------------------------
+ * Definitions (d = head_dim, P = d/2 pairs, b = angle bits)
+ * ---------------------------------------------------------------------------
+ *   H      Sylvester-ordered Hadamard matrix, H[j][k] = (-1)^popcount(j & k)
+ *          (reading: natural order; H*H = d*I).
+ *   D      diagonal of signs s[k] in {+1,-1}, one vector per (layer, K|V),
+ *          passed in as data (int8, values +1 / -1).
+ *   z      = H * D * x / sqrt(d)                        (rotation, x fp16)
+ *   r_i    = |(z[2i], z[2i+1])|,  theta_i = atan2(z[2i+1], z[2i])
+ *   a_i    = floor((theta_i + pi) * L / (2 pi)) mod L   (uniform angle code;
+ *            a pair that is exactly (0,0) gets a_i = 0 (reading))
+ *   b      = smallest integer >= 1 with 2^b >= L        (bits per angle code)
+ *   Reconstruction angle (reading: bin centre, so |theta - theta^| <= pi/L):
+ *          theta^_a = -pi + (a + 1/2) * 2 pi / L
+ *
+ *   Norm modes (per codec):
+ *   KVQ_NORM_LIN8  M = fp16(max_i r_i) (round to nearest even; saturates to
+ *                  65504; reading), c_i = min(255, floor(255 r_i / M + 1/2)),
+ *                  all c_i = 0 when M = 0.  r^_i = c_i * M / 255.
+ *   KVQ_NORM_LOG4  l_i = log2(max(r_i, 2^-24)), LO = fp16(min_i l_i),
+ *                  HI = fp16(max_i l_i),
+ *                  c_i = clamp(floor(15 (l_i - LO) / (HI - LO) + 1/2), 0, 15),
+ *                  all c_i = 0 when HI = LO.
+ *                  r^_i = 2^(LO + c_i (HI - LO) / 15).
+ *   (round-half-up and the 2^-24 floor are readings.)
+ *
+ *   Dequantized vector: z^[2i] = r^_i cos theta^_i, z^[2i+1] = r^_i sin theta^_i,
+ *                       x^ = D * H * z^ / sqrt(d)   (the exact inverse rotation).
+ *
+ *   Decode attention for query head h (GQA: KV head = h / (H_q / H_kv),
+ *   reading: the usual grouped-query convention):
+ *     q'       = H * D_K * q / sqrt(d)                  (once per head)
+ *     s_t      = tau * sum_i r^K_{t,i} (q'[2i] cos theta^K_{t,i} + q'[2i+1] sin theta^K_{t,i})
+ *              (= tau * q . k^_t, because H*D/sqrt(d) is orthogonal)
+ *     p_t      = softmax_t(s_t) over t < ctx_len[b]  (no mask inside the range)
+ *     acc      = sum_t p_t z^V_t                        (rotated domain)
+ *     out      = D_V * H * acc / sqrt(d)                (one inverse FWHT per head)
+ *   tau is the softmax_scale argument (1/sqrt(d) is the usual choice).
+ *
+ * ---------------------------------------------------------------------------
+ * Packed layout of the compressed cache (one "plane" per K or V per layer)
+ * ---------------------------------------------------------------------------
+ * A plane is three caller-owned device arrays, each laid out
+ * [B][H_kv][capacity][row], row sizes from kvq_row_bytes():
+ *   angles  ceil(P*b/32) 32-bit little-endian words per token; code i lives in
+ *           bits [i*b, i*b + b) of the row's bit stream, where bit k of word w
+ *           is stream bit 32w + k (LSB first).
+ *   norms   LIN8: P bytes, byte i = c_i.
+ *           LOG4: P/2 bytes, byte j = c_{2j} | c_{2j+1} << 4.
+ *   params  LIN8: one IEEE fp16 M (2 bytes).  LOG4: fp16 LO then fp16 HI
+ *           (4 bytes).
+ * Requirements checked by every call: capacity % 16 == 0; every array
+ * 16-byte aligned.  Token t of sequence (b, h) is row (b*H_kv + h)*capacity + t.
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions
+ * ---------------------------------------------------------------------------
+ * Ownership: all memory is owned by the caller.  The library never allocates
+ *   or frees device memory; scratch space is passed in (workspace).
+ * Execution: every compute call is asynchronous on `stream` (a cudaStream_t,
+ *   passed as void*; NULL = legacy default stream).
+ * Errors: invalid arguments return KVQ_EINVAL or KVQ_EUNSUPPORTED before any
+ *   launch; a failed launch returns KVQ_ECUDA.  The message for the last
+ *   non-OK status of the calling thread is kvq_last_error().  Conditions seen
+ *   on the device (a ctx_len outside [0, capacity], a bounded wait that ran
+ *   out) are OR-ed into *err_word (KVQ_DEVERR_* bits) when err_word is not
+ *   NULL; the kernels never trap.
+ * Inputs must be finite; NaN or Inf inputs give unspecified codes.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_EINVAL = -1,       /* argument out of range, misaligned or NULL    */
+    KVQ_EUNSUPPORTED = -2, /* valid for the codec, not built into kernels  */
+    KVQ_ECUDA = -3,        /* CUDA runtime reported an error on launch     */
+    KVQ_ETIMEOUT = -4      /* reserved: a device-side bounded wait expired */
+} kvq_status;
+
+typedef enum { KVQ_NORM_LIN8 = 0, KVQ_NORM_LOG4 = 1 } kvq_norm_mode;
+
+/* Device error bits OR-ed into *err_word. */
+#define KVQ_DEVERR_CTX_RANGE 0x1  /* ctx_len[b] < 0 or > capacity: clipped   */
+#define KVQ_DEVERR_TIMEOUT 0x2    /* an mbarrier wait hit its iteration cap  */
+
+/* One codec: per layer and separately for K and V ("per-layer early-boost").
+ * head_dim: power of two, 4..256 for encode/dequant; 64 or 128 for decode.
+ * L: 2..65536 for encode/dequant; 2..256 for decode. */
+typedef struct {
+    int32_t head_dim;
+    int32_t L;
+    int32_t norm_mode; /* kvq_norm_mode */
+} kvq_codec;
+
+/* One compressed plane (see "Packed layout").  Pointers are device pointers
+ * owned by the caller; capacity is tokens per (batch, KV head). */
+typedef struct {
+    void* angles;
+    void* norms;
+    void* params;
+    int64_t capacity;
+} kvq_plane;
+
+/* Bytes per token of one plane array: which = 0 angles, 1 norms, 2 params.
+ * Returns a negative kvq_status for an invalid codec or `which`.  Host only. */
+int64_t kvq_row_bytes(const kvq_codec* codec, int32_t which);
+
+/* Bits per angle code for codebook size L (smallest b >= 1 with 2^b >= L);
+ * negative for L outside 2..65536.  Host only. */
+int32_t kvq_angle_bits(int32_t L);
+
+/* Encode (prefill when T > 1, append when T == 1).
+ * Follows the encode steps of the TurboAngle abstract (random diagonal, FWHT
+ * domain, consecutive pairs, uniform angles, 8-bit / 4-bit log norms).
+ *   signs  device int8 [head_dim], +1 / -1 (the diagonal D of this layer/K|V)
+ *   x      device fp16 [B][H_kv][T][head_dim], contiguous, 16-byte aligned
+ *   out    plane receiving tokens pos0 .. pos0+T-1 of every (b, h);
+ *          requires 0 <= pos0 and pos0 + T <= out->capacity.
+ * Codes are bit-exact to the definitions above except where a value lies
+ * within floating-point error of a decision edge of the definition (there
+ * the kernel re-decides from the exactly computed rotation in fp64).
+ * T == 0 is a no-op. */
+int kvq_encode(const kvq_codec* codec, const int8_t* signs, const void* x,
+               int32_t B, int32_t H_kv, int32_t T, int64_t pos0,
+               const kvq_plane* out, void* stream);
+
+/* Dequantize tokens pos0 .. pos0+T-1 of a plane back to fp16:
+ *   y  device fp16 [B][H_kv][T][head_dim], 16-byte aligned (x^ above). */
+int kvq_dequant(const kvq_codec* codec, const int8_t* signs,
+                const kvq_plane* in, int32_t B, int32_t H_kv, int32_t T,
+                int64_t pos0, void* y, void* stream);
+
+/* Split count the library would choose for a decode launch (host logic,
+ * deterministic): spreads B*H_kv*max_ctx over about two waves of CTAs on
+ * sm_count SMs, at least 1 and at most ceil(max_ctx / 16). */
+int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx,
+                              int32_t sm_count);
+
+/* Workspace bytes kvq_decode_attn needs for `num_splits` splits: per
+ * (b, query head, split) an fp32 running max, an fp32 softmax denominator
+ * and an fp32 [head_dim] partial accumulator (rotated domain). */
+int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim,
+                                   int32_t num_splits);
+
+/* Split-K decode attention over the compressed cache, one layer, one new
+ * query per sequence.
+ *   q          device fp16 [B][H_q][head_dim]
+ *   kc, vc     K and V codecs (same head_dim; kc LIN8, vc LOG4 in the
+ *              kernels built here, other mode pairs return EUNSUPPORTED)
+ *   signs_k/v  device int8 [head_dim] diagonals used when K / V were encoded
+ *   K, V       planes holding the cache; tokens 0 .. ctx_len[b]-1 are read
+ *   ctx_len    device int32 [B]; values are clipped to [0, min(max_ctx,
+ *              capacity)] and a clip sets KVQ_DEVERR_CTX_RANGE
+ *   max_ctx    host upper bound of ctx_len used to size the splits (>= 0)
+ *   softmax_scale  tau
+ *   num_splits >= 1 (kvq_decode_num_splits gives the default)
+ *   workspace  device scratch of ws_bytes >= kvq_decode_workspace_bytes(),
+ *              16-byte aligned; no initialisation needed; calls that share
+ *              a workspace must be stream-ordered
+ *   err_word   device int32 or NULL (see Errors)
+ *   out        device [B][H_q][head_dim], fp16 (out_dtype 0) or fp32 (1);
+ *              a sequence with ctx_len 0 gets zeros.
+ * Two kernels run on `stream`: the split-K pass and the combine pass (merge
+ * of the per-split softmax states, inverse FWHT, D_V / sqrt(d)). */
+int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc,
+                    const int8_t* signs_k, const int8_t* signs_v,
+                    const kvq_plane* K, const kvq_plane* V,
+                    const int32_t* ctx_len, int32_t B, int32_t H_q,
+                    int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                    int32_t num_splits, void* workspace, int64_t ws_bytes,
+                    int32_t* err_word, void* out, int32_t out_dtype,
+                    void* stream);
+
+/* Message for the last non-OK status returned on the calling thread
+ * (empty string if none).  The pointer stays valid until the next call on
+ * the same thread. */
+const char* kvq_last_error(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int32_t kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */
