@@ -1,0 +1,239 @@
+// kvq_abi.cu - the C ABI of include/kvq.h: argument checks, launch choice,
+// error reporting.  Every compute step runs in the kernels of this library.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "kvq_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok() {
+    g_err[0] = '\0';
+    return KVQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int sm_count_current() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+// Validate a codec and fill the device descriptor.  d_min/d_max bound head_dim.
+int check_codec(const kvq_codec* c, const char* what, kvq::CodecDev* out) {
+    if (!c) return fail(KVQ_EINVAL, "%s: codec is NULL", what);
+    if (!pow2(c->head_dim) || c->head_dim < 4 || c->head_dim > 256)
+        return fail(KVQ_EINVAL, "%s: head_dim %d is not a power of two in 4..256", what, c->head_dim);
+    const int b = kvq_angle_bits(c->L);
+    if (b < 0) return fail(KVQ_EINVAL, "%s: L = %d outside 2..65536", what, c->L);
+    if (c->norm_mode != KVQ_NORM_LIN8 && c->norm_mode != KVQ_NORM_LOG4)
+        return fail(KVQ_EINVAL, "%s: unknown norm_mode %d", what, c->norm_mode);
+    out->d = c->head_dim;
+    out->L = c->L;
+    out->bits = b;
+    out->mode = c->norm_mode;
+    out->angle_words = (int)(kvq_row_bytes(c, 0) / 4);
+    out->norm_bytes = (int)kvq_row_bytes(c, 1);
+    out->param_bytes = (int)kvq_row_bytes(c, 2);
+    return KVQ_OK;
+}
+
+int check_plane(const kvq_plane* p, const char* what, kvq::PlaneDev* out) {
+    if (!p) return fail(KVQ_EINVAL, "%s: plane is NULL", what);
+    if (!p->angles || !p->norms || !p->params)
+        return fail(KVQ_EINVAL, "%s: NULL plane array", what);
+    if (!aligned16(p->angles) || !aligned16(p->norms) || !aligned16(p->params))
+        return fail(KVQ_EINVAL, "%s: plane arrays must be 16-byte aligned", what);
+    if (p->capacity <= 0 || p->capacity % 16 != 0)
+        return fail(KVQ_EINVAL, "%s: capacity %lld must be a positive multiple of 16", what,
+                    (long long)p->capacity);
+    out->angles = static_cast<uint8_t*>(p->angles);
+    out->norms = static_cast<uint8_t*>(p->norms);
+    out->params = static_cast<uint8_t*>(p->params);
+    out->capacity = p->capacity;
+    return KVQ_OK;
+}
+
+int cuda_status(cudaError_t e, const char* what) {
+    if (e != cudaSuccess)
+        return fail(KVQ_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t kvq_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+const char* kvq_last_error(void) { return g_err; }
+
+int32_t kvq_angle_bits(int32_t L) {
+    if (L < 2 || L > 65536) return KVQ_EINVAL;
+    int32_t b = 1;
+    while ((1L << b) < (long)L) b++;
+    return b;
+}
+
+int64_t kvq_row_bytes(const kvq_codec* c, int32_t which) {
+    if (!c || !pow2(c->head_dim) || c->head_dim < 4 || c->head_dim > 256) return KVQ_EINVAL;
+    const int32_t b = kvq_angle_bits(c->L);
+    if (b < 0) return KVQ_EINVAL;
+    const int64_t P = c->head_dim / 2;
+    switch (which) {
+        case 0: return 4 * ((P * b + 31) / 32);
+        case 1:
+            if (c->norm_mode == KVQ_NORM_LIN8) return P;
+            if (c->norm_mode == KVQ_NORM_LOG4) return P / 2;
+            return KVQ_EINVAL;
+        case 2:
+            if (c->norm_mode == KVQ_NORM_LIN8) return 2;
+            if (c->norm_mode == KVQ_NORM_LOG4) return 4;
+            return KVQ_EINVAL;
+        default: return KVQ_EINVAL;
+    }
+}
+
+int kvq_encode(const kvq_codec* codec, const int8_t* signs, const void* x, int32_t B, int32_t H_kv,
+               int32_t T, int64_t pos0, const kvq_plane* out, void* stream) {
+    kvq::CodecDev c;
+    kvq::PlaneDev p;
+    int rc = check_codec(codec, "kvq_encode", &c);
+    if (rc) return rc;
+    rc = check_plane(out, "kvq_encode", &p);
+    if (rc) return rc;
+    if (B < 0 || H_kv < 0 || T < 0) return fail(KVQ_EINVAL, "kvq_encode: negative size");
+    if (pos0 < 0 || pos0 + (int64_t)T > p.capacity)
+        return fail(KVQ_EINVAL, "kvq_encode: tokens [%lld, %lld) exceed capacity %lld",
+                    (long long)pos0, (long long)(pos0 + T), (long long)p.capacity);
+    const int64_t n = (int64_t)B * H_kv * T;
+    if (n == 0) return ok();
+    if (!signs || !x) return fail(KVQ_EINVAL, "kvq_encode: NULL signs or x");
+    if (!aligned16(x)) return fail(KVQ_EINVAL, "kvq_encode: x must be 16-byte aligned");
+    return cuda_status(kvq::launch_encode(c, signs, static_cast<const __half*>(x), n, T, pos0, p,
+                                          sm_count_current(), static_cast<cudaStream_t>(stream)),
+                       "kvq_encode");
+}
+
+int kvq_dequant(const kvq_codec* codec, const int8_t* signs, const kvq_plane* in, int32_t B,
+                int32_t H_kv, int32_t T, int64_t pos0, void* y, void* stream) {
+    kvq::CodecDev c;
+    kvq::PlaneDev p;
+    int rc = check_codec(codec, "kvq_dequant", &c);
+    if (rc) return rc;
+    rc = check_plane(in, "kvq_dequant", &p);
+    if (rc) return rc;
+    if (B < 0 || H_kv < 0 || T < 0) return fail(KVQ_EINVAL, "kvq_dequant: negative size");
+    if (pos0 < 0 || pos0 + (int64_t)T > p.capacity)
+        return fail(KVQ_EINVAL, "kvq_dequant: tokens [%lld, %lld) exceed capacity %lld",
+                    (long long)pos0, (long long)(pos0 + T), (long long)p.capacity);
+    const int64_t n = (int64_t)B * H_kv * T;
+    if (n == 0) return ok();
+    if (!signs || !y) return fail(KVQ_EINVAL, "kvq_dequant: NULL signs or y");
+    if (!aligned16(y)) return fail(KVQ_EINVAL, "kvq_dequant: y must be 16-byte aligned");
+    return cuda_status(kvq::launch_dequant(c, signs, p, n, T, pos0, static_cast<__half*>(y),
+                                           sm_count_current(), static_cast<cudaStream_t>(stream)),
+                       "kvq_dequant");
+}
+
+int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx, int32_t sm_count) {
+    if (B <= 0 || H_kv <= 0 || max_ctx <= 0 || sm_count <= 0) return 1;
+    const int64_t units = (int64_t)B * H_kv;
+    const int64_t max_splits = (max_ctx + 15) / 16;
+    // about two waves of CTAs, and at least 64 tokens per split
+    int64_t s = (2LL * sm_count + units - 1) / units;
+    const int64_t by_len = (max_ctx + 63) / 64;
+    if (s > by_len) s = by_len;
+    if (s > max_splits) s = max_splits;
+    if (s > 65535) s = 65535;
+    if (s < 1) s = 1;
+    return (int32_t)s;
+}
+
+int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim, int32_t num_splits) {
+    if (B < 0 || H_q < 0 || head_dim <= 0 || num_splits <= 0) return KVQ_EINVAL;
+    return (int64_t)sizeof(float) * (kvq::ws_stat_floats(B, H_q, num_splits) +
+                                     kvq::ws_acc_floats(B, H_q, num_splits, head_dim));
+}
+
+int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc, const int8_t* signs_k,
+                    const int8_t* signs_v, const kvq_plane* K, const kvq_plane* V,
+                    const int32_t* ctx_len, int32_t B, int32_t H_q, int32_t H_kv, int64_t max_ctx,
+                    float softmax_scale, int32_t num_splits, void* workspace, int64_t ws_bytes,
+                    int32_t* err_word, void* out, int32_t out_dtype, void* stream) {
+    kvq::DecodeArgs a;
+    int rc = check_codec(kc, "kvq_decode_attn (K)", &a.kc);
+    if (rc) return rc;
+    rc = check_codec(vc, "kvq_decode_attn (V)", &a.vc);
+    if (rc) return rc;
+    rc = check_plane(K, "kvq_decode_attn (K)", &a.K);
+    if (rc) return rc;
+    rc = check_plane(V, "kvq_decode_attn (V)", &a.V);
+    if (rc) return rc;
+    if (a.kc.d != a.vc.d) return fail(KVQ_EINVAL, "kvq_decode_attn: K and V head_dim differ");
+    if (a.K.capacity != a.V.capacity)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: K and V capacity differ");
+    if (B < 0 || H_q < 0 || H_kv < 0 || max_ctx < 0)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: negative size");
+    if (B == 0 || H_q == 0) return ok();
+    if (B > 65535 || H_kv > 65535)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: B and H_kv must be at most 65535");
+    if (H_kv <= 0 || H_q % H_kv != 0)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: H_q %d is not a multiple of H_kv %d", H_q, H_kv);
+    if (num_splits < 1 || num_splits > 65535)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: num_splits %d outside 1..65535", num_splits);
+    if (out_dtype != 0 && out_dtype != 1)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: out_dtype must be 0 (fp16) or 1 (fp32)");
+    if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: softmax_scale is not finite");
+    const int G = H_q / H_kv;
+    if (!kvq::decode_supported(a.kc.d, G, a.kc.L, a.vc.L, a.kc.mode, a.vc.mode))
+        return fail(KVQ_EUNSUPPORTED,
+                    "kvq_decode_attn: no kernel for head_dim %d, G %d, L_K %d, L_V %d "
+                    "(built: head_dim 64/128, G 1/2/4/8, L <= 256)",
+                    a.kc.d, G, a.kc.L, a.vc.L);
+    const int64_t need = kvq_decode_workspace_bytes(B, H_q, a.kc.d, num_splits);
+    if (!workspace || ws_bytes < need)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: workspace of %lld bytes is below the %lld needed",
+                    (long long)ws_bytes, (long long)need);
+    if (!aligned16(workspace)) return fail(KVQ_EINVAL, "kvq_decode_attn: workspace not 16-byte aligned");
+    if (!q || !signs_k || !signs_v || !ctx_len || !out)
+        return fail(KVQ_EINVAL, "kvq_decode_attn: NULL q, signs, ctx_len or out");
+    a.q = static_cast<const __half*>(q);
+    a.signs_k = signs_k;
+    a.signs_v = signs_v;
+    a.ctx_len = ctx_len;
+    a.B = B;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.max_ctx = max_ctx;
+    a.scale_log2 = softmax_scale * 1.4426950408889634f;
+    a.num_splits = num_splits;
+    int64_t sl = (max_ctx + num_splits - 1) / num_splits;
+    sl = (sl + 15) / 16 * 16;
+    a.split_len = sl < 16 ? 16 : sl;
+    a.ws = static_cast<float*>(workspace);
+    a.err_word = err_word;
+    a.out = out;
+    a.out_dtype = out_dtype;
+    return cuda_status(kvq::launch_decode(a, static_cast<cudaStream_t>(stream)), "kvq_decode_attn");
+}
+
+}  // extern "C"

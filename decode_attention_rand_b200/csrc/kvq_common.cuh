@@ -1,0 +1,162 @@
+// kvq_common.cuh - device helpers shared by the kvq kernels (sm_100a).
+//
+// Codec of "TurboAngle: Near-Lossless KV Cache Compression via Uniform Angle
+// Quantization" (Abstract): +-1 diagonal, Walsh-Hadamard transform scaled by
+// 1/sqrt(d), consecutive pairs as (norm, uniformly quantized angle).  The
+// exact formulas and the byte layout are the ones stated in include/kvq.h.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+
+#define KVQ_FULL_MASK 0xffffffffu
+
+namespace kvq {
+
+constexpr float kPiF = 3.14159265358979323846f;
+constexpr double kPi = 3.14159265358979323846264338327950288;
+
+// ---------------------------------------------------------------- codec --
+
+struct CodecDev {
+    int d;          // head dim
+    int L;          // codebook size
+    int bits;       // bits per angle code
+    int mode;       // KVQ_NORM_LIN8 / KVQ_NORM_LOG4
+    int angle_words;  // 32-bit words per token row
+    int norm_bytes;   // bytes per token row
+    int param_bytes;  // 2 (LIN8) or 4 (LOG4)
+};
+
+struct PlaneDev {
+    uint8_t* angles;
+    uint8_t* norms;
+    uint8_t* params;
+    int64_t capacity;
+};
+
+// --------------------------------------------------------------- warps --
+
+template <int WIDTH>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+    for (int o = WIDTH / 2; o > 0; o >>= 1) v += __shfl_xor_sync(KVQ_FULL_MASK, v, o);
+    return v;
+}
+
+template <int WIDTH>
+__device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+    for (int o = WIDTH / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(KVQ_FULL_MASK, v, o));
+    return v;
+}
+
+template <int WIDTH>
+__device__ __forceinline__ float group_min(float v) {
+#pragma unroll
+    for (int o = WIDTH / 2; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(KVQ_FULL_MASK, v, o));
+    return v;
+}
+
+template <int WIDTH>
+__device__ __forceinline__ double group_max_d(double v) {
+#pragma unroll
+    for (int o = WIDTH / 2; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(KVQ_FULL_MASK, v, o));
+    return v;
+}
+
+template <int WIDTH>
+__device__ __forceinline__ double group_min_d(double v) {
+#pragma unroll
+    for (int o = WIDTH / 2; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(KVQ_FULL_MASK, v, o));
+    return v;
+}
+
+template <int WIDTH>
+__device__ __forceinline__ bool group_any(bool p) {
+    unsigned b = __ballot_sync(KVQ_FULL_MASK, p);
+    if (WIDTH == 32) return b != 0u;
+    const int lane = threadIdx.x & 31;
+    const unsigned gmask = ((1u << WIDTH) - 1u) << (lane & ~(WIDTH - 1));
+    return (b & gmask) != 0u;
+}
+
+// ------------------------------------------------------------ FWHT -------
+// In-register Sylvester-ordered Walsh-Hadamard butterflies over the EPL
+// elements a lane holds, followed by the cross-lane stages over NL lanes.
+// Element g of the vector lives in lane g / EPL (within its group), slot
+// g % EPL, so stage p pairs g with g ^ (1 << p): out[g] = v[g] + v[g'] for the
+// lower index and v[g] - v[g'] for the upper one (natural-order transform).
+
+template <int EPL, typename T>
+__device__ __forceinline__ void fwht_local(T (&v)[EPL]) {
+#pragma unroll
+    for (int h = 1; h < EPL; h <<= 1) {
+#pragma unroll
+        for (int e = 0; e < EPL; e++) {
+            if ((e & h) == 0) {
+                T a = v[e], b = v[e + h];
+                v[e] = a + b;
+                v[e + h] = a - b;
+            }
+        }
+    }
+}
+
+template <int EPL, int NL, typename T>
+__device__ __forceinline__ void fwht_cross(T (&v)[EPL], int lane_g) {
+#pragma unroll
+    for (int m = 1; m < NL; m <<= 1) {
+        const bool upper = (lane_g & m) != 0;
+#pragma unroll
+        for (int e = 0; e < EPL; e++) {
+            T o = __shfl_xor_sync(KVQ_FULL_MASK, v[e], m);
+            v[e] = upper ? (o - v[e]) : (v[e] + o);
+        }
+    }
+}
+
+// -------------------------------------------------------------- fp16 ----
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+    return __half2float(__ushort_as_half(h));
+}
+
+// fp16 round-to-nearest-even of a non-negative fp32 value, saturated to the
+// largest finite fp16 (the codec's parameter rule).
+__device__ __forceinline__ uint16_t f32_to_f16_sat(float x) {
+    uint16_t h = __half_as_ushort(__float2half_rn(x));
+    if ((h & 0x7FFF) >= 0x7C00) h = (uint16_t)((h & 0x8000) | 0x7BFF);
+    return h;
+}
+
+__device__ __forceinline__ uint16_t f64_to_f16_sat(double x) {
+    uint16_t h = __half_as_ushort(__double2half(x));
+    if ((h & 0x7FFF) >= 0x7C00) h = (uint16_t)((h & 0x8000) | 0x7BFF);
+    return h;
+}
+
+// True when |x| lies within tol of a midpoint between two adjacent finite
+// fp16 values, i.e. where the fp16 rounding of the exact value could differ
+// from the rounding of x.  Midpoints of fp16 values are exact in fp32.
+__device__ __forceinline__ bool near_f16_midpoint(float x, float tol) {
+    const float a = fabsf(x);
+    uint16_t h = __half_as_ushort(__float2half_rn(a));
+    if (h >= 0x7C00) h = 0x7BFF;
+    const float hv = half_bits_to_float(h);
+    bool near = false;
+    if (h < 0x7BFF) near |= fabsf(a - 0.5f * (hv + half_bits_to_float((uint16_t)(h + 1)))) <= tol;
+    if (h > 0) near |= fabsf(a - 0.5f * (hv + half_bits_to_float((uint16_t)(h - 1)))) <= tol;
+    return near;
+}
+
+// ------------------------------------------------------ device errors ----
+
+__device__ __forceinline__ void report(int32_t* err_word, int bits) {
+    if (err_word) atomicOr(err_word, bits);
+}
+
+}  // namespace kvq

@@ -1,0 +1,415 @@
+// kvq_encode.cu - encode/append kernel: fp16 head vectors -> packed angle and
+// norm codes ("TurboAngle: Near-Lossless KV Cache Compression via Uniform
+// Angle Quantization", Abstract: random diagonal, FWHT domain, consecutive
+// pairs, uniform angles, 8-bit linear K norms / 4-bit log-space V norms).
+//
+// Layout of the work: one head vector per group of NL = d/EPL lanes, each
+// lane holding EPL (<= 16) consecutive elements, loaded with 128-bit loads.
+// The Walsh-Hadamard transform runs in registers (log2 EPL stages) and
+// across the group with shuffles (log2 NL stages).
+//
+// Exactness.  Codes must equal the definition's exactly except within a hair
+// of a decision edge.  The fast path works in fp32 and carries a rigorous
+// error bound for every quantity that feeds a decision:
+//   - FWHT: every butterfly rounds once, so after S stages each output is
+//     within S * 2^-24 * |x|_1 of the exact value (|x|_1 = L1 norm of the
+//     input), the classical bound for a +-1 butterfly network;
+//   - sqrt and division are correctly rounded (IEEE, no fast-math);
+//     atan2f is documented to 3 ulp and log2f to 1 ulp; the margins below
+//     allow several times that.
+// Any decision (angle bin, norm code, fp16 parameter) whose fp32 value lies
+// within its error bound of the edge sends the whole warp through an exact
+// path: the transform is recomputed in fp64, where it is exact (fp16 inputs
+// are integer multiples of 2^-24 below 2^16, so all partial sums over d <= 256
+// terms fit in 53 bits), and the flagged decisions are re-taken in fp64 with
+// the definition's own formula.  The remaining disagreement with any other
+// exact implementation is confined to values within an fp64 rounding of an
+// edge.
+#include "kvq_internal.h"
+
+namespace kvq {
+
+template <int D>
+struct EncCfg {
+    static constexpr int EPL = D < 16 ? D : 16;  // elements per lane
+    static constexpr int NL = D / EPL;           // lanes per vector
+    static constexpr int PPL = EPL / 2;          // pairs per lane
+    static constexpr int VPW = 32 / NL;          // vectors per warp
+    static constexpr int S = D == 4 ? 2 : D == 8 ? 3 : D == 16 ? 4 : D == 32 ? 5 : D == 64 ? 6
+                           : D == 128 ? 7 : 8;   // log2 D
+};
+
+constexpr int kEncWarps = 8;
+constexpr int kEncStageWords = 128;  // max VPW * angle_words over all D, b <= 16
+
+struct EncArgs {
+    const __half* x;
+    const int8_t* signs;
+    int64_t n_vec;
+    int64_t T;
+    int64_t pos0;
+    CodecDev c;
+    PlaneDev out;
+    float inv_sqrt_d;
+    float bins_per_rad;  // L / (2 pi)
+};
+
+__device__ __forceinline__ int exact_angle_code(double u, double v, int L) {
+    if (u == 0.0 && v == 0.0) return 0;
+    const double theta = atan2(v, u);
+    const double t = (theta + kPi) * (double)L / (2.0 * kPi);
+    return (int)floor(t) % L;
+}
+
+__device__ __forceinline__ int lin8_code_exact(double r, double M) {
+    if (M == 0.0) return 0;
+    const double q = floor(255.0 * r / M + 0.5);
+    return q > 255.0 ? 255 : (int)q;
+}
+
+__device__ __forceinline__ int log4_code_exact(double l, double LO, double HI) {
+    if (HI == LO) return 0;
+    const double q = floor(15.0 * (l - LO) / (HI - LO) + 0.5);
+    return q < 0.0 ? 0 : (q > 15.0 ? 15 : (int)q);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kEncWarps * 32)
+encode_kernel(EncArgs A) {
+    using Cfg = EncCfg<D>;
+    constexpr int EPL = Cfg::EPL, NL = Cfg::NL, PPL = Cfg::PPL, VPW = Cfg::VPW;
+    __shared__ uint32_t stage[kEncWarps][kEncStageWords];
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int grp = lane / NL;
+    const int lg = lane % NL;
+    const int L = A.c.L;
+    const int bits = A.c.bits;
+    const int AW = A.c.angle_words;
+    const float Lf = (float)L;
+
+    uint32_t* st = stage[warp];
+    for (int i = lane; i < kEncStageWords; i += 32) st[i] = 0u;
+
+    // signs of this lane's elements (bit e set: negate element lg*EPL + e)
+    uint32_t negmask = 0;
+#pragma unroll
+    for (int e = 0; e < EPL; e++) negmask |= (A.signs[lg * EPL + e] < 0 ? 1u : 0u) << e;
+
+    const double sqrt_d = sqrt((double)D);
+    const float ez_scale = (float)Cfg::S * 5.9604645e-8f * 1.0001f;  // S * 2^-24, padded
+    const int64_t n_warps_total = (int64_t)gridDim.x * kEncWarps;
+    const int64_t n_warp_tiles = (A.n_vec + VPW - 1) / VPW;
+
+    for (int64_t wt = (int64_t)blockIdx.x * kEncWarps + warp; wt < n_warp_tiles; wt += n_warps_total) {
+        const int64_t v = wt * VPW + grp;
+        const bool valid = v < A.n_vec;
+
+        // ---- load EPL fp16 values (128-bit loads) ----------------------
+        uint32_t raw[EPL / 2];
+        {
+            const __half* src = A.x + (valid ? v : 0) * D + lg * EPL;
+            if constexpr (EPL == 16) {
+                const uint4 q0 = reinterpret_cast<const uint4*>(src)[0];
+                const uint4 q1 = reinterpret_cast<const uint4*>(src)[1];
+                raw[0] = q0.x; raw[1] = q0.y; raw[2] = q0.z; raw[3] = q0.w;
+                raw[4] = q1.x; raw[5] = q1.y; raw[6] = q1.z; raw[7] = q1.w;
+            } else if constexpr (EPL == 8) {
+                const uint4 q0 = reinterpret_cast<const uint4*>(src)[0];
+                raw[0] = q0.x; raw[1] = q0.y; raw[2] = q0.z; raw[3] = q0.w;
+            } else {
+                const uint2 q0 = reinterpret_cast<const uint2*>(src)[0];
+                raw[0] = q0.x; raw[1] = q0.y;
+            }
+            if (!valid) {
+#pragma unroll
+                for (int i = 0; i < EPL / 2; i++) raw[i] = 0u;
+            }
+        }
+
+        // ---- D x in fp32 (exact), L1 norm, FWHT --------------------------
+        float z[EPL];
+        float l1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; e++) {
+            const uint16_t hb = (uint16_t)(raw[e / 2] >> (16 * (e & 1)));
+            float f = half_bits_to_float(hb);
+            f = ((negmask >> e) & 1u) ? -f : f;
+            z[e] = f;
+            l1 += fabsf(f);
+        }
+        l1 = group_sum<NL>(l1);
+        fwht_local<EPL>(z);
+        fwht_cross<EPL, NL>(z, lg);
+        const float Ez = ez_scale * l1;  // bound on |z_fp32 - z_exact| (unscaled)
+
+        // ---- per pair: angle code and norm, with margins -------------------
+        int acode[PPL];
+        float rr[PPL];
+        float er[PPL];
+        uint32_t need_a = 0, need_n = 0;
+#pragma unroll
+        for (int i = 0; i < PPL; i++) {
+            const float x = z[2 * i], y = z[2 * i + 1];
+            const float rho = sqrtf(fmaf(x, x, y * y));
+            int a = 0;
+            if (!(rho > 4.f * Ez) || rho == 0.f) {
+                need_a |= 1u << i;
+            } else {
+                const float th = atan2f(y, x);
+                const float u = (th + kPiF) * A.bins_per_rad;
+                const float fl = floorf(u);
+                const float fr = u - fl;
+                const float dth = 2.f * Ez / (rho - 2.f * Ez);
+                const float du = A.bins_per_rad * (4.5e-6f + dth) + Lf * 1.2e-7f;
+                if (fr < du || fr > 1.f - du) need_a |= 1u << i;
+                a = (int)fl;
+                a = a >= L ? a - L : (a < 0 ? a + L : a);
+            }
+            acode[i] = a;
+            rr[i] = rho * A.inv_sqrt_d;
+            er[i] = 1.5f * Ez * A.inv_sqrt_d + rr[i] * 4e-7f;
+        }
+
+        int ncode[PPL];
+        uint32_t prm = 0;    // packed fp16 parameter(s)
+        bool need_p = false;  // group-uniform
+        if (A.c.mode == KVQ_NORM_LIN8) {
+            float m = 0.f;
+#pragma unroll
+            for (int i = 0; i < PPL; i++) m = fmaxf(m, rr[i]);
+            m = group_max<NL>(m);
+            const float eM = 1.5f * Ez * A.inv_sqrt_d + m * 4e-7f;
+            need_p = near_f16_midpoint(m, eM);
+            const uint16_t Mh = f32_to_f16_sat(m);
+            const float Mf = half_bits_to_float(Mh);
+            prm = Mh;
+            const float inv = Mf > 0.f ? 255.f / Mf : 0.f;
+#pragma unroll
+            for (int i = 0; i < PPL; i++) {
+                int cc = 0;
+                if (Mf > 0.f) {
+                    const float vq = rr[i] * inv;
+                    const float t = vq + 0.5f;
+                    const float fl = floorf(t);
+                    const float fr = t - fl;
+                    const float dv = er[i] * inv * 1.0001f + vq * 2.5e-7f + 1e-6f;
+                    if (fr < dv || fr > 1.f - dv) need_n |= 1u << i;
+                    cc = min(255, (int)fl);
+                }
+                ncode[i] = cc;
+            }
+        } else {
+            float lmin = 1e30f, lmax = -1e30f, elmax = 0.f;
+            bool unsure = false;
+            float ll[PPL], el[PPL];
+#pragma unroll
+            for (int i = 0; i < PPL; i++) {
+                const float r = rr[i];
+                unsure |= (r < 2.3841858e-7f) || (er[i] > 0.01f * r);  // r < 2^-22
+                const float l = log2f(fmaxf(r, 5.9604645e-8f));
+                ll[i] = l;
+                el[i] = er[i] / (fmaxf(r, 1e-30f) * 0.69314718f) * 1.02f + fabsf(l) * 2.4e-7f + 1e-7f;
+                lmin = fminf(lmin, l);
+                lmax = fmaxf(lmax, l);
+                elmax = fmaxf(elmax, el[i]);
+            }
+            lmin = group_min<NL>(lmin);
+            lmax = group_max<NL>(lmax);
+            elmax = group_max<NL>(elmax);
+            unsure = group_any<NL>(unsure);
+            need_p = unsure || near_f16_midpoint(lmin, elmax) || near_f16_midpoint(lmax, elmax);
+            const uint16_t LOh = f32_to_f16_sat(lmin), HIh = f32_to_f16_sat(lmax);
+            const float LOf = half_bits_to_float(LOh), HIf = half_bits_to_float(HIh);
+            prm = (uint32_t)LOh | ((uint32_t)HIh << 16);
+            const float inv = HIf != LOf ? 15.f / (HIf - LOf) : 0.f;
+#pragma unroll
+            for (int i = 0; i < PPL; i++) {
+                int cc = 0;
+                if (HIf != LOf) {
+                    const float vq = (ll[i] - LOf) * inv;
+                    const float t = vq + 0.5f;
+                    const float fl = floorf(t);
+                    const float fr = t - fl;
+                    const float dv = (el[i] + (fabsf(ll[i]) + fabsf(LOf)) * 1.2e-7f) * inv * 1.01f +
+                                     fabsf(vq) * 2.5e-7f + 1e-6f;
+                    if (fr < dv || fr > 1.f - dv) need_n |= 1u << i;
+                    cc = min(15, max(0, (int)fl));
+                }
+                ncode[i] = cc;
+            }
+        }
+
+        // ---- exact path: fp64 transform, re-decide what was near an edge --
+        const bool lane_need = valid && ((need_a | need_n) != 0u || need_p);
+        if (__any_sync(KVQ_FULL_MASK, lane_need)) {
+            double zd[EPL];
+#pragma unroll
+            for (int e = 0; e < EPL; e++) {
+                const uint16_t hb = (uint16_t)(raw[e / 2] >> (16 * (e & 1)));
+                const double f = (double)half_bits_to_float(hb);
+                zd[e] = ((negmask >> e) & 1u) ? -f : f;
+            }
+            fwht_local<EPL>(zd);
+            fwht_cross<EPL, NL>(zd, lg);
+            double r64[PPL];
+#pragma unroll
+            for (int i = 0; i < PPL; i++) {
+                if ((need_a >> i) & 1u) acode[i] = exact_angle_code(zd[2 * i], zd[2 * i + 1], L);
+                r64[i] = hypot(zd[2 * i] / sqrt_d, zd[2 * i + 1] / sqrt_d);
+            }
+            const bool gp = need_p;  // uniform within the group
+            if (A.c.mode == KVQ_NORM_LIN8) {
+                double m = 0.0;
+#pragma unroll
+                for (int i = 0; i < PPL; i++) m = fmax(m, r64[i]);
+                m = group_max_d<NL>(m);
+                if (gp) prm = f64_to_f16_sat(m);
+                const double M = (double)half_bits_to_float((uint16_t)prm);
+#pragma unroll
+                for (int i = 0; i < PPL; i++)
+                    if (gp || ((need_n >> i) & 1u)) ncode[i] = lin8_code_exact(r64[i], M);
+            } else {
+                double l64[PPL];
+                double lo = 1e300, hi = -1e300;
+#pragma unroll
+                for (int i = 0; i < PPL; i++) {
+                    l64[i] = log2(fmax(r64[i], 5.9604644775390625e-8));
+                    lo = fmin(lo, l64[i]);
+                    hi = fmax(hi, l64[i]);
+                }
+                lo = group_min_d<NL>(lo);
+                hi = group_max_d<NL>(hi);
+                if (gp) prm = (uint32_t)f64_to_f16_sat(lo) | ((uint32_t)f64_to_f16_sat(hi) << 16);
+                const double LO = (double)half_bits_to_float((uint16_t)(prm & 0xFFFF));
+                const double HI = (double)half_bits_to_float((uint16_t)(prm >> 16));
+#pragma unroll
+                for (int i = 0; i < PPL; i++)
+                    if (gp || ((need_n >> i) & 1u)) ncode[i] = log4_code_exact(l64[i], LO, HI);
+            }
+        }
+
+        // ---- pack and store ------------------------------------------------
+        int64_t row = 0;
+        if (valid) {
+            const int64_t bh = v / A.T;
+            row = bh * A.out.capacity + A.pos0 + (v - bh * A.T);
+        }
+        // angle bit stream: this lane's PPL codes occupy bits [cb, cb + PPL*bits)
+        {
+            uint64_t lo = 0, hi = 0;
+#pragma unroll
+            for (int k = 0; k < PPL; k++) {
+                const int pos = k * bits;
+                const uint64_t a = (uint64_t)(uint32_t)acode[k];
+                if (pos < 64) {
+                    lo |= a << pos;
+                    if (pos + bits > 64) hi |= a >> (64 - pos);
+                } else {
+                    hi |= a << (pos - 64);
+                }
+            }
+            const int cb = lg * PPL * bits;
+            const int w0 = cb >> 5, sh = cb & 31;
+            uint32_t w[5];
+            // 160-bit shift of (hi:lo) left by sh, split in words
+            {
+                const uint64_t l2 = sh ? (lo << sh) : lo;
+                const uint64_t h2 = sh ? ((hi << sh) | (lo >> (64 - sh))) : hi;
+                const uint32_t top = sh ? (uint32_t)(hi >> (64 - sh)) : 0u;
+                w[0] = (uint32_t)l2;
+                w[1] = (uint32_t)(l2 >> 32);
+                w[2] = (uint32_t)h2;
+                w[3] = (uint32_t)(h2 >> 32);
+                w[4] = top;
+            }
+            if (valid) {
+#pragma unroll
+                for (int j = 0; j < 5; j++)
+                    if (w[j] != 0u && w0 + j < AW) atomicOr(&st[grp * AW + w0 + j], w[j]);
+            }
+            __syncwarp();
+            if (valid) {
+                uint32_t* dst = reinterpret_cast<uint32_t*>(A.out.angles) + row * AW;
+                for (int j = lg; j < AW; j += NL) {
+                    dst[j] = st[grp * AW + j];
+                    st[grp * AW + j] = 0u;
+                }
+            }
+            __syncwarp();
+        }
+        if (valid) {
+            if (A.c.mode == KVQ_NORM_LIN8) {
+                uint8_t* dst = A.out.norms + row * (D / 2) + lg * PPL;
+                if constexpr (PPL == 8) {
+                    uint2 q;
+                    q.x = (uint32_t)ncode[0] | (uint32_t)ncode[1] << 8 | (uint32_t)ncode[2] << 16 |
+                          (uint32_t)ncode[3] << 24;
+                    q.y = (uint32_t)ncode[4] | (uint32_t)ncode[5] << 8 | (uint32_t)ncode[6] << 16 |
+                          (uint32_t)ncode[7] << 24;
+                    *reinterpret_cast<uint2*>(dst) = q;
+                } else if constexpr (PPL == 4) {
+                    *reinterpret_cast<uint32_t*>(dst) = (uint32_t)ncode[0] | (uint32_t)ncode[1] << 8 |
+                                                        (uint32_t)ncode[2] << 16 |
+                                                        (uint32_t)ncode[3] << 24;
+                } else {
+                    *reinterpret_cast<uint16_t*>(dst) = (uint16_t)(ncode[0] | ncode[1] << 8);
+                }
+                if (lg == 0) reinterpret_cast<uint16_t*>(A.out.params)[row] = (uint16_t)prm;
+            } else {
+                uint8_t* dst = A.out.norms + row * (D / 4) + lg * (PPL / 2);
+                uint32_t packed = 0;
+#pragma unroll
+                for (int i = 0; i < PPL; i++) packed |= (uint32_t)ncode[i] << (4 * i);
+                if constexpr (PPL == 8) {
+                    *reinterpret_cast<uint32_t*>(dst) = packed;
+                } else if constexpr (PPL == 4) {
+                    *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+                } else {
+                    *dst = (uint8_t)packed;
+                }
+                if (lg == 0) reinterpret_cast<uint32_t*>(A.out.params)[row] = prm;
+            }
+        }
+    }
+}
+
+template <int D>
+static cudaError_t launch_encode_d(const EncArgs& a, int sm_count, cudaStream_t stream) {
+    constexpr int VPW = EncCfg<D>::VPW;
+    const int64_t tiles = (a.n_vec + VPW - 1) / VPW;
+    int64_t blocks = (tiles + kEncWarps - 1) / kEncWarps;
+    const int64_t cap = (int64_t)sm_count * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    encode_kernel<D><<<(unsigned)blocks, kEncWarps * 32, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_encode(const CodecDev& c, const int8_t* signs, const __half* x, int64_t n_vec,
+                          int64_t T, int64_t pos0, const PlaneDev& out, int sm_count,
+                          cudaStream_t stream) {
+    EncArgs a;
+    a.x = x;
+    a.signs = signs;
+    a.n_vec = n_vec;
+    a.T = T;
+    a.pos0 = pos0;
+    a.c = c;
+    a.out = out;
+    a.inv_sqrt_d = (float)(1.0 / sqrt((double)c.d));
+    a.bins_per_rad = (float)((double)c.L / (2.0 * kPi));
+    switch (c.d) {
+        case 4: return launch_encode_d<4>(a, sm_count, stream);
+        case 8: return launch_encode_d<8>(a, sm_count, stream);
+        case 16: return launch_encode_d<16>(a, sm_count, stream);
+        case 32: return launch_encode_d<32>(a, sm_count, stream);
+        case 64: return launch_encode_d<64>(a, sm_count, stream);
+        case 128: return launch_encode_d<128>(a, sm_count, stream);
+        case 256: return launch_encode_d<256>(a, sm_count, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace kvq

@@ -1,0 +1,45 @@
+// kvq_internal.h - declarations shared between the kvq kernels and the C ABI
+// layer (not installed; the public interface is include/kvq.h).
+#pragma once
+
+#include "kvq_common.cuh"
+
+namespace kvq {
+
+cudaError_t launch_encode(const CodecDev& c, const int8_t* signs, const __half* x, int64_t n_vec,
+                          int64_t T, int64_t pos0, const PlaneDev& out, int sm_count,
+                          cudaStream_t stream);
+
+cudaError_t launch_dequant(const CodecDev& c, const int8_t* signs, const PlaneDev& in,
+                           int64_t n_vec, int64_t T, int64_t pos0, __half* y, int sm_count,
+                           cudaStream_t stream);
+
+struct DecodeArgs {
+    const __half* q;        // [B][H_q][d]
+    CodecDev kc, vc;
+    const int8_t* signs_k;
+    const int8_t* signs_v;
+    PlaneDev K, V;
+    const int32_t* ctx_len;  // [B]
+    int B, H_q, H_kv;
+    int64_t max_ctx;
+    float scale_log2;        // softmax_scale * log2(e)
+    int num_splits;
+    int64_t split_len;       // tokens per split, multiple of 16
+    float* ws;               // partials: [B][H_q][S] x (m, l) then acc [B][H_q][S][d]
+    int32_t* err_word;
+    void* out;
+    int out_dtype;
+};
+
+// True when the decode kernels are built for this (head_dim, G, L_K, L_V)
+// and norm-mode combination.
+bool decode_supported(int d, int G, int LK, int LV, int mode_k, int mode_v);
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Workspace layout helpers (host and device agree through these).
+__host__ __device__ inline int64_t ws_stat_floats(int B, int H_q, int S) { return (int64_t)B * H_q * S * 2; }
+__host__ __device__ inline int64_t ws_acc_floats(int B, int H_q, int S, int d) { return (int64_t)B * H_q * S * d; }
+
+}  // namespace kvq

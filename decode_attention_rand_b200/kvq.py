@@ -1,0 +1,244 @@
+"""Thin ctypes binding of libkvq.so (include/kvq.h).
+
+Argument marshalling only: every step of encode, dequant and decode attention
+runs in the CUDA kernels of libkvq.so.  PyTorch provides device memory and
+streams.  The functions named ``kvq_*`` mirror the C entry points one to one
+(they take the same arguments, as ctypes values or torch tensors, and raise
+KvqError on a non-OK status); the small helpers below them only allocate
+caller-owned buffers with torch and fill the C structs.
+
+A missing or unloadable libkvq.so raises at first use: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+import threading
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvq.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "kvq.h")
+
+KVQ_OK, KVQ_EINVAL, KVQ_EUNSUPPORTED, KVQ_ECUDA, KVQ_ETIMEOUT = 0, -1, -2, -3, -4
+KVQ_NORM_LIN8, KVQ_NORM_LOG4 = 0, 1
+KVQ_DEVERR_CTX_RANGE, KVQ_DEVERR_TIMEOUT = 0x1, 0x2
+OUT_FP16, OUT_FP32 = 0, 1
+
+
+class KvqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"kvq status {status}: {message}")
+        self.status = status
+
+
+class kvq_codec(C.Structure):
+    _fields_ = [("head_dim", C.c_int32), ("L", C.c_int32), ("norm_mode", C.c_int32)]
+
+
+class kvq_plane(C.Structure):
+    _fields_ = [("angles", C.c_void_p), ("norms", C.c_void_p), ("params", C.c_void_p),
+                ("capacity", C.c_int64)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+_SIGNATURES = {
+    "kvq_version": (C.c_int32, []),
+    "kvq_last_error": (C.c_char_p, []),
+    "kvq_angle_bits": (C.c_int32, [C.c_int32]),
+    "kvq_row_bytes": (C.c_int64, [C.POINTER(kvq_codec), C.c_int32]),
+    "kvq_encode": (C.c_int, [C.POINTER(kvq_codec), C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
+                             C.c_int32, C.c_int64, C.POINTER(kvq_plane), C.c_void_p]),
+    "kvq_dequant": (C.c_int, [C.POINTER(kvq_codec), C.c_void_p, C.POINTER(kvq_plane), C.c_int32,
+                              C.c_int32, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]),
+    "kvq_decode_num_splits": (C.c_int32, [C.c_int32, C.c_int32, C.c_int64, C.c_int32]),
+    "kvq_decode_workspace_bytes": (C.c_int64, [C.c_int32, C.c_int32, C.c_int32, C.c_int32]),
+    "kvq_decode_attn": (C.c_int, [C.c_void_p, C.POINTER(kvq_codec), C.POINTER(kvq_codec),
+                                  C.c_void_p, C.c_void_p, C.POINTER(kvq_plane),
+                                  C.POINTER(kvq_plane), C.c_void_p, C.c_int32, C.c_int32,
+                                  C.c_int32, C.c_int64, C.c_float, C.c_int32, C.c_void_p,
+                                  C.c_int64, C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p]),
+}
+
+
+def lib():
+    """The loaded libkvq.so (raises if it is missing or does not load)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise KvqError(KVQ_EUNSUPPORTED,
+                               f"{LIB_PATH} is missing; build it with "
+                               "`python -m decode_attention_rand_b200.build`")
+            L = C.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGNATURES.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/kvq.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(rc: int):
+    if rc != KVQ_OK:
+        raise KvqError(rc, lib().kvq_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------ C ABI --
+
+def kvq_version() -> int:
+    return lib().kvq_version()
+
+
+def kvq_last_error() -> str:
+    return lib().kvq_last_error().decode()
+
+
+def kvq_angle_bits(L: int) -> int:
+    return lib().kvq_angle_bits(L)
+
+
+def kvq_row_bytes(codec: kvq_codec, which: int) -> int:
+    return lib().kvq_row_bytes(C.byref(codec), which)
+
+
+def kvq_encode(codec: kvq_codec, signs, x, B: int, H_kv: int, T: int, pos0: int,
+               out: kvq_plane, stream=None):
+    _check(lib().kvq_encode(C.byref(codec), _ptr(signs), _ptr(x), B, H_kv, T, pos0,
+                            C.byref(out), _stream(stream)))
+
+
+def kvq_dequant(codec: kvq_codec, signs, plane: kvq_plane, B: int, H_kv: int, T: int,
+                pos0: int, y, stream=None):
+    _check(lib().kvq_dequant(C.byref(codec), _ptr(signs), C.byref(plane), B, H_kv, T, pos0,
+                             _ptr(y), _stream(stream)))
+
+
+def kvq_decode_num_splits(B: int, H_kv: int, max_ctx: int, sm_count: int) -> int:
+    return lib().kvq_decode_num_splits(B, H_kv, max_ctx, sm_count)
+
+
+def kvq_decode_workspace_bytes(B: int, H_q: int, head_dim: int, num_splits: int) -> int:
+    return lib().kvq_decode_workspace_bytes(B, H_q, head_dim, num_splits)
+
+
+def kvq_decode_attn(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: kvq_plane,
+                    V: kvq_plane, ctx_len, B: int, H_q: int, H_kv: int, max_ctx: int,
+                    softmax_scale: float, num_splits: int, workspace, ws_bytes: int, err_word,
+                    out, out_dtype: int, stream=None):
+    _check(lib().kvq_decode_attn(_ptr(q), C.byref(kc), C.byref(vc), _ptr(signs_k),
+                                 _ptr(signs_v), C.byref(K), C.byref(V), _ptr(ctx_len), B, H_q,
+                                 H_kv, max_ctx, softmax_scale, num_splits, _ptr(workspace),
+                                 ws_bytes, _ptr(err_word), _ptr(out), out_dtype,
+                                 _stream(stream)))
+
+
+# ------------------------------------------------------ torch-side helpers --
+
+def codec(head_dim: int, L: int, norm_mode: int) -> kvq_codec:
+    return kvq_codec(head_dim, L, norm_mode)
+
+
+@dataclass
+class Plane:
+    """Caller-owned device arrays of one compressed plane [B][H_kv][capacity][row]."""
+    codec: kvq_codec
+    B: int
+    H_kv: int
+    capacity: int
+    angles: object
+    norms: object
+    params: object
+
+    def c(self) -> kvq_plane:
+        return kvq_plane(self.angles.data_ptr(), self.norms.data_ptr(), self.params.data_ptr(),
+                         self.capacity)
+
+    def rows(self, which: int):
+        """uint8 view [B, H_kv, capacity, row_bytes] of one array."""
+        t = (self.angles, self.norms, self.params)[which]
+        return t.view(self.B, self.H_kv, self.capacity, -1)
+
+
+def alloc_plane(c: kvq_codec, B: int, H_kv: int, capacity: int, device="cuda") -> Plane:
+    import torch
+    if capacity % 16:
+        raise ValueError("capacity must be a multiple of 16")
+    n = B * H_kv * capacity
+    arrs = [torch.zeros(max(1, n * kvq_row_bytes(c, w)), dtype=torch.uint8, device=device)
+            for w in range(3)]
+    return Plane(c, B, H_kv, capacity, *arrs)
+
+
+def encode(c: kvq_codec, signs, x, plane: Plane, pos0: int = 0, stream=None):
+    """Encode x [B, H_kv, T, d] (fp16, contiguous) into plane tokens pos0.."""
+    B, H, T, d = x.shape
+    kvq_encode(c, signs, x, B, H, T, pos0, plane.c(), stream)
+
+
+def dequant(c: kvq_codec, signs, plane: Plane, T: int, pos0: int = 0, out=None, stream=None):
+    import torch
+    if out is None:
+        out = torch.empty((plane.B, plane.H_kv, T, c.head_dim), dtype=torch.float16,
+                          device=plane.angles.device)
+    kvq_dequant(c, signs, plane.c(), plane.B, plane.H_kv, T, pos0, out, stream)
+    return out
+
+
+class DecodeWorkspace:
+    """Scratch for kvq_decode_attn sized for (B, H_q, d, num_splits)."""
+
+    def __init__(self, B, H_q, d, num_splits, device="cuda"):
+        import torch
+        self.num_splits = num_splits
+        self.nbytes = kvq_decode_workspace_bytes(B, H_q, d, num_splits)
+        self.buf = torch.empty(max(16, self.nbytes), dtype=torch.uint8, device=device)
+
+
+def decode_attn(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: Plane, V: Plane,
+                ctx_len, max_ctx: int, softmax_scale: float | None = None, num_splits=None,
+                workspace: DecodeWorkspace | None = None, err_word=None, out=None,
+                out_dtype: int = OUT_FP32, stream=None):
+    import torch
+    B, H_q, d = q.shape
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    if num_splits is None:
+        sm = torch.cuda.get_device_properties(q.device).multi_processor_count
+        num_splits = kvq_decode_num_splits(B, K.H_kv, max_ctx, sm)
+    if workspace is None or workspace.num_splits != num_splits:
+        workspace = DecodeWorkspace(B, H_q, d, num_splits, q.device)
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float16 if out_dtype == OUT_FP16
+                          else torch.float32, device=q.device)
+    kvq_decode_attn(q, kc, vc, signs_k, signs_v, K.c(), V.c(), ctx_len, B, H_q, K.H_kv, max_ctx,
+                    softmax_scale, num_splits, workspace.buf, workspace.nbytes, err_word, out,
+                    out_dtype, stream)
+    return out

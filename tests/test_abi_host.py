@@ -1,0 +1,145 @@
+"""Host-side checks of libkvq.so that need no GPU: it builds for sm_100a, it
+loads, it exports every function include/kvq.h declares, its layout queries
+agree with the byte layout, and invalid arguments are rejected before any
+CUDA call (no compute call is made here)."""
+import ctypes as C
+import os
+
+import numpy as np
+import pytest
+
+from decode_attention_rand_b200 import build as kbuild
+from decode_attention_rand_b200 import kvq
+
+import oracle as O
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    kbuild.build()
+    return kvq.lib()
+
+
+def test_exports_every_declared_function():
+    names = kvq.header_functions()
+    assert {"kvq_encode", "kvq_dequant", "kvq_decode_attn", "kvq_last_error"} <= set(names)
+    L = C.CDLL(kvq.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    assert kvq.kvq_version() >= 10000
+
+
+def test_angle_bits_and_row_bytes_match_layout():
+    for L in [2, 3, 4, 5, 7, 8, 100, 128, 129, 255, 256, 4096, 65535, 65536]:
+        assert kvq.kvq_angle_bits(L) == O.angle_bits(L)
+    assert kvq.kvq_angle_bits(1) < 0 and kvq.kvq_angle_bits(65537) < 0
+    for d in [4, 8, 16, 32, 64, 128, 256]:
+        for L in [2, 3, 5, 32, 64, 128, 256, 1000, 65536]:
+            for mode in (kvq.KVQ_NORM_LIN8, kvq.KVQ_NORM_LOG4):
+                c = kvq.codec(d, L, mode)
+                for w in range(3):
+                    assert kvq.kvq_row_bytes(c, w) == O.row_bytes(d, L, mode, w)
+    assert kvq.kvq_row_bytes(kvq.codec(48, 16, 0), 0) < 0
+    assert kvq.kvq_row_bytes(kvq.codec(64, 16, 7), 1) < 0
+
+
+def test_split_heuristic():
+    for B, H, ctx, sm in [(1, 8, 4096, 148), (8, 8, 32768, 148), (4, 4, 65536, 148),
+                          (1, 2, 256, 148), (1, 1, 1, 148), (64, 8, 100, 148)]:
+        s = kvq.kvq_decode_num_splits(B, H, ctx, sm)
+        assert 1 <= s <= max(1, (ctx + 15) // 16)
+        assert s == kvq.kvq_decode_num_splits(B, H, ctx, sm)
+        assert B * H * s <= 2 * sm + B * H
+    assert kvq.kvq_decode_num_splits(0, 8, 100, 148) == 1
+    assert kvq.kvq_decode_workspace_bytes(2, 8, 128, 3) == 4 * (2 * 8 * 3 * 2 + 2 * 8 * 3 * 128)
+
+
+FAKE = 1 << 20  # 16-byte aligned non-NULL addresses; never dereferenced
+
+
+def _plane(cap=32, base=FAKE):
+    return kvq.kvq_plane(base, base + 4096, base + 8192, cap)
+
+
+@pytest.mark.parametrize("case", [
+    dict(codec=(100, 128, 0), msg="head_dim"),
+    dict(codec=(128, 1, 0), msg="L = 1"),
+    dict(codec=(128, 70000, 0), msg="L = 70000"),
+    dict(codec=(128, 128, 3), msg="norm_mode"),
+    dict(plane=kvq.kvq_plane(FAKE + 4, FAKE, FAKE, 32), msg="aligned"),
+    dict(plane=kvq.kvq_plane(FAKE, FAKE, FAKE, 40), msg="capacity"),
+    dict(plane=kvq.kvq_plane(0, FAKE, FAKE, 32), msg="NULL"),
+    dict(T=20, pos0=20, msg="exceed capacity"),
+    dict(T=-1, msg="negative"),
+    dict(x=FAKE + 2, msg="x must be 16-byte aligned"),
+])
+def test_encode_rejects_bad_arguments(case):
+    c = kvq.codec(*case.get("codec", (128, 128, 0)))
+    p = case.get("plane", _plane())
+    rc = kvq.lib().kvq_encode(C.byref(c), FAKE, case.get("x", FAKE), 1, 2, case.get("T", 4),
+                              case.get("pos0", 0), C.byref(p), None)
+    assert rc in (kvq.KVQ_EINVAL, kvq.KVQ_EUNSUPPORTED)
+    assert case["msg"] in kvq.kvq_last_error()
+
+
+def test_encode_and_dequant_empty_is_ok_without_gpu():
+    c = kvq.codec(128, 128, 0)
+    p = _plane()
+    assert kvq.lib().kvq_encode(C.byref(c), None, None, 0, 2, 4, 0, C.byref(p), None) == 0
+    assert kvq.lib().kvq_dequant(C.byref(c), None, C.byref(p), 1, 2, 0, 0, None, None) == 0
+    assert kvq.kvq_last_error() == ""
+
+
+def _decode_rc(**kw):
+    kc = kvq.codec(*kw.get("kc", (128, 128, 0)))
+    vc = kvq.codec(*kw.get("vc", (128, 64, 1)))
+    K, V = kw.get("K", _plane()), kw.get("V", _plane())
+    B, H_q, H_kv = kw.get("B", 1), kw.get("H_q", 8), kw.get("H_kv", 2)
+    S = kw.get("S", 2)
+    ws = kw.get("ws", kvq.kvq_decode_workspace_bytes(B, H_q, kc.head_dim, S))
+    return kvq.lib().kvq_decode_attn(FAKE, C.byref(kc), C.byref(vc), FAKE, FAKE, C.byref(K),
+                                     C.byref(V), FAKE, B, H_q, H_kv, kw.get("max_ctx", 32),
+                                     kw.get("scale", 0.1), S, kw.get("wsp", FAKE), ws, None,
+                                     FAKE, kw.get("out_dtype", 0), None)
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(H_q=6, H_kv=4), kvq.KVQ_EINVAL, "multiple"),
+    (dict(H_q=32, H_kv=2), kvq.KVQ_EUNSUPPORTED, "no kernel"),
+    (dict(kc=(32, 128, 0), vc=(32, 64, 1)), kvq.KVQ_EUNSUPPORTED, "no kernel"),
+    (dict(kc=(128, 512, 0)), kvq.KVQ_EUNSUPPORTED, "no kernel"),
+    (dict(vc=(64, 64, 1)), kvq.KVQ_EINVAL, "head_dim differ"),
+    (dict(V=_plane(48)), kvq.KVQ_EINVAL, "capacity differ"),
+    (dict(S=0), kvq.KVQ_EINVAL, "num_splits"),
+    (dict(ws=100), kvq.KVQ_EINVAL, "workspace"),
+    (dict(wsp=FAKE + 8), kvq.KVQ_EINVAL, "workspace not 16-byte"),
+    (dict(out_dtype=3), kvq.KVQ_EINVAL, "out_dtype"),
+    (dict(scale=float("nan")), kvq.KVQ_EINVAL, "softmax_scale"),
+    (dict(max_ctx=-1), kvq.KVQ_EINVAL, "negative"),
+])
+def test_decode_rejects_bad_arguments(kw, status, msg):
+    assert _decode_rc(**kw) == status
+    assert msg in kvq.kvq_last_error()
+
+
+def test_error_state_is_per_thread():
+    import threading
+    c = kvq.codec(128, 1, 0)
+    p = _plane()
+    kvq.lib().kvq_encode(C.byref(c), FAKE, FAKE, 1, 1, 1, 0, C.byref(p), None)
+    seen = {}
+
+    def other():
+        seen["msg"] = kvq.kvq_last_error()
+
+    t = threading.Thread(target=other)
+    t.start()
+    t.join()
+    assert seen["msg"] == "" and "L = 1" in kvq.kvq_last_error()
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(kvq, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(kvq, "_lib", None)
+    with pytest.raises(kvq.KvqError):
+        kvq.lib()
