@@ -247,7 +247,10 @@ def time_graph(state, K, W, dist_ctx):
     torch.cuda.synchronize()
     unit = max(1, min(K, state.nbuf * max(1, math.ceil(64 / state.nbuf))))
     n_full, rem = divmod(K, unit)
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+    # external events become event-record nodes of the graph, so each decode
+    # launch is timed inside the replay
+    evs = [[[torch.cuda.Event(enable_timing=True, external=True),
+             torch.cuda.Event(enable_timing=True, external=True)]
             for _ in state.layers] for _ in range(unit)]
     g_unit = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_unit, stream=stream):

@@ -125,18 +125,19 @@ __device__ __forceinline__ float half_bits_to_float(uint16_t h) {
     return __half2float(__ushort_as_half(h));
 }
 
-// fp16 round-to-nearest-even of a non-negative fp32 value, saturated to the
-// largest finite fp16 (the codec's parameter rule).
-__device__ __forceinline__ uint16_t f32_to_f16_sat(float x) {
-    uint16_t h = __half_as_ushort(__float2half_rn(x));
+// The codec's fp16 parameter rule: round to nearest even, saturate to the
+// largest finite fp16, store a zero as +0.
+__device__ __forceinline__ uint16_t f16_param_bits(uint16_t h) {
     if ((h & 0x7FFF) >= 0x7C00) h = (uint16_t)((h & 0x8000) | 0x7BFF);
-    return h;
+    return h == 0x8000 ? (uint16_t)0 : h;
+}
+
+__device__ __forceinline__ uint16_t f32_to_f16_sat(float x) {
+    return f16_param_bits(__half_as_ushort(__float2half_rn(x)));
 }
 
 __device__ __forceinline__ uint16_t f64_to_f16_sat(double x) {
-    uint16_t h = __half_as_ushort(__double2half(x));
-    if ((h & 0x7FFF) >= 0x7C00) h = (uint16_t)((h & 0x8000) | 0x7BFF);
-    return h;
+    return f16_param_bits(__half_as_ushort(__double2half(x)));
 }
 
 // True when |x| lies within tol of a midpoint between two adjacent finite

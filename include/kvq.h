@@ -68,7 +68,7 @@
  *   norms   LIN8: P bytes, byte i = c_i.
  *           LOG4: P/2 bytes, byte j = c_{2j} | c_{2j+1} << 4.
  *   params  LIN8: one IEEE fp16 M (2 bytes).  LOG4: fp16 LO then fp16 HI
- *           (4 bytes).
+ *           (4 bytes).  A zero parameter is stored as +0 (reading).
  * Requirements checked by every call: capacity % 16 == 0; every array
  * 16-byte aligned.  Token t of sequence (b, h) is row (b*H_kv + h)*capacity + t.
  *

@@ -184,9 +184,14 @@ static void bytes_to_words(const uint8_t* in, long nwords, uint32_t* words) {
     }
 }
 
+/* fp16 parameter: round to nearest even, saturate to the largest finite
+ * value, and store a zero as +0 (reading: the sign of a zero parameter
+ * carries no value, and for an exactly zero log-norm it would only echo the
+ * rounding of the fp64 logarithm). */
 static void put_half(uint8_t* dst, double v) {
     uint16_t h = double_to_half(v);
     if ((h & 0x7FFF) >= 0x7C00) h = (uint16_t)((h & 0x8000) | 0x7BFF); /* saturate */
+    if (h == 0x8000) h = 0; /* -0 -> +0 */
     dst[0] = (uint8_t)(h & 0xFF);
     dst[1] = (uint8_t)(h >> 8);
 }

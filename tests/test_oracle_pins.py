@@ -392,3 +392,16 @@ def test_attention_special_cases():
         assert np.allclose(o[0], vh[7], atol=1e-6 * np.abs(vh).max())
     # scores shift-invariance: adding a multiple of nothing; scaling tau by 0 gives mean
     assert np.allclose(O.attend(q, kh, vh, 0.0)[1], vh.mean(0), atol=1e-13)
+
+
+def test_zero_parameter_is_stored_as_plus_zero():
+    """A vector whose pair norms are all exactly 1 has log2 r = 0, so LO = HI = 0;
+    fp64 rounding of the logarithm can come out as -1.6e-16, and the stored
+    parameter must still be +0 (bits 0x0000), not -0."""
+    d = 128
+    x = np.zeros((1, d), np.float16)
+    x[0, 78] = 8.0  # r = 8 sqrt(2) / sqrt(128) = 1 for every pair
+    for seed in range(4):
+        s = _rand_signs(_rng(seed), d)
+        c = O.encode(x, s, 64, O.MODE_LOG4)
+        assert c.params[0].tolist() == [0, 0, 0, 0]
