@@ -169,7 +169,8 @@ int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx, int32_t 
 
 int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim, int32_t num_splits) {
     if (B < 0 || H_q < 0 || head_dim <= 0 || num_splits <= 0) return KVQ_EINVAL;
-    return (int64_t)sizeof(float) * (kvq::ws_stat_floats(B, H_q, num_splits) +
+    return (int64_t)sizeof(float) * (kvq::ws_counter_floats(B, H_q) +
+                                     kvq::ws_stat_floats(B, H_q, num_splits) +
                                      kvq::ws_acc_floats(B, H_q, num_splits, head_dim));
 }
 

@@ -26,10 +26,14 @@ struct DecodeArgs {
     float scale_log2;        // softmax_scale * log2(e)
     int num_splits;
     int64_t split_len;       // tokens per split, multiple of 16
-    float* ws;               // partials: [B][H_q][S] x (m, l) then acc [B][H_q][S][d]
+    float* ws;               // counters [B*H_q] int32, stats [B][H_q][S][2], acc [B][H_q][S][d]
     int32_t* err_word;
     void* out;
     int out_dtype;
+    // shared-memory staging layout, filled by the launcher
+    int lay[6];              // byte offsets of the six arrays inside a stage
+    int stage_bytes;
+    int stage_offset;
 };
 
 // True when the decode kernels are built for this (head_dim, G, L_K, L_V)
@@ -38,7 +42,12 @@ bool decode_supported(int d, int G, int LK, int LV, int mode_k, int mode_v);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
-// Workspace layout helpers (host and device agree through these).
+// Workspace layout helpers (host and device agree through these): completion
+// counters of the fused combine (int32, zero between calls), then per split
+// (m, l) pairs, then per split rotated-domain accumulators.
+__host__ __device__ inline int64_t ws_counter_floats(int B, int H_q) {
+    return ((int64_t)B * H_q + 3) / 4 * 4;
+}
 __host__ __device__ inline int64_t ws_stat_floats(int B, int H_q, int S) { return (int64_t)B * H_q * S * 2; }
 __host__ __device__ inline int64_t ws_acc_floats(int B, int H_q, int S, int d) { return (int64_t)B * H_q * S * d; }
 

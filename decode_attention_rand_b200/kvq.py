@@ -213,13 +213,14 @@ def dequant(c: kvq_codec, signs, plane: Plane, T: int, pos0: int = 0, out=None, 
 
 
 class DecodeWorkspace:
-    """Scratch for kvq_decode_attn sized for (B, H_q, d, num_splits)."""
+    """Scratch for kvq_decode_attn sized for (B, H_q, d, num_splits); zero-filled
+    once, as the C ABI requires before first use."""
 
     def __init__(self, B, H_q, d, num_splits, device="cuda"):
         import torch
         self.num_splits = num_splits
         self.nbytes = kvq_decode_workspace_bytes(B, H_q, d, num_splits)
-        self.buf = torch.empty(max(16, self.nbytes), dtype=torch.uint8, device=device)
+        self.buf = torch.zeros(max(16, self.nbytes), dtype=torch.uint8, device=device)
 
 
 def decode_attn(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: Plane, V: Plane,

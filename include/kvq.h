@@ -164,9 +164,10 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs,
 int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx,
                               int32_t sm_count);
 
-/* Workspace bytes kvq_decode_attn needs for `num_splits` splits: per
- * (b, query head, split) an fp32 running max, an fp32 softmax denominator
- * and an fp32 [head_dim] partial accumulator (rotated domain). */
+/* Workspace bytes kvq_decode_attn needs for `num_splits` splits: B*H_q int32
+ * completion counters (rounded up to 16 bytes), then per (b, query head,
+ * split) an fp32 running max and softmax denominator, then an fp32
+ * [head_dim] partial accumulator (rotated domain). */
 int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim,
                                    int32_t num_splits);
 
@@ -183,13 +184,16 @@ int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim,
  *   softmax_scale  tau
  *   num_splits >= 1 (kvq_decode_num_splits gives the default)
  *   workspace  device scratch of ws_bytes >= kvq_decode_workspace_bytes(),
- *              16-byte aligned; no initialisation needed; calls that share
- *              a workspace must be stream-ordered
+ *              16-byte aligned, zero-filled before its first use (every call
+ *              leaves its counters at zero again); calls that share a
+ *              workspace must be stream-ordered
  *   err_word   device int32 or NULL (see Errors)
  *   out        device [B][H_q][head_dim], fp16 (out_dtype 0) or fp32 (1);
  *              a sequence with ctx_len 0 gets zeros.
- * Two kernels run on `stream`: the split-K pass and the combine pass (merge
- * of the per-split softmax states, inverse FWHT, D_V / sqrt(d)). */
+ * One kernel runs on `stream`: each CTA handles one (split, KV head, batch
+ * entry); the last CTA of a (batch entry, KV head) to finish merges the
+ * per-split softmax states, applies the inverse FWHT and D_V / sqrt(d) and
+ * writes the output. */
 int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc,
                     const int8_t* signs_k, const int8_t* signs_v,
                     const kvq_plane* K, const kvq_plane* V,
