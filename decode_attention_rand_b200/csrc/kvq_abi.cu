@@ -154,17 +154,31 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs, const kvq_plane* in
 }
 
 int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx, int32_t sm_count) {
+    // One CTA runs per SM.  Pick the fewest waves whose split count keeps at
+    // least 90% of the CTA slots busy, with at least 128 tokens per split;
+    // otherwise the most balanced choice within 8 waves.
     if (B <= 0 || H_kv <= 0 || max_ctx <= 0 || sm_count <= 0) return 1;
     const int64_t units = (int64_t)B * H_kv;
-    const int64_t max_splits = (max_ctx + 15) / 16;
-    // about two waves of CTAs, and at least 64 tokens per split
-    int64_t s = (2LL * sm_count + units - 1) / units;
-    const int64_t by_len = (max_ctx + 63) / 64;
-    if (s > by_len) s = by_len;
-    if (s > max_splits) s = max_splits;
-    if (s > 65535) s = 65535;
-    if (s < 1) s = 1;
-    return (int32_t)s;
+    int64_t max_s = (max_ctx + 127) / 128;
+    if (max_s > 65535) max_s = 65535;
+    if (max_s < 1) max_s = 1;
+    int64_t best = 1;
+    double best_eff = -1.0;
+    for (int64_t w = 1; w <= 8; w++) {
+        int64_t s = w * sm_count / units;
+        if (s < 1) s = 1;
+        if (s > max_s) s = max_s;
+        const int64_t ctas = units * s;
+        const int64_t waves = (ctas + sm_count - 1) / sm_count;
+        const double eff = (double)ctas / (double)(waves * sm_count);
+        if (eff >= 0.9) return (int32_t)s;
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = s;
+        }
+        if (s == max_s) break;
+    }
+    return (int32_t)best;
 }
 
 int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim, int32_t num_splits) {

@@ -1,0 +1,775 @@
+// kvq_decode_impl.cuh - the split-K decode attention kernel (template), with
+// the split combine fused in.  Instantiated per (head_dim, G) in the
+// kvq_decode_d*_g*.cu files; dispatched from kvq_decode.cu.
+//
+// The cache is never dequantized ("OCTOPUS: Joint Triplet Quantization for KV
+// Cache via Octahedral Parametrization", "Why it matters": keys are rebuilt on
+// the fly inside attention).  With the rotation R = H D / sqrt(d) orthogonal,
+// q . k^ = (R q) . z^_K, so each query head is rotated once and every cached
+// token is scored in the rotated domain from its codes:
+//     s_t = tau * sum_i r^_i (q'[2i] cos theta^_i + q'[2i+1] sin theta^_i),
+// the softmax runs online, values are accumulated in the rotated domain
+// (acc = sum_t p_t z^_V,t) and one inverse rotation D_V H / sqrt(d) per head
+// finishes the output.  Codec: "TurboAngle: Near-Lossless KV Cache
+// Compression via Uniform Angle Quantization", Abstract (8-bit linear K
+// norms, 4-bit log-space V norms).
+//
+// One CTA per (split, KV head, batch entry):
+//   - thread 0 streams tiles of kTT tokens of the six code arrays (K/V
+//     angles, norms, params) into a 2..4-deep shared-memory ring with 1-D bulk
+//     asynchronous copies (TMA, no multicast), tracked by "full" mbarriers
+//     (transaction bytes) and recycled through "empty" mbarriers that every
+//     warp arrives on; a stage is refilled one tile after it was released,
+//     so the refill never waits on the warps still working; every wait is
+//     bounded, a timeout is reported in the error word and the kernel drains
+//     its copies and returns instead of trapping;
+//   - consumer warps take blocks of consecutive tokens; a group of NL lanes
+//     owns four tokens, each lane PP pairs of them and the matching pairs of
+//     all G query heads of the KV head (GQA), so every unpacked code serves G
+//     heads; partial scores meet in a transpose-reduce over the group, the
+//     softmax weights travel back the same way;
+//   - angle codes have compile-time widths (BK, BV in 5..8; 0 = runtime) so
+//     a code becomes a table offset in two integer operations; bin-centre
+//     cos/sin tables are replicated 16 times so a half-warp's 64-bit lookups
+//     never share a bank;
+//   - the online softmax rescales lazily, only when a score exceeds the
+//     running reference max by more than 2^8;
+//   - per-split partials (m, l, acc[d]) go to the workspace; the last CTA of a
+//     (batch, KV head) to finish (atomic counter, no waiting) merges the
+//     splits, divides by l, applies the inverse FWHT and D_V / sqrt(d).
+#pragma once
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+constexpr int kTT = 128;          // tokens per staged tile
+constexpr int kMaxStages = 4;     // ring depth (2..4, chosen per launch)
+constexpr int kTPG = 4;           // tokens per group chunk
+constexpr float kLazyThr = 8.f;   // log2 units
+constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr int kTabRep = 16;       // table replicas (one per half-warp lane)
+constexpr int kTabShift = 7;      // log2(kTabRep * sizeof(float2))
+
+template <int D, int G>
+struct DecCfg {
+    static constexpr int P = D / 2;
+    static constexpr int PP = (32 / G) > 16 ? 16 : (32 / G);  // pairs per lane
+    static constexpr int NL = P / PP;                          // lanes per token group
+    static constexpr int GPW = 32 / NL;                        // groups per warp
+    static constexpr int TW = GPW * kTPG;                      // tokens per warp block
+    static constexpr int WARPS = (kTT / TW) > 8 ? 8 : ((kTT / TW) < 2 ? 2 : (kTT / TW));
+    static constexpr int THREADS = WARPS * 32;
+    static constexpr int NG = WARPS * GPW;                     // groups per CTA
+    static constexpr int V = kTPG * G;                         // partial sums per lane
+    static constexpr int VF = V / NL;                          // final sums per lane
+    static_assert(VF >= 1, "group too wide");
+    static_assert(PP % 4 == 0, "codes are unpacked four at a time");
+    static_assert(kTT % (TW * WARPS) == 0, "blocks must tile the stage");
+};
+
+// --------------------------------------------------------------- PTX ----
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+        "selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0u;
+}
+
+// Bounded wait: false when the limit ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kWaitLimit; ++it)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+typedef unsigned long long f32x2;  // two packed fp32 lanes
+
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+    f32x2 v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+__device__ __forceinline__ float lo2(f32x2 v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi2(f32x2 v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// ------------------------------------------------------- group exchange --
+
+// Transpose-reduce over the NL lanes of a group: on return v[0..VF) holds the
+// group sums of entries lg*VF + e.
+template <int V, int NL>
+__device__ __forceinline__ void transpose_reduce(float (&v)[V], int lg) {
+#pragma unroll
+    for (int r = 0; (NL >> (r + 1)) >= 1; r++) {
+        const int o = NL >> (r + 1);
+        const int half = V >> (r + 1);
+        const bool upper = (lg & o) != 0;
+#pragma unroll
+        for (int i = 0; i < half; i++) {
+            const float send = upper ? v[i] : v[i + half];
+            const float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(KVQ_FULL_MASK, send, o);
+        }
+    }
+}
+
+// Inverse of transpose_reduce: from v[0..VF) (entries lg*VF + e) rebuild all
+// V entries in every lane of the group.
+template <int V, int NL>
+__device__ __forceinline__ void transpose_gather(float (&v)[V], int lg) {
+    constexpr int VF = V / NL;
+#pragma unroll
+    for (int r = 0; (1 << r) < NL; r++) {
+        const int o = 1 << r;
+        const int cur = VF << r;
+        const bool upper = (lg & o) != 0;
+#pragma unroll
+        for (int i = 0; i < cur; i++) {
+            const float mine = v[i];
+            const float other = __shfl_xor_sync(KVQ_FULL_MASK, mine, o);
+            v[i] = upper ? other : mine;
+            v[i + cur] = upper ? mine : other;
+        }
+    }
+}
+
+// Byte offsets (entry * 128 + lane16 * 8) into a 16x replicated float2
+// table for the PP angle codes of this lane: bits [cb, cb + PP*B) of a row.
+// B > 0: compile-time width; B == 0: runtime width `bits`.
+template <int PP, int B>
+__device__ __forceinline__ void angle_offsets(const uint32_t* row, int cb, int bits,
+                                              uint32_t lane_off, uint32_t (&off)[PP]) {
+    if constexpr (B > 0) {
+        constexpr int NB = PP * B;             // chunk bits
+        constexpr int NW = (NB + 31) / 32;     // normalised words
+        constexpr uint32_t mask = ((1u << B) - 1u) << kTabShift;
+        uint32_t n[NW + 1];
+        const int w0 = cb >> 5;
+        if constexpr (NB % 32 == 0) {
+#pragma unroll
+            for (int i = 0; i < NW; i++) n[i] = row[w0 + i];
+        } else {
+            const int sh = cb & 31;
+            uint32_t w[NW + 1];
+#pragma unroll
+            for (int i = 0; i <= NW; i++) w[i] = row[w0 + i];
+#pragma unroll
+            for (int i = 0; i < NW; i++) n[i] = __funnelshift_r(w[i], w[i + 1], sh);
+        }
+        n[NW] = 0u;
+#pragma unroll
+        for (int k = 0; k < PP; k++) {
+            constexpr int dummy = 0;
+            (void)dummy;
+            const int pos = k * B;             // compile-time after unrolling
+            const int wi = pos >> 5, bi = pos & 31;
+            uint32_t x;
+            if (bi + B <= 32) {
+                x = bi >= kTabShift ? (n[wi] >> (bi - kTabShift)) : (n[wi] << (kTabShift - bi));
+            } else {
+                x = __funnelshift_r(n[wi], n[wi + 1], bi - kTabShift);
+            }
+            off[k] = (x & mask) | lane_off;
+        }
+    } else {
+        const uint32_t mask = (1u << bits) - 1u;
+#pragma unroll
+        for (int q = 0; q < PP / 4; q++) {
+            const int pos = cb + q * 4 * bits;
+            const uint32_t win = __funnelshift_r(row[pos >> 5], row[(pos >> 5) + 1], pos & 31);
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+                off[4 * q + k] = (((win >> (k * bits)) & mask) << kTabShift) | lane_off;
+        }
+    }
+}
+
+template <int NBYTES>
+__device__ __forceinline__ void load_bytes(const uint8_t* p, uint32_t (&w)[(NBYTES + 3) / 4]) {
+    if constexpr (NBYTES == 16) {
+        const uint4 q = *reinterpret_cast<const uint4*>(p);
+        w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
+    } else if constexpr (NBYTES == 8) {
+        const uint2 q = *reinterpret_cast<const uint2*>(p);
+        w[0] = q.x; w[1] = q.y;
+    } else if constexpr (NBYTES == 4) {
+        w[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else {
+        w[0] = *reinterpret_cast<const uint16_t*>(p);
+    }
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t smem_addr) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(smem_addr));
+    return v;
+}
+
+// ------------------------------------------------------------- kernel ---
+
+template <int D, int G, int BK, int BV>
+__global__ void __launch_bounds__(DecCfg<D, G>::THREADS, 1)
+decode_kernel(DecodeArgs A) {
+    using Cfg = DecCfg<D, G>;
+    constexpr int P = Cfg::P, PP = Cfg::PP, NL = Cfg::NL, GPW = Cfg::GPW, NG = Cfg::NG;
+    constexpr int WARPS = Cfg::WARPS, TW = Cfg::TW;
+    constexpr int V = Cfg::V, VF = Cfg::VF;
+    constexpr int EPQ = D / 32;
+    constexpr int CONSUMERS = WARPS * 32;
+
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int NST = A.nstages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);           // [kMaxStages]
+    uint64_t* empty = full + kMaxStages;                          // [kMaxStages]
+    int* sflag = reinterpret_cast<int*>(smem + 16 * kMaxStages);  // timeout, last
+    const int nK = 1 << A.kc.bits, nV = 1 << A.vc.bits;
+    float2* tabK = reinterpret_cast<float2*>(smem + 16 * kMaxStages + 16);  // [2^bK][16]
+    float2* tabV = tabK + nK * kTabRep;                           // [2^bV][16]
+    float* qs = reinterpret_cast<float*>(tabV + nV * kTabRep);    // [G][D]
+    unsigned char* stages = smem + A.stage_offset;                // [kStages][stage]
+
+    const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // ---- token range of this split -----------------------------------------
+    int64_t ctx = A.ctx_len[b];
+    const int64_t lim = A.max_ctx < A.K.capacity ? A.max_ctx : A.K.capacity;
+    if (ctx < 0 || ctx > lim) {
+        if (split == 0 && kvh == 0 && tid == 0) report(A.err_word, KVQ_DEVERR_CTX_RANGE);
+        ctx = ctx < 0 ? 0 : lim;
+    }
+    const int64_t t0 = (int64_t)split * A.split_len;
+    const int64_t t1 = (t0 + A.split_len < ctx) ? t0 + A.split_len : ctx;
+    const int ntiles = t1 > t0 ? (int)((t1 - t0 + kTT - 1) / kTT) : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < NST; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], WARPS);
+        }
+        mbar_fence_init();
+        sflag[0] = 0;
+        sflag[1] = 0;
+    }
+    __syncthreads();
+
+    // ---- producer lane: the first NST tiles go out before the prologue ------
+    const int64_t row0 = ((int64_t)b * A.H_kv + kvh) * A.K.capacity;
+    int issued = 0;  // tiles issued (producer lane 0)
+    auto issue_tile = [&](int tile) {
+        const int rbK = A.kc.angle_words * 4, rbV = A.vc.angle_words * 4;
+        const uint8_t* srcs[6] = {A.K.angles + row0 * rbK, A.K.norms + row0 * A.kc.norm_bytes,
+                                  A.K.params + row0 * A.kc.param_bytes, A.V.angles + row0 * rbV,
+                                  A.V.norms + row0 * A.vc.norm_bytes,
+                                  A.V.params + row0 * A.vc.param_bytes};
+        const int rbs[6] = {rbK, A.kc.norm_bytes, A.kc.param_bytes, rbV, A.vc.norm_bytes,
+                            A.vc.param_bytes};
+        const int s = tile % NST;
+        const int64_t tt0 = t0 + (int64_t)tile * kTT;
+        const int64_t left = t1 - tt0;
+        const int n16 = (int)(((left < kTT ? left : kTT) + 15) / 16 * 16);
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int k = 0; k < 6; k++) bytes += (uint32_t)(n16 * rbs[k]);
+        fence_proxy_async();
+        mbar_expect_tx(&full[s], bytes);
+        unsigned char* dst = stages + (size_t)s * A.stage_bytes;
+#pragma unroll
+        for (int k = 0; k < 6; k++)
+            bulk_g2s(dst + A.lay[k], srcs[k] + tt0 * rbs[k], (uint32_t)(n16 * rbs[k]), &full[s]);
+    };
+    // tile t + NST - 1 is issued once tile t - 1 is released, so NST - 1 tiles
+    // are in flight ahead of the one being consumed
+    if (tid == 0)
+        for (; issued < NST - 1 && issued < ntiles; issued++) issue_tile(issued);
+
+    // ---- everyone: tables and q' (overlaps the first copies) -----------------
+    for (int j = tid; j < nK; j += CONSUMERS) {
+        float s, c;
+        sincospif((float)(2 * j + 1) / (float)A.kc.L - 1.f, &s, &c);
+#pragma unroll
+        for (int r = 0; r < kTabRep; r++) tabK[j * kTabRep + r] = make_float2(c, s);
+    }
+    for (int j = tid; j < nV; j += CONSUMERS) {
+        float s, c;
+        sincospif((float)(2 * j + 1) / (float)A.vc.L - 1.f, &s, &c);
+#pragma unroll
+        for (int r = 0; r < kTabRep; r++) tabV[j * kTabRep + r] = make_float2(c, s);
+    }
+    for (int h = warp; h < G; h += WARPS) {
+        const __half* qh = A.q + ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * D;
+        float v[EPQ];
+#pragma unroll
+        for (int e = 0; e < EPQ; e++) {
+            const int j = lane * EPQ + e;
+            const float f = __half2float(qh[j]);
+            v[e] = A.signs_k[j] < 0 ? -f : f;
+        }
+        fwht_local<EPQ>(v);
+        fwht_cross<EPQ, 32>(v, lane);
+        const float isd = rsqrtf((float)D);
+#pragma unroll
+        for (int e = 0; e < EPQ; e++) qs[h * D + lane * EPQ + e] = v[e] * isd;
+    }
+    __syncthreads();
+
+    const int grp = lane / NL, lg = lane % NL;
+    const int gidx = warp * GPW + grp;
+    f32x2 acc[G][PP];
+    float mref[G];
+    float lpart[VF];
+#pragma unroll
+    for (int h = 0; h < G; h++) {
+        mref[h] = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < PP; k++) acc[h][k] = 0ull;
+    }
+#pragma unroll
+    for (int e = 0; e < VF; e++) lpart[e] = 0.f;
+
+    {
+        f32x2 q2[G][PP];
+#pragma unroll
+        for (int h = 0; h < G; h++)
+#pragma unroll
+            for (int k = 0; k < PP; k++) {
+                const float2 qq = reinterpret_cast<const float2*>(qs + h * D)[lg * PP + k];
+                q2[h][k] = pack2(qq.x, qq.y);
+            }
+        const int bitsK = BK > 0 ? BK : A.kc.bits, bitsV = BV > 0 ? BV : A.vc.bits;
+        const int cbK = lg * PP * bitsK, cbV = lg * PP * bitsV;
+        const uint32_t lane_off = (uint32_t)(lane & 15) * 8u;
+        const uint32_t tK = smem_u32(tabK), tV = smem_u32(tabV);
+        const int awK = A.kc.angle_words, awV = A.vc.angle_words;
+
+        for (int tile = 0; tile < ntiles; tile++) {
+            const int s = tile % NST;
+            const bool got = mbar_wait_bounded(&full[s], (uint32_t)(tile / NST) & 1u);
+            if (!__all_sync(KVQ_FULL_MASK, got)) {
+                if (lane == 0) atomicOr(&sflag[0], 1);
+                break;
+            }
+            if (__any_sync(KVQ_FULL_MASK, *((volatile int*)&sflag[0]) != 0)) break;
+            const unsigned char* st = stages + (size_t)s * A.stage_bytes;
+            const uint32_t* sKa = reinterpret_cast<const uint32_t*>(st + A.lay[0]);
+            const uint8_t* sKn = st + A.lay[1];
+            const uint16_t* sKp = reinterpret_cast<const uint16_t*>(st + A.lay[2]);
+            const uint32_t* sVa = reinterpret_cast<const uint32_t*>(st + A.lay[3]);
+            const uint8_t* sVn = st + A.lay[4];
+            const uint32_t* sVp = reinterpret_cast<const uint32_t*>(st + A.lay[5]);
+            const int64_t tt0 = t0 + (int64_t)tile * kTT;
+            const int ntok = (int)((t1 - tt0) < kTT ? (t1 - tt0) : kTT);
+
+            for (int blk = warp; blk < kTT / TW; blk += WARPS) {
+                // token of slot j of this group: consecutive rows across the warp
+                // -- scores: partial dot products of this lane's pairs --------
+                float part[V];
+#pragma unroll
+                for (int j = 0; j < kTPG; j++) {
+                    const int t = blk * TW + j * GPW + grp;
+                    uint32_t off[PP];
+                    angle_offsets<PP, BK>(sKa + t * awK, cbK, bitsK, lane_off, off);
+                    uint32_t nw[(PP + 3) / 4];
+                    load_bytes<PP>(sKn + t * P + lg * PP, nw);
+                    f32x2 dot[G];
+#pragma unroll
+                    for (int h = 0; h < G; h++) dot[h] = 0ull;
+#pragma unroll
+                    for (int k = 0; k < PP; k++) {
+                        const float cf = (float)((nw[k / 4] >> (8 * (k % 4))) & 0xFFu);
+                        const float2 cs = lds_f2(tK + off[k]);
+                        const f32x2 xy = pack2(cf * cs.x, cf * cs.y);
+#pragma unroll
+                        for (int h = 0; h < G; h++) dot[h] = fma2(q2[h][k], xy, dot[h]);
+                    }
+#pragma unroll
+                    for (int h = 0; h < G; h++) part[j * G + h] = lo2(dot[h]) + hi2(dot[h]);
+                }
+                transpose_reduce<V, NL>(part, lg);
+                // -- scale by M/255 * tau * log2(e), mask, lazy softmax reference
+                bool need = false;
+#pragma unroll
+                for (int e = 0; e < VF; e++) {
+                    const int idx = lg * VF + e;
+                    const int j = idx / G, h = idx % G;
+                    const int t = blk * TW + j * GPW + grp;
+                    const float M = half_bits_to_float(sKp[t]);
+                    float sv = part[e] * (M * (1.f / 255.f)) * A.scale_log2;
+                    sv = t < ntok ? sv : -INFINITY;
+                    part[e] = sv;
+                    float mh = mref[0];
+#pragma unroll
+                    for (int hh = 1; hh < G; hh++) mh = (hh == h) ? mref[hh] : mh;
+                    need |= sv > mh + kLazyThr;
+                }
+                if (__any_sync(KVQ_FULL_MASK, need)) {
+                    float mx[G];
+#pragma unroll
+                    for (int h = 0; h < G; h++) mx[h] = -INFINITY;
+#pragma unroll
+                    for (int e = 0; e < VF; e++) {
+                        const int h = (lg * VF + e) % G;
+#pragma unroll
+                        for (int hh = 0; hh < G; hh++)
+                            if (hh == h) mx[hh] = fmaxf(mx[hh], part[e]);
+                    }
+#pragma unroll
+                    for (int h = 0; h < G; h++) {
+                        mx[h] = group_max<NL>(mx[h]);
+                        const float mn = fmaxf(mref[h], mx[h]);
+                        const float al = (mn == -INFINITY) ? 0.f : ex2(mref[h] - mn);
+                        const f32x2 al2 = pack2(al, al);
+#pragma unroll
+                        for (int k = 0; k < PP; k++) acc[h][k] = mul2(acc[h][k], al2);
+#pragma unroll
+                        for (int e = 0; e < VF; e++)
+                            if ((lg * VF + e) % G == h) lpart[e] *= al;
+                        mref[h] = mn;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < VF; e++) {
+                    const int h = (lg * VF + e) % G;
+                    float mh = mref[0];
+#pragma unroll
+                    for (int hh = 1; hh < G; hh++) mh = (hh == h) ? mref[hh] : mh;
+                    const float p = part[e] == -INFINITY ? 0.f : ex2(part[e] - mh);
+                    part[e] = p;
+                    lpart[e] += p;
+                }
+                transpose_gather<V, NL>(part, lg);
+                // -- values: acc[h] += p[t][h] * r^ (cos, sin), rotated domain --
+#pragma unroll
+                for (int j = 0; j < kTPG; j++) {
+                    const int t = blk * TW + j * GPW + grp;
+                    uint32_t off[PP];
+                    angle_offsets<PP, BV>(sVa + t * awV, cbV, bitsV, lane_off, off);
+                    uint32_t nw[(PP / 2 + 3) / 4];
+                    load_bytes<PP / 2>(sVn + t * (P / 2) + lg * (PP / 2), nw);
+                    const uint32_t pr = sVp[t];
+                    float LO = half_bits_to_float((uint16_t)(pr & 0xFFFF));
+                    float step = (half_bits_to_float((uint16_t)(pr >> 16)) - LO) * (1.f / 15.f);
+                    // rows past the context hold stale bytes: make their r^ finite
+                    // (their softmax weight is already 0)
+                    LO = t < ntok ? LO : -64.f;
+                    step = t < ntok ? step : 0.f;
+                    f32x2 pw[G];
+#pragma unroll
+                    for (int h = 0; h < G; h++) pw[h] = pack2(part[j * G + h], part[j * G + h]);
+#pragma unroll
+                    for (int k = 0; k < PP; k++) {
+                        const float cf = (float)((nw[k / 8] >> (4 * (k % 8))) & 0xFu);
+                        const float r = ex2(fmaf(cf, step, LO));
+                        const float2 cs = lds_f2(tV + off[k]);
+                        const f32x2 xy = pack2(r * cs.x, r * cs.y);
+#pragma unroll
+                        for (int h = 0; h < G; h++) acc[h][k] = fma2(pw[h], xy, acc[h][k]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            // refill: tile + NST - 1 goes into the stage tile - 1 used, once every
+            // warp has released it (normally already true)
+            if (tid == 0 && issued < ntiles && issued == tile + NST - 1) {
+                const int nxt = issued;
+                const int sn = nxt % NST;
+                bool ok = true;
+                if (nxt >= NST) ok = mbar_wait_bounded(&empty[sn], (uint32_t)((nxt / NST) - 1) & 1u);
+                if (ok) {
+                    issue_tile(nxt);
+                    issued = nxt + 1;
+                } else {
+                    atomicOr(&sflag[0], 1);
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (sflag[0]) {
+        // a wait ran out: report, then wait (bounded) for the copies still in
+        // flight before the shared memory is released; this CTA contributes
+        // nothing to the output
+        if (tid == 0) {
+            report(A.err_word, KVQ_DEVERR_TIMEOUT);
+            // the newest tile of each stage covers the older ones
+            for (int t = issued - NST > 0 ? issued - NST : 0; t < issued; t++)
+                (void)mbar_wait_bounded(&full[t % NST], (uint32_t)(t / NST) & 1u);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int h = 0; h < G; h++) {
+            mref[h] = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < PP; k++) acc[h][k] = 0ull;
+        }
+#pragma unroll
+        for (int e = 0; e < VF; e++) lpart[e] = 0.f;
+    }
+
+    // ---- merge the NG group states of this CTA (reuses the stage memory) --
+    float* gm = reinterpret_cast<float*>(stages);  // [NG][G]
+    float* gl = gm + NG * G;                      // [NG][G]
+    float* gacc = gl + NG * G;                    // [NG][G][D]
+    {
+        float lh[G];
+#pragma unroll
+        for (int h = 0; h < G; h++) lh[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < VF; e++) {
+            const int h = (lg * VF + e) % G;
+#pragma unroll
+            for (int hh = 0; hh < G; hh++)
+                if (hh == h) lh[hh] += lpart[e];
+        }
+#pragma unroll
+        for (int h = 0; h < G; h++) lh[h] = group_sum<NL>(lh[h]);
+        if (lg == 0) {
+#pragma unroll
+            for (int h = 0; h < G; h++) {
+                gm[gidx * G + h] = mref[h];
+                gl[gidx * G + h] = lh[h];
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < G; h++)
+#pragma unroll
+            for (int k = 0; k < PP; k++) {
+                const int i = lg * PP + k;
+                reinterpret_cast<float2*>(gacc + (gidx * G + h) * D)[i] =
+                    make_float2(lo2(acc[h][k]), hi2(acc[h][k]));
+            }
+    }
+    __syncthreads();
+
+    const int S = A.num_splits;
+    float* stats = A.ws + ws_counter_floats(A.B, A.H_q);
+    float* accs = stats + ws_stat_floats(A.B, A.H_q, S);
+    for (int idx = tid; idx < G * D; idx += CONSUMERS) {
+        const int h = idx / D, j = idx % D;
+        float mx = -INFINITY;
+        for (int g = 0; g < NG; g++) mx = fmaxf(mx, gm[g * G + h]);
+        float sum_l = 0.f, sum_a = 0.f;
+        if (mx != -INFINITY) {
+            for (int g = 0; g < NG; g++) {
+                const float w = ex2(gm[g * G + h] - mx);
+                sum_l += w * gl[g * G + h];
+                sum_a += w * gacc[(g * G + h) * D + j];
+            }
+        }
+        const int64_t slot = ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * S + split;
+        accs[slot * D + j] = sum_a;
+        if (j == 0) {
+            stats[slot * 2] = mx;
+            stats[slot * 2 + 1] = sum_l;
+        }
+    }
+
+    // ---- the last CTA of this (b, KV head) merges the splits ----------------
+    __threadfence();
+    __syncthreads();
+    int* counters = reinterpret_cast<int*>(A.ws);
+    if (tid == 0) {
+        const int prev = atomicAdd(&counters[b * A.H_kv + kvh], 1);
+        sflag[1] = (prev == S - 1);
+    }
+    __syncthreads();
+    if (!sflag[1]) return;
+    __threadfence();
+    constexpr int ALLW = WARPS;
+    constexpr int ALLT = CONSUMERS;
+    float* hm = gm;          // [G] reuse of the merge scratch
+    float* hl = gm + G;      // [G]
+    float* vo = gm + 2 * G;  // [G][D]
+    // pass 1 (one warp per head): the common max and the softmax denominator
+    for (int h = warp; h < G; h += ALLW) {
+        const int64_t hq = (int64_t)b * A.H_q + (int64_t)kvh * G + h;
+        const float* stp = stats + hq * S * 2;
+        float mx = -INFINITY;
+        for (int s = lane; s < S; s += 32) mx = fmaxf(mx, __ldcg(stp + 2 * s));
+        mx = group_max<32>(mx);
+        float sl = 0.f;
+        if (mx != -INFINITY)
+            for (int s = lane; s < S; s += 32) sl += ex2(__ldcg(stp + 2 * s) - mx) * __ldcg(stp + 2 * s + 1);
+        sl = group_sum<32>(sl);
+        if (lane == 0) {
+            hm[h] = mx;
+            hl[h] = sl;
+        }
+    }
+    __syncthreads();
+    // pass 2 (one thread per output element): weighted sum over the splits
+    for (int idx = tid; idx < G * D; idx += ALLT) {
+        const int h = idx / D, j = idx % D;
+        const int64_t hq = (int64_t)b * A.H_q + (int64_t)kvh * G + h;
+        const float* stp = stats + hq * S * 2;
+        const float* ac = accs + hq * S * D + j;
+        const float mx = hm[h];
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        if (mx != -INFINITY) {
+            int s = 0;
+            for (; s + 4 <= S; s += 4) {
+                const float m0 = __ldcg(stp + 2 * s), m1 = __ldcg(stp + 2 * s + 2);
+                const float m2 = __ldcg(stp + 2 * s + 4), m3 = __ldcg(stp + 2 * s + 6);
+                const float x0 = __ldcg(ac + (int64_t)s * D), x1 = __ldcg(ac + (int64_t)(s + 1) * D);
+                const float x2 = __ldcg(ac + (int64_t)(s + 2) * D), x3 = __ldcg(ac + (int64_t)(s + 3) * D);
+                a0 = fmaf(ex2(m0 - mx), x0, a0);
+                a1 = fmaf(ex2(m1 - mx), x1, a1);
+                a2 = fmaf(ex2(m2 - mx), x2, a2);
+                a3 = fmaf(ex2(m3 - mx), x3, a3);
+            }
+            for (; s < S; s++) a0 = fmaf(ex2(__ldcg(stp + 2 * s) - mx), __ldcg(ac + (int64_t)s * D), a0);
+        }
+        const float l = hl[h];
+        vo[h * D + j] = l > 0.f ? ((a0 + a1) + (a2 + a3)) / l : 0.f;
+    }
+    __syncthreads();
+    // pass 3 (one warp per head): inverse FWHT, D_V / sqrt(d), store
+    for (int h = warp; h < G; h += ALLW) {
+        const int64_t hq = (int64_t)b * A.H_q + (int64_t)kvh * G + h;
+        float v[EPQ];
+#pragma unroll
+        for (int e = 0; e < EPQ; e++) v[e] = vo[h * D + lane * EPQ + e];
+        fwht_local<EPQ>(v);
+        fwht_cross<EPQ, 32>(v, lane);
+        const float isd = rsqrtf((float)D);
+#pragma unroll
+        for (int e = 0; e < EPQ; e++) {
+            const int j = lane * EPQ + e;
+            float o = v[e] * isd;
+            o = A.signs_v[j] < 0 ? -o : o;
+            if (A.out_dtype == 0)
+                reinterpret_cast<__half*>(A.out)[hq * D + j] = __float2half_rn(o);
+            else
+                reinterpret_cast<float*>(A.out)[hq * D + j] = o;
+        }
+    }
+    if (tid == 0) atomicExch(&counters[b * A.H_kv + kvh], 0);
+}
+
+// ------------------------------------------------------------------ host --
+
+// Shared-memory plan of one launch (ring depth 4, 3 or 2, whichever fits);
+// returns 0 bytes when even two stages do not fit.
+template <int D, int G>
+inline size_t decode_smem_plan(DecodeArgs& a) {
+    using Cfg = DecCfg<D, G>;
+    size_t off = 16 * kMaxStages + 16 +
+                 sizeof(float2) * kTabRep * (size_t)((1 << a.kc.bits) + (1 << a.vc.bits)) +
+                 sizeof(float) * G * D;
+    off = (off + 15) / 16 * 16;
+    a.stage_offset = (int)off;
+    const int rb[6] = {a.kc.angle_words * 4, a.kc.norm_bytes, a.kc.param_bytes,
+                       a.vc.angle_words * 4, a.vc.norm_bytes, a.vc.param_bytes};
+    int sb = 0;
+    for (int k = 0; k < 6; k++) {
+        a.lay[k] = sb;
+        // +16: the last row's code window may read one word past its region
+        sb += (kTT * rb[k] + 16 + 15) / 16 * 16;
+    }
+    a.stage_bytes = sb;
+    const size_t merge = sizeof(float) * ((size_t)2 * Cfg::NG * G + (size_t)Cfg::NG * G * D);
+    for (int ns = kMaxStages; ns >= 2; ns--) {
+        size_t ring = (size_t)ns * sb;
+        if (ring < merge) ring = merge;
+        if (off + ring <= 227 * 1024) {
+            a.nstages = ns;
+            return off + ring;
+        }
+    }
+    return 0;
+}
+
+template <int D, int G, int BK, int BV>
+inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
+    using Cfg = DecCfg<D, G>;
+    const size_t smem = decode_smem_plan<D, G>(a);
+    if (smem == 0) return cudaErrorInvalidConfiguration;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        e = cudaFuncSetAttribute(decode_kernel<D, G, BK, BV>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = true;
+    }
+    dim3 grid((unsigned)a.num_splits, (unsigned)a.H_kv, (unsigned)a.B);
+    decode_kernel<D, G, BK, BV><<<grid, Cfg::THREADS, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+// Fast kernels for code widths 5..8 (codebooks of 17..256 entries), the
+// runtime-width kernel for anything else.
+template <int D, int G>
+inline cudaError_t launch_decode_dg(const DecodeArgs& a, cudaStream_t stream) {
+    const int bk = a.kc.bits, bv = a.vc.bits;
+#define KVQ_BB(X, Y) \
+    if (bk == X && bv == Y) return launch_decode_kernel<D, G, X, Y>(a, stream);
+    KVQ_BB(5, 5) KVQ_BB(5, 6) KVQ_BB(5, 7) KVQ_BB(5, 8)
+    KVQ_BB(6, 5) KVQ_BB(6, 6) KVQ_BB(6, 7) KVQ_BB(6, 8)
+    KVQ_BB(7, 5) KVQ_BB(7, 6) KVQ_BB(7, 7) KVQ_BB(7, 8)
+    KVQ_BB(8, 5) KVQ_BB(8, 6) KVQ_BB(8, 7) KVQ_BB(8, 8)
+#undef KVQ_BB
+    return launch_decode_kernel<D, G, 0, 0>(a, stream);
+}
+
+}  // namespace kvq

@@ -34,6 +34,7 @@ struct DecodeArgs {
     int lay[6];              // byte offsets of the six arrays inside a stage
     int stage_bytes;
     int stage_offset;
+    int nstages;             // ring depth
 };
 
 // True when the decode kernels are built for this (head_dim, G, L_K, L_V)
@@ -41,6 +42,14 @@ struct DecodeArgs {
 bool decode_supported(int d, int G, int LK, int LV, int mode_k, int mode_v);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_d64_g1(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_d64_g2(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_d64_g4(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_d64_g8(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_d128_g1(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_d128_g2(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_d128_g4(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_d128_g8(const DecodeArgs& a, cudaStream_t stream);
 
 // Workspace layout helpers (host and device agree through these): completion
 // counters of the fused combine (int32, zero between calls), then per split

@@ -47,9 +47,14 @@ def test_split_heuristic():
     for B, H, ctx, sm in [(1, 8, 4096, 148), (8, 8, 32768, 148), (4, 4, 65536, 148),
                           (1, 2, 256, 148), (1, 1, 1, 148), (64, 8, 100, 148)]:
         s = kvq.kvq_decode_num_splits(B, H, ctx, sm)
-        assert 1 <= s <= max(1, (ctx + 15) // 16)
+        assert 1 <= s <= max(1, (ctx + 127) // 128)
         assert s == kvq.kvq_decode_num_splits(B, H, ctx, sm)
-        assert B * H * s <= 2 * sm + B * H
+        assert B * H * s <= 8 * sm + B * H
+    # wave quantisation: the chosen split count fills at least 90% of the slots
+    for B, H, ctx in [(8, 8, 32768), (4, 4, 65536), (1, 8, 4096)]:
+        s = kvq.kvq_decode_num_splits(B, H, ctx, 148)
+        ctas = B * H * s
+        assert ctas / (-(-ctas // 148) * 148) >= 0.9, (B, H, ctx, s)
     assert kvq.kvq_decode_num_splits(0, 8, 100, 148) == 1
     # counters (B*H_q int32, rounded to 16 bytes), (m, l) per split, acc per split
     assert kvq.kvq_decode_workspace_bytes(2, 8, 128, 3) == 4 * (16 + 2 * 8 * 3 * 2 + 2 * 8 * 3 * 128)
