@@ -79,6 +79,10 @@ int cuda_status(cudaError_t e, const char* what) {
 
 }  // namespace
 
+namespace kvq {
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace kvq
+
 extern "C" {
 
 int32_t kvq_version(void) { return 1 * 10000 + 0 * 100 + 0; }

@@ -51,6 +51,9 @@ cudaError_t launch_decode_d128_g2(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d128_g4(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d128_g8(const DecodeArgs& a, cudaStream_t stream);
 
+// Set the calling thread's kvq_last_error() message; returns `code`.
+int record_error(int code, const char* msg);
+
 // Workspace layout helpers (host and device agree through these): completion
 // counters of the fused combine (int32, zero between calls), then per split
 // (m, l) pairs, then per split rotated-domain accumulators.

@@ -56,6 +56,11 @@ _SIGNATURES = {
                               C.c_int32, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]),
     "kvq_decode_num_splits": (C.c_int32, [C.c_int32, C.c_int32, C.c_int64, C.c_int32]),
     "kvq_decode_workspace_bytes": (C.c_int64, [C.c_int32, C.c_int32, C.c_int32, C.c_int32]),
+    "kvq_decode_attn_noalloc": (C.c_int, [C.c_void_p, C.POINTER(kvq_codec), C.POINTER(kvq_codec),
+                                          C.c_void_p, C.c_void_p, C.POINTER(kvq_plane),
+                                          C.POINTER(kvq_plane), C.c_void_p, C.c_int32, C.c_int32,
+                                          C.c_int32, C.c_int64, C.c_float, C.c_int32, C.c_void_p,
+                                          C.c_void_p, C.c_int32, C.c_void_p]),
     "kvq_decode_attn": (C.c_int, [C.c_void_p, C.POINTER(kvq_codec), C.POINTER(kvq_codec),
                                   C.c_void_p, C.c_void_p, C.POINTER(kvq_plane),
                                   C.POINTER(kvq_plane), C.c_void_p, C.c_int32, C.c_int32,
@@ -158,6 +163,18 @@ def kvq_decode_attn(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: kvq_pl
                                  H_kv, max_ctx, softmax_scale, num_splits, _ptr(workspace),
                                  ws_bytes, _ptr(err_word), _ptr(out), out_dtype,
                                  _stream(stream)))
+
+
+def kvq_decode_attn_noalloc(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: kvq_plane,
+                            V: kvq_plane, ctx_len, B: int, H_q: int, H_kv: int, max_ctx: int,
+                            softmax_scale: float, num_splits: int, err_word, out, out_dtype: int,
+                            stream=None):
+    """kvq_decode_attn with the library's built-in scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    _check(lib().kvq_decode_attn_noalloc(_ptr(q), C.byref(kc), C.byref(vc), _ptr(signs_k),
+                                         _ptr(signs_v), C.byref(K), C.byref(V), _ptr(ctx_len), B,
+                                         H_q, H_kv, max_ctx, softmax_scale, num_splits,
+                                         _ptr(err_word), _ptr(out), out_dtype, _stream(stream)))
 
 
 # ------------------------------------------------------ torch-side helpers --

@@ -203,6 +203,34 @@ int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc,
                     int32_t* err_word, void* out, int32_t out_dtype,
                     void* stream);
 
+/* Size of the scratch array built into the library for
+ * kvq_decode_attn_noalloc (4 MiB of device memory per GPU that loads it). */
+#define KVQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* kvq_decode_attn without a workspace argument, for callers that cannot
+ * allocate device memory: a serving loop whose device memory all belongs to
+ * its own pooling allocator, a plain C program with no allocator, or code
+ * that must not risk the synchronisation or out-of-memory failure of a fresh
+ * cudaMalloc.  (The TurboAngle page has no counterpart: this is a library
+ * convenience.)  Arguments and results are those of kvq_decode_attn; the
+ * scratch comes from a KVQ_NOALLOC_SCRATCH_BYTES array compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  A call whose kvq_decode_workspace_bytes() exceeds that size returns
+ * KVQ_EINVAL before any launch (fewer splits reduce it).  The first call on a
+ * device looks up the array's device address (with that device current):
+ * make it before any stream capture.  Each call first clears the completion
+ * counters with an asynchronous memset on `stream`; the call allocates
+ * nothing.  All calls share the one array, so calls whose kernels overlap on
+ * the GPU race on it and must be ordered by the caller. */
+int kvq_decode_attn_noalloc(const void* q, const kvq_codec* kc,
+                            const kvq_codec* vc, const int8_t* signs_k,
+                            const int8_t* signs_v, const kvq_plane* K,
+                            const kvq_plane* V, const int32_t* ctx_len,
+                            int32_t B, int32_t H_q, int32_t H_kv,
+                            int64_t max_ctx, float softmax_scale,
+                            int32_t num_splits, int32_t* err_word, void* out,
+                            int32_t out_dtype, void* stream);
+
 /* Message for the last non-OK status returned on the calling thread
  * (empty string if none).  The pointer stays valid until the next call on
  * the same thread. */
