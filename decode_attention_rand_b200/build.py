@@ -25,7 +25,7 @@ FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std
 
 
 def _deps_mtime() -> float:
-    files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
+    files = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if not f.endswith(".py")]
     files.append(os.path.join(ROOT, "include", "kvq.h"))
     files.append(os.path.abspath(__file__))
     return max(os.path.getmtime(f) for f in files)

@@ -10,7 +10,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/kvq.h"
+#include "kvq.h"  // include/ is on the include path
 
 #define KVQ_FULL_MASK 0xffffffffu
 

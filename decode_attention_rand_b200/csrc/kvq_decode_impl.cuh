@@ -288,15 +288,13 @@ decode_kernel(DecodeArgs A) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // ---- token range of this split -----------------------------------------
-    int64_t ctx = A.ctx_len[b];
+    // Copies start before ctx_len is known: they cover the split up to the
+    // host bound min(max_ctx, capacity); tokens past ctx_len[b] are masked.
     const int64_t lim = A.max_ctx < A.K.capacity ? A.max_ctx : A.K.capacity;
-    if (ctx < 0 || ctx > lim) {
-        if (split == 0 && kvh == 0 && tid == 0) report(A.err_word, KVQ_DEVERR_CTX_RANGE);
-        ctx = ctx < 0 ? 0 : lim;
-    }
     const int64_t t0 = (int64_t)split * A.split_len;
-    const int64_t t1 = (t0 + A.split_len < ctx) ? t0 + A.split_len : ctx;
-    const int ntiles = t1 > t0 ? (int)((t1 - t0 + kTT - 1) / kTT) : 0;
+    const int64_t t1m = (t0 + A.split_len < lim) ? t0 + A.split_len : lim;
+    const int ntiles_max = t1m > t0 ? (int)((t1m - t0 + kTT - 1) / kTT) : 0;
+    const int64_t ctx_in = A.ctx_len[b];
 
     if (tid == 0) {
         for (int s = 0; s < NST; s++) {
@@ -322,7 +320,7 @@ decode_kernel(DecodeArgs A) {
                             A.vc.param_bytes};
         const int s = tile % NST;
         const int64_t tt0 = t0 + (int64_t)tile * kTT;
-        const int64_t left = t1 - tt0;
+        const int64_t left = t1m - tt0;
         const int n16 = (int)(((left < kTT ? left : kTT) + 15) / 16 * 16);
         uint32_t bytes = 0;
 #pragma unroll
@@ -337,20 +335,22 @@ decode_kernel(DecodeArgs A) {
     // tile t + NST - 1 is issued once tile t - 1 is released, so NST - 1 tiles
     // are in flight ahead of the one being consumed
     if (tid == 0)
-        for (; issued < NST - 1 && issued < ntiles; issued++) issue_tile(issued);
+        for (; issued < NST - 1 && issued < ntiles_max; issued++) issue_tile(issued);
 
     // ---- everyone: tables and q' (overlaps the first copies) -----------------
-    for (int j = tid; j < nK; j += CONSUMERS) {
+    // consecutive threads write consecutive replicas (no bank conflicts); the
+    // 16 threads of an entry compute the same value in the same instruction
+#pragma unroll 1
+    for (int idx = tid; idx < nK * kTabRep; idx += CONSUMERS) {
         float s, c;
-        sincospif((float)(2 * j + 1) / (float)A.kc.L - 1.f, &s, &c);
-#pragma unroll
-        for (int r = 0; r < kTabRep; r++) tabK[j * kTabRep + r] = make_float2(c, s);
+        sincospif((float)(2 * (idx / kTabRep) + 1) / (float)A.kc.L - 1.f, &s, &c);
+        tabK[idx] = make_float2(c, s);
     }
-    for (int j = tid; j < nV; j += CONSUMERS) {
+#pragma unroll 1
+    for (int idx = tid; idx < nV * kTabRep; idx += CONSUMERS) {
         float s, c;
-        sincospif((float)(2 * j + 1) / (float)A.vc.L - 1.f, &s, &c);
-#pragma unroll
-        for (int r = 0; r < kTabRep; r++) tabV[j * kTabRep + r] = make_float2(c, s);
+        sincospif((float)(2 * (idx / kTabRep) + 1) / (float)A.vc.L - 1.f, &s, &c);
+        tabV[idx] = make_float2(c, s);
     }
     for (int h = warp; h < G; h += WARPS) {
         const __half* qh = A.q + ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * D;
@@ -364,9 +364,25 @@ decode_kernel(DecodeArgs A) {
         fwht_local<EPQ>(v);
         fwht_cross<EPQ, 32>(v, lane);
         const float isd = rsqrtf((float)D);
+        if constexpr (EPQ == 4) {
+            reinterpret_cast<float4*>(qs + h * D)[lane] =
+                make_float4(v[0] * isd, v[1] * isd, v[2] * isd, v[3] * isd);
+        } else {
 #pragma unroll
-        for (int e = 0; e < EPQ; e++) qs[h * D + lane * EPQ + e] = v[e] * isd;
+            for (int e = 0; e < EPQ; e++) qs[h * D + lane * EPQ + e] = v[e] * isd;
+        }
     }
+    int64_t ctx = ctx_in;
+    if (ctx < 0 || ctx > lim) {
+        if (split == 0 && kvh == 0 && tid == 0) report(A.err_word, KVQ_DEVERR_CTX_RANGE);
+        ctx = ctx < 0 ? 0 : lim;
+    }
+    const int64_t t1 = t1m < ctx ? t1m : ctx;
+    const int ntiles = t1 > t0 ? (int)((t1 - t0 + kTT - 1) / kTT) : 0;
+    // every issued tile is consumed (tiles past the context are fully masked)
+    const int nloop = ntiles > (NST - 1 < ntiles_max ? NST - 1 : ntiles_max)
+                          ? ntiles
+                          : (NST - 1 < ntiles_max ? NST - 1 : ntiles_max);
     __syncthreads();
 
     const int grp = lane / NL, lg = lane % NL;
@@ -398,7 +414,7 @@ decode_kernel(DecodeArgs A) {
         const uint32_t tK = smem_u32(tabK), tV = smem_u32(tabV);
         const int awK = A.kc.angle_words, awV = A.vc.angle_words;
 
-        for (int tile = 0; tile < ntiles; tile++) {
+        for (int tile = 0; tile < nloop; tile++) {
             const int s = tile % NST;
             const bool got = mbar_wait_bounded(&full[s], (uint32_t)(tile / NST) & 1u);
             if (!__all_sync(KVQ_FULL_MASK, got)) {
@@ -416,7 +432,7 @@ decode_kernel(DecodeArgs A) {
             const int64_t tt0 = t0 + (int64_t)tile * kTT;
             const int ntok = (int)((t1 - tt0) < kTT ? (t1 - tt0) : kTT);
 
-            for (int blk = warp; blk < kTT / TW; blk += WARPS) {
+            for (int blk = warp; blk * TW < ntok; blk += WARPS) {
                 // token of slot j of this group: consecutive rows across the warp
                 // -- scores: partial dot products of this lane's pairs --------
                 float part[V];
@@ -527,7 +543,7 @@ decode_kernel(DecodeArgs A) {
             if (lane == 0) mbar_arrive(&empty[s]);
             // refill: tile + NST - 1 goes into the stage tile - 1 used, once every
             // warp has released it (normally already true)
-            if (tid == 0 && issued < ntiles && issued == tile + NST - 1) {
+            if (tid == 0 && issued < nloop && issued == tile + NST - 1) {
                 const int nxt = issued;
                 const int sn = nxt % NST;
                 bool ok = true;
@@ -565,9 +581,14 @@ decode_kernel(DecodeArgs A) {
     }
 
     // ---- merge the NG group states of this CTA (reuses the stage memory) --
-    float* gm = reinterpret_cast<float*>(stages);  // [NG][G]
-    float* gl = gm + NG * G;                      // [NG][G]
-    float* gacc = gl + NG * G;                    // [NG][G][D]
+    // accumulators as [G][PP][NG * 2 NL + pad]: a warp writes one (h, k) row
+    // segment of 32 consecutive float2 (no bank conflicts), and the pad puts
+    // the next k row on the other half of the banks for the summing pass
+    constexpr int ROW = NG * 2 * NL + 16;
+    float* gm = reinterpret_cast<float*>(stages);  // [NG][G]  running maxima
+    float* gl = gm + NG * G;                      // [NG][G]  denominators, then weights
+    float* gacc = gl + NG * G;                    // [G][PP][ROW]
+    float* hml = gacc + G * PP * ROW;             // [G][2]   CTA max and denominator
     {
         float lh[G];
 #pragma unroll
@@ -591,34 +612,52 @@ decode_kernel(DecodeArgs A) {
 #pragma unroll
         for (int h = 0; h < G; h++)
 #pragma unroll
-            for (int k = 0; k < PP; k++) {
-                const int i = lg * PP + k;
-                reinterpret_cast<float2*>(gacc + (gidx * G + h) * D)[i] =
+            for (int k = 0; k < PP; k++)
+                reinterpret_cast<float2*>(gacc + (h * PP + k) * ROW)[gidx * NL + lg] =
                     make_float2(lo2(acc[h][k]), hi2(acc[h][k]));
-            }
+    }
+    __syncthreads();
+    // per head: the CTA max, each group's weight 2^(m_g - max), the denominator
+    for (int h = warp; h < G; h += WARPS) {
+        float mx = -INFINITY;
+        for (int g = lane; g < NG; g += 32) mx = fmaxf(mx, gm[g * G + h]);
+        mx = group_max<32>(mx);
+        float sl = 0.f;
+        for (int g = lane; g < NG; g += 32) {
+            const float w = mx == -INFINITY ? 0.f : ex2(gm[g * G + h] - mx);
+            sl += w * gl[g * G + h];
+            gl[g * G + h] = w;
+        }
+        sl = group_sum<32>(sl);
+        if (lane == 0) {
+            hml[2 * h] = mx;
+            hml[2 * h + 1] = sl;
+        }
     }
     __syncthreads();
 
     const int S = A.num_splits;
     float* stats = A.ws + ws_counter_floats(A.B, A.H_q);
     float* accs = stats + ws_stat_floats(A.B, A.H_q, S);
+    // thread -> (h, k, lg, c) with (lg, c) fastest: consecutive threads read
+    // consecutive floats of a row; element j = 2 (lg PP + k) + c
     for (int idx = tid; idx < G * D; idx += CONSUMERS) {
-        const int h = idx / D, j = idx % D;
-        float mx = -INFINITY;
-        for (int g = 0; g < NG; g++) mx = fmaxf(mx, gm[g * G + h]);
-        float sum_l = 0.f, sum_a = 0.f;
-        if (mx != -INFINITY) {
-            for (int g = 0; g < NG; g++) {
-                const float w = ex2(gm[g * G + h] - mx);
-                sum_l += w * gl[g * G + h];
-                sum_a += w * gacc[(g * G + h) * D + j];
-            }
+        const int lc = idx % (2 * NL), hk = idx / (2 * NL);
+        const int h = hk / PP, k = hk % PP;
+        const int j = 2 * ((lc >> 1) * PP + k) + (lc & 1);
+        const float* row = gacc + hk * ROW + lc;
+        float a0 = 0.f, a1 = 0.f;
+        int g = 0;
+        for (; g + 2 <= NG; g += 2) {
+            a0 = fmaf(gl[g * G + h], row[g * 2 * NL], a0);
+            a1 = fmaf(gl[(g + 1) * G + h], row[(g + 1) * 2 * NL], a1);
         }
+        for (; g < NG; g++) a0 = fmaf(gl[g * G + h], row[g * 2 * NL], a0);
         const int64_t slot = ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * S + split;
-        accs[slot * D + j] = sum_a;
+        accs[slot * D + j] = a0 + a1;
         if (j == 0) {
-            stats[slot * 2] = mx;
-            stats[slot * 2 + 1] = sum_l;
+            stats[slot * 2] = hml[2 * h];
+            stats[slot * 2 + 1] = hml[2 * h + 1];
         }
     }
 
@@ -633,60 +672,53 @@ decode_kernel(DecodeArgs A) {
     __syncthreads();
     if (!sflag[1]) return;
     __threadfence();
-    constexpr int ALLW = WARPS;
-    constexpr int ALLT = CONSUMERS;
-    float* hm = gm;          // [G] reuse of the merge scratch
-    float* hl = gm + G;      // [G]
-    float* vo = gm + 2 * G;  // [G][D]
-    // pass 1 (one warp per head): the common max and the softmax denominator
-    for (int h = warp; h < G; h += ALLW) {
+    // one warp per head: the common max and denominator over the splits (lane
+    // s holds split s), the weighted sum of the split accumulators, the inverse
+    // FWHT, D_V / sqrt(d), the store
+    for (int h = warp; h < G; h += WARPS) {
         const int64_t hq = (int64_t)b * A.H_q + (int64_t)kvh * G + h;
         const float* stp = stats + hq * S * 2;
+        const float* ac = accs + hq * S * D + lane * EPQ;
         float mx = -INFINITY;
         for (int s = lane; s < S; s += 32) mx = fmaxf(mx, __ldcg(stp + 2 * s));
         mx = group_max<32>(mx);
         float sl = 0.f;
-        if (mx != -INFINITY)
-            for (int s = lane; s < S; s += 32) sl += ex2(__ldcg(stp + 2 * s) - mx) * __ldcg(stp + 2 * s + 1);
-        sl = group_sum<32>(sl);
-        if (lane == 0) {
-            hm[h] = mx;
-            hl[h] = sl;
-        }
-    }
-    __syncthreads();
-    // pass 2 (one thread per output element): weighted sum over the splits
-    for (int idx = tid; idx < G * D; idx += ALLT) {
-        const int h = idx / D, j = idx % D;
-        const int64_t hq = (int64_t)b * A.H_q + (int64_t)kvh * G + h;
-        const float* stp = stats + hq * S * 2;
-        const float* ac = accs + hq * S * D + j;
-        const float mx = hm[h];
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        if (mx != -INFINITY) {
-            int s = 0;
-            for (; s + 4 <= S; s += 4) {
-                const float m0 = __ldcg(stp + 2 * s), m1 = __ldcg(stp + 2 * s + 2);
-                const float m2 = __ldcg(stp + 2 * s + 4), m3 = __ldcg(stp + 2 * s + 6);
-                const float x0 = __ldcg(ac + (int64_t)s * D), x1 = __ldcg(ac + (int64_t)(s + 1) * D);
-                const float x2 = __ldcg(ac + (int64_t)(s + 2) * D), x3 = __ldcg(ac + (int64_t)(s + 3) * D);
-                a0 = fmaf(ex2(m0 - mx), x0, a0);
-                a1 = fmaf(ex2(m1 - mx), x1, a1);
-                a2 = fmaf(ex2(m2 - mx), x2, a2);
-                a3 = fmaf(ex2(m3 - mx), x3, a3);
-            }
-            for (; s < S; s++) a0 = fmaf(ex2(__ldcg(stp + 2 * s) - mx), __ldcg(ac + (int64_t)s * D), a0);
-        }
-        const float l = hl[h];
-        vo[h * D + j] = l > 0.f ? ((a0 + a1) + (a2 + a3)) / l : 0.f;
-    }
-    __syncthreads();
-    // pass 3 (one warp per head): inverse FWHT, D_V / sqrt(d), store
-    for (int h = warp; h < G; h += ALLW) {
-        const int64_t hq = (int64_t)b * A.H_q + (int64_t)kvh * G + h;
         float v[EPQ];
 #pragma unroll
-        for (int e = 0; e < EPQ; e++) v[e] = vo[h * D + lane * EPQ + e];
+        for (int e = 0; e < EPQ; e++) v[e] = 0.f;
+        if (mx != -INFINITY) {
+            for (int c0 = 0; c0 < S; c0 += 32) {
+                const int s_l = c0 + lane;
+                const float w_l = s_l < S ? ex2(__ldcg(stp + 2 * s_l) - mx) : 0.f;
+                sl += s_l < S ? w_l * __ldcg(stp + 2 * s_l + 1) : 0.f;
+                const int n = S - c0 < 32 ? S - c0 : 32;
+                if constexpr (EPQ == 4) {
+#pragma unroll 8
+                    for (int k = 0; k < n; k++) {
+                        const float w = __shfl_sync(KVQ_FULL_MASK, w_l, k);
+                        const float4 x =
+                            __ldcg(reinterpret_cast<const float4*>(ac + (int64_t)(c0 + k) * D));
+                        v[0] = fmaf(w, x.x, v[0]);
+                        v[1] = fmaf(w, x.y, v[1]);
+                        v[2] = fmaf(w, x.z, v[2]);
+                        v[3] = fmaf(w, x.w, v[3]);
+                    }
+                } else {
+#pragma unroll 8
+                    for (int k = 0; k < n; k++) {
+                        const float w = __shfl_sync(KVQ_FULL_MASK, w_l, k);
+                        const float2 x =
+                            __ldcg(reinterpret_cast<const float2*>(ac + (int64_t)(c0 + k) * D));
+                        v[0] = fmaf(w, x.x, v[0]);
+                        v[1] = fmaf(w, x.y, v[1]);
+                    }
+                }
+            }
+        }
+        sl = group_sum<32>(sl);
+        const float inv = sl > 0.f ? 1.f / sl : 0.f;
+#pragma unroll
+        for (int e = 0; e < EPQ; e++) v[e] *= inv;
         fwht_local<EPQ>(v);
         fwht_cross<EPQ, 32>(v, lane);
         const float isd = rsqrtf((float)D);
@@ -725,7 +757,9 @@ inline size_t decode_smem_plan(DecodeArgs& a) {
         sb += (kTT * rb[k] + 16 + 15) / 16 * 16;
     }
     a.stage_bytes = sb;
-    const size_t merge = sizeof(float) * ((size_t)2 * Cfg::NG * G + (size_t)Cfg::NG * G * D);
+    const size_t merge =
+        sizeof(float) * ((size_t)2 * Cfg::NG * G +
+                         (size_t)G * Cfg::PP * (Cfg::NG * 2 * Cfg::NL + 16) + 2 * (size_t)G);
     for (int ns = kMaxStages; ns >= 2; ns--) {
         size_t ring = (size_t)ns * sb;
         if (ring < merge) ring = merge;

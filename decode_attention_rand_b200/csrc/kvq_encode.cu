@@ -5,26 +5,31 @@
 //
 // Layout of the work: one head vector per group of NL = d/EPL lanes, each
 // lane holding EPL (<= 16) consecutive elements, loaded with 128-bit loads.
-// The Walsh-Hadamard transform runs in registers (log2 EPL stages) and
+// The Walsh-Hadamard transform runs in registers (log2 EPL stages, packed
+// two butterflies per f32x2 instruction from the second stage on) and
 // across the group with shuffles (log2 NL stages).
 //
 // Exactness.  Codes must equal the definition's exactly except within a hair
-// of a decision edge.  The fast path works in fp32 and carries a rigorous
-// error bound for every quantity that feeds a decision:
+// of a decision edge.  The fast path works in fp32 and carries an error bound
+// for every quantity that feeds a decision:
 //   - FWHT: every butterfly rounds once, so after S stages each output is
 //     within S * 2^-24 * |x|_1 of the exact value (|x|_1 = L1 norm of the
 //     input), the classical bound for a +-1 butterfly network;
-//   - sqrt and division are correctly rounded (IEEE, no fast-math);
-//     atan2f is documented to 3 ulp and log2f to 1 ulp; the margins below
-//     allow several times that.
+//   - the angle comes from an octant reduction and an odd polynomial for
+//     atan on [0, 1] (kvq_atan_poly.h, fitted to 3.7e-8 rad); with the
+//     approximate reciprocal, fp32 coefficients and Horner rounding its error
+//     stays far below the 1.5e-6 rad the margin allows;
+//   - sqrt, reciprocal and log2 use the hardware approximations
+//     (sqrt/rcp/lg2.approx, documented to about 2^-22 relative or absolute),
+//     budgeted at several times that.
 // Any decision (angle bin, norm code, fp16 parameter) whose fp32 value lies
 // within its error bound of the edge sends the whole warp through an exact
 // path: the transform is recomputed in fp64, where it is exact (fp16 inputs
 // are integer multiples of 2^-24 below 2^16, so all partial sums over d <= 256
 // terms fit in 53 bits), and the flagged decisions are re-taken in fp64 with
-// the definition's own formula.  The remaining disagreement with any other
-// exact implementation is confined to values within an fp64 rounding of an
-// edge.
+// the definition's own formulas.  What remains open is a value within an
+// fp64 rounding of an edge.
+#include "kvq_atan_poly.h"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -41,6 +46,7 @@ struct EncCfg {
 
 constexpr int kEncWarps = 8;
 constexpr int kEncStageWords = 128;  // max VPW * angle_words over all D, b <= 16
+constexpr float kAngleSlack = 1.5e-6f;  // rad: polynomial, reciprocal, constants, rounding
 
 struct EncArgs {
     const __half* x;
@@ -54,12 +60,83 @@ struct EncArgs {
     float bins_per_rad;  // L / (2 pi)
 };
 
-__device__ __forceinline__ int exact_angle_code(double u, double v, int L) {
+// ------------------------------------------------------------ fp32 math --
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float y;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk(float lo, float hi) {
+    f32x2 v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+__device__ __forceinline__ float plo(f32x2 v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float phi(f32x2 v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// atan2(y, x) for (x, y) != (0, 0): octant reduction to t in [0, 1] and the
+// fitted odd polynomial.  Same conventions as atan2 on the axes.
+__device__ __forceinline__ float atan2_poly(float y, float x) {
+    const float ax = fabsf(x), ay = fabsf(y);
+    const float mx = fmaxf(ax, ay), mn = fminf(ax, ay);
+    const float t = mn * rcp_approx(mx);
+    const float t2 = t * t;
+    static_assert(KVQ_ATAN_NCOEF == 8, "Horner chain below has eight terms");
+    float p = fmaf(KVQ_ATAN_C7, t2, KVQ_ATAN_C6);
+    p = fmaf(p, t2, KVQ_ATAN_C5);
+    p = fmaf(p, t2, KVQ_ATAN_C4);
+    p = fmaf(p, t2, KVQ_ATAN_C3);
+    p = fmaf(p, t2, KVQ_ATAN_C2);
+    p = fmaf(p, t2, KVQ_ATAN_C1);
+    p = fmaf(p, t2, KVQ_ATAN_C0);
+    float th = p * t;
+    th = ay > ax ? 1.5707963267948966f - th : th;
+    th = x < 0.f ? kPiF - th : th;
+    return y < 0.f ? -th : th;
+}
+
+// ------------------------------------------------ exact (fp64) decisions --
+
+__device__ __noinline__ int exact_angle_code(double u, double v, int L) {
     if (u == 0.0 && v == 0.0) return 0;
     const double theta = atan2(v, u);
     const double t = (theta + kPi) * (double)L / (2.0 * kPi);
     return (int)floor(t) % L;
 }
+
+__device__ __noinline__ double exact_norm(double u, double v, double sqrt_d) {
+    return hypot(u / sqrt_d, v / sqrt_d);
+}
+
+__device__ __noinline__ double exact_log2(double r) { return log2(fmax(r, 5.9604644775390625e-8)); }
 
 __device__ __forceinline__ int lin8_code_exact(double r, double M) {
     if (M == 0.0) return 0;
@@ -78,6 +155,7 @@ __global__ void __launch_bounds__(kEncWarps * 32)
 encode_kernel(EncArgs A) {
     using Cfg = EncCfg<D>;
     constexpr int EPL = Cfg::EPL, NL = Cfg::NL, PPL = Cfg::PPL, VPW = Cfg::VPW;
+    constexpr int NW = EPL / 2;  // packed pairs per lane (= PPL)
     __shared__ uint32_t stage[kEncWarps][kEncStageWords];
 
     const int lane = threadIdx.x & 31;
@@ -92,10 +170,13 @@ encode_kernel(EncArgs A) {
     uint32_t* st = stage[warp];
     for (int i = lane; i < kEncStageWords; i += 32) st[i] = 0u;
 
-    // signs of this lane's elements (bit e set: negate element lg*EPL + e)
-    uint32_t negmask = 0;
+    // fp16 sign-bit masks of this lane's elements (element pairs per word)
+    uint32_t smask[NW];
 #pragma unroll
-    for (int e = 0; e < EPL; e++) negmask |= (A.signs[lg * EPL + e] < 0 ? 1u : 0u) << e;
+    for (int w = 0; w < NW; w++) {
+        const int e = lg * EPL + 2 * w;
+        smask[w] = (A.signs[e] < 0 ? 0x8000u : 0u) | (A.signs[e + 1] < 0 ? 0x80000000u : 0u);
+    }
 
     const double sqrt_d = sqrt((double)D);
     const float ez_scale = (float)Cfg::S * 5.9604645e-8f * 1.0001f;  // S * 2^-24, padded
@@ -106,8 +187,8 @@ encode_kernel(EncArgs A) {
         const int64_t v = wt * VPW + grp;
         const bool valid = v < A.n_vec;
 
-        // ---- load EPL fp16 values (128-bit loads) ----------------------
-        uint32_t raw[EPL / 2];
+        // ---- load EPL fp16 values (128-bit loads), apply D -------------
+        uint32_t raw[NW];
         {
             const __half* src = A.x + (valid ? v : 0) * D + lg * EPL;
             if constexpr (EPL == 16) {
@@ -122,83 +203,95 @@ encode_kernel(EncArgs A) {
                 const uint2 q0 = reinterpret_cast<const uint2*>(src)[0];
                 raw[0] = q0.x; raw[1] = q0.y;
             }
-            if (!valid) {
 #pragma unroll
-                for (int i = 0; i < EPL / 2; i++) raw[i] = 0u;
-            }
+            for (int w = 0; w < NW; w++) raw[w] = valid ? (raw[w] ^ smask[w]) : 0u;
         }
 
-        // ---- D x in fp32 (exact), L1 norm, FWHT --------------------------
-        float z[EPL];
+        // ---- fp32 (exact), L1 norm, FWHT ----------------------------------
+        f32x2 W[NW];  // W[k] = (z[2k], z[2k+1])
         float l1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < EPL; e++) {
-            const uint16_t hb = (uint16_t)(raw[e / 2] >> (16 * (e & 1)));
-            float f = half_bits_to_float(hb);
-            f = ((negmask >> e) & 1u) ? -f : f;
-            z[e] = f;
-            l1 += fabsf(f);
+        for (int w = 0; w < NW; w++) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&raw[w]));
+            l1 += fabsf(f.x) + fabsf(f.y);
+            W[w] = pk(f.x + f.y, f.x - f.y);  // first stage (h = 1) inside the pair
+        }
+#pragma unroll
+        for (int h = 1; h < NW; h <<= 1) {  // stages h = 2, 4, 8 on packed pairs
+#pragma unroll
+            for (int k = 0; k < NW; k++) {
+                if ((k & h) == 0) {
+                    const f32x2 a = W[k], b = W[k + h];
+                    W[k] = add2(a, b);
+                    W[k + h] = sub2(a, b);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 1; m < NL; m <<= 1) {  // cross-lane stages: v' = s * v + o
+            const float sg = (lg & m) ? -1.f : 1.f;
+            const f32x2 s2 = pk(sg, sg);
+#pragma unroll
+            for (int k = 0; k < NW; k++) {
+                const float o0 = __shfl_xor_sync(KVQ_FULL_MASK, plo(W[k]), m);
+                const float o1 = __shfl_xor_sync(KVQ_FULL_MASK, phi(W[k]), m);
+                W[k] = fma2(s2, W[k], pk(o0, o1));
+            }
         }
         l1 = group_sum<NL>(l1);
-        fwht_local<EPL>(z);
-        fwht_cross<EPL, NL>(z, lg);
         const float Ez = ez_scale * l1;  // bound on |z_fp32 - z_exact| (unscaled)
+        const float ezr = 1.5f * Ez * A.inv_sqrt_d;
 
         // ---- per pair: angle code and norm, with margins -------------------
         int acode[PPL];
         float rr[PPL];
-        float er[PPL];
         uint32_t need_a = 0, need_n = 0;
 #pragma unroll
         for (int i = 0; i < PPL; i++) {
-            const float x = z[2 * i], y = z[2 * i + 1];
-            const float rho = sqrtf(fmaf(x, x, y * y));
+            const float x = plo(W[i]), y = phi(W[i]);
+            const float rho = sqrt_approx(fmaf(x, x, y * y));
             int a = 0;
             if (!(rho > 4.f * Ez) || rho == 0.f) {
                 need_a |= 1u << i;
             } else {
-                const float th = atan2f(y, x);
-                const float u = (th + kPiF) * A.bins_per_rad;
+                const float th = atan2_poly(y, x);
+                const float u = fmaf(th, A.bins_per_rad, kPiF * A.bins_per_rad);
                 const float fl = floorf(u);
                 const float fr = u - fl;
-                const float dth = 2.f * Ez / (rho - 2.f * Ez);
-                const float du = A.bins_per_rad * (4.5e-6f + dth) + Lf * 1.2e-7f;
+                const float dth = 2.2f * Ez * rcp_approx(rho - 2.f * Ez);
+                const float du = A.bins_per_rad * (kAngleSlack + dth) + Lf * 2.4e-7f;
                 if (fr < du || fr > 1.f - du) need_a |= 1u << i;
                 a = (int)fl;
                 a = a >= L ? a - L : (a < 0 ? a + L : a);
             }
             acode[i] = a;
             rr[i] = rho * A.inv_sqrt_d;
-            er[i] = 1.5f * Ez * A.inv_sqrt_d + rr[i] * 4e-7f;
         }
 
         int ncode[PPL];
-        uint32_t prm = 0;    // packed fp16 parameter(s)
+        uint32_t prm = 0;     // packed fp16 parameter(s)
         bool need_p = false;  // group-uniform
         if (A.c.mode == KVQ_NORM_LIN8) {
             float m = 0.f;
 #pragma unroll
             for (int i = 0; i < PPL; i++) m = fmaxf(m, rr[i]);
             m = group_max<NL>(m);
-            const float eM = 1.5f * Ez * A.inv_sqrt_d + m * 4e-7f;
+            const float eM = ezr + m * 1e-6f;
             need_p = near_f16_midpoint(m, eM);
             const uint16_t Mh = f32_to_f16_sat(m);
             const float Mf = half_bits_to_float(Mh);
             prm = Mh;
-            const float inv = Mf > 0.f ? 255.f / Mf : 0.f;
+            const float inv = Mf > 0.f ? 255.f * rcp_approx(Mf) : 0.f;
+            const float dvc = ezr * inv * 1.01f + 2e-6f;
 #pragma unroll
             for (int i = 0; i < PPL; i++) {
-                int cc = 0;
-                if (Mf > 0.f) {
-                    const float vq = rr[i] * inv;
-                    const float t = vq + 0.5f;
-                    const float fl = floorf(t);
-                    const float fr = t - fl;
-                    const float dv = er[i] * inv * 1.0001f + vq * 2.5e-7f + 1e-6f;
-                    if (fr < dv || fr > 1.f - dv) need_n |= 1u << i;
-                    cc = min(255, (int)fl);
-                }
-                ncode[i] = cc;
+                const float vq = rr[i] * inv;
+                const float t = vq + 0.5f;
+                const float fl = floorf(t);
+                const float fr = t - fl;
+                const float dv = fmaf(vq, 1.2e-6f, dvc);
+                if (Mf > 0.f && (fr < dv || fr > 1.f - dv)) need_n |= 1u << i;
+                ncode[i] = Mf > 0.f ? min(255, (int)fl) : 0;
             }
         } else {
             float lmin = 1e30f, lmax = -1e30f, elmax = 0.f;
@@ -207,10 +300,11 @@ encode_kernel(EncArgs A) {
 #pragma unroll
             for (int i = 0; i < PPL; i++) {
                 const float r = rr[i];
-                unsure |= (r < 2.3841858e-7f) || (er[i] > 0.01f * r);  // r < 2^-22
-                const float l = log2f(fmaxf(r, 5.9604645e-8f));
+                const float er = fmaf(r, 1e-6f, ezr);
+                unsure |= (r < 2.3841858e-7f) || (er > 0.01f * r);  // r < 2^-22
+                const float l = lg2_approx(fmaxf(r, 5.9604645e-8f));
                 ll[i] = l;
-                el[i] = er[i] / (fmaxf(r, 1e-30f) * 0.69314718f) * 1.02f + fabsf(l) * 2.4e-7f + 1e-7f;
+                el[i] = er * rcp_approx(fmaxf(r, 1e-30f)) * 1.4717f + 1.2e-6f;
                 lmin = fminf(lmin, l);
                 lmax = fmaxf(lmax, l);
                 elmax = fmaxf(elmax, el[i]);
@@ -223,21 +317,17 @@ encode_kernel(EncArgs A) {
             const uint16_t LOh = f32_to_f16_sat(lmin), HIh = f32_to_f16_sat(lmax);
             const float LOf = half_bits_to_float(LOh), HIf = half_bits_to_float(HIh);
             prm = (uint32_t)LOh | ((uint32_t)HIh << 16);
-            const float inv = HIf != LOf ? 15.f / (HIf - LOf) : 0.f;
+            const float inv = HIf != LOf ? 15.f * rcp_approx(HIf - LOf) : 0.f;
 #pragma unroll
             for (int i = 0; i < PPL; i++) {
-                int cc = 0;
-                if (HIf != LOf) {
-                    const float vq = (ll[i] - LOf) * inv;
-                    const float t = vq + 0.5f;
-                    const float fl = floorf(t);
-                    const float fr = t - fl;
-                    const float dv = (el[i] + (fabsf(ll[i]) + fabsf(LOf)) * 1.2e-7f) * inv * 1.01f +
-                                     fabsf(vq) * 2.5e-7f + 1e-6f;
-                    if (fr < dv || fr > 1.f - dv) need_n |= 1u << i;
-                    cc = min(15, max(0, (int)fl));
-                }
-                ncode[i] = cc;
+                const float vq = (ll[i] - LOf) * inv;
+                const float t = vq + 0.5f;
+                const float fl = floorf(t);
+                const float fr = t - fl;
+                const float dv = (el[i] + (fabsf(ll[i]) + fabsf(LOf)) * 1.2e-7f) * inv * 1.02f +
+                                 fabsf(vq) * 1e-6f + 2e-6f;
+                if (HIf != LOf && (fr < dv || fr > 1.f - dv)) need_n |= 1u << i;
+                ncode[i] = HIf != LOf ? min(15, max(0, (int)fl)) : 0;
             }
         }
 
@@ -246,47 +336,64 @@ encode_kernel(EncArgs A) {
         if (__any_sync(KVQ_FULL_MASK, lane_need)) {
             double zd[EPL];
 #pragma unroll
-            for (int e = 0; e < EPL; e++) {
-                const uint16_t hb = (uint16_t)(raw[e / 2] >> (16 * (e & 1)));
-                const double f = (double)half_bits_to_float(hb);
-                zd[e] = ((negmask >> e) & 1u) ? -f : f;
+            for (int w = 0; w < NW; w++) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&raw[w]));
+                zd[2 * w] = (double)f.x;
+                zd[2 * w + 1] = (double)f.y;
             }
             fwht_local<EPL>(zd);
             fwht_cross<EPL, NL>(zd, lg);
-            double r64[PPL];
+            const bool gp = valid && need_p;  // uniform within the group
 #pragma unroll
-            for (int i = 0; i < PPL; i++) {
+            for (int i = 0; i < PPL; i++)
                 if ((need_a >> i) & 1u) acode[i] = exact_angle_code(zd[2 * i], zd[2 * i + 1], L);
-                r64[i] = hypot(zd[2 * i] / sqrt_d, zd[2 * i + 1] / sqrt_d);
-            }
-            const bool gp = need_p;  // uniform within the group
-            if (A.c.mode == KVQ_NORM_LIN8) {
-                double m = 0.0;
+            if (__any_sync(KVQ_FULL_MASK, gp)) {
+                // some group's parameter is in doubt: recompute all its norms
+                double r64[PPL];
 #pragma unroll
-                for (int i = 0; i < PPL; i++) m = fmax(m, r64[i]);
-                m = group_max_d<NL>(m);
-                if (gp) prm = f64_to_f16_sat(m);
-                const double M = (double)half_bits_to_float((uint16_t)prm);
+                for (int i = 0; i < PPL; i++) r64[i] = exact_norm(zd[2 * i], zd[2 * i + 1], sqrt_d);
+                if (A.c.mode == KVQ_NORM_LIN8) {
+                    double m = 0.0;
 #pragma unroll
-                for (int i = 0; i < PPL; i++)
-                    if (gp || ((need_n >> i) & 1u)) ncode[i] = lin8_code_exact(r64[i], M);
-            } else {
-                double l64[PPL];
-                double lo = 1e300, hi = -1e300;
+                    for (int i = 0; i < PPL; i++) m = fmax(m, r64[i]);
+                    m = group_max_d<NL>(m);
+                    if (gp) prm = f64_to_f16_sat(m);
+                    const double M = (double)half_bits_to_float((uint16_t)prm);
+#pragma unroll
+                    for (int i = 0; i < PPL; i++)
+                        if (gp || ((need_n >> i) & 1u)) ncode[i] = lin8_code_exact(r64[i], M);
+                } else {
+                    double l64[PPL];
+                    double lo = 1e300, hi = -1e300;
+#pragma unroll
+                    for (int i = 0; i < PPL; i++) {
+                        l64[i] = exact_log2(r64[i]);
+                        lo = fmin(lo, l64[i]);
+                        hi = fmax(hi, l64[i]);
+                    }
+                    lo = group_min_d<NL>(lo);
+                    hi = group_max_d<NL>(hi);
+                    if (gp) prm = (uint32_t)f64_to_f16_sat(lo) | ((uint32_t)f64_to_f16_sat(hi) << 16);
+                    const double LO = (double)half_bits_to_float((uint16_t)(prm & 0xFFFF));
+                    const double HI = (double)half_bits_to_float((uint16_t)(prm >> 16));
+#pragma unroll
+                    for (int i = 0; i < PPL; i++)
+                        if (gp || ((need_n >> i) & 1u)) ncode[i] = log4_code_exact(l64[i], LO, HI);
+                }
+            } else if (need_n) {
+                // only single codes in doubt: their norms alone, against the kept parameter
 #pragma unroll
                 for (int i = 0; i < PPL; i++) {
-                    l64[i] = log2(fmax(r64[i], 5.9604644775390625e-8));
-                    lo = fmin(lo, l64[i]);
-                    hi = fmax(hi, l64[i]);
+                    if (!((need_n >> i) & 1u)) continue;
+                    const double r = exact_norm(zd[2 * i], zd[2 * i + 1], sqrt_d);
+                    if (A.c.mode == KVQ_NORM_LIN8) {
+                        ncode[i] = lin8_code_exact(r, (double)half_bits_to_float((uint16_t)prm));
+                    } else {
+                        ncode[i] = log4_code_exact(exact_log2(r),
+                                                   (double)half_bits_to_float((uint16_t)(prm & 0xFFFF)),
+                                                   (double)half_bits_to_float((uint16_t)(prm >> 16)));
+                    }
                 }
-                lo = group_min_d<NL>(lo);
-                hi = group_max_d<NL>(hi);
-                if (gp) prm = (uint32_t)f64_to_f16_sat(lo) | ((uint32_t)f64_to_f16_sat(hi) << 16);
-                const double LO = (double)half_bits_to_float((uint16_t)(prm & 0xFFFF));
-                const double HI = (double)half_bits_to_float((uint16_t)(prm >> 16));
-#pragma unroll
-                for (int i = 0; i < PPL; i++)
-                    if (gp || ((need_n >> i) & 1u)) ncode[i] = log4_code_exact(l64[i], LO, HI);
             }
         }
 
@@ -313,7 +420,6 @@ encode_kernel(EncArgs A) {
             const int cb = lg * PPL * bits;
             const int w0 = cb >> 5, sh = cb & 31;
             uint32_t w[5];
-            // 160-bit shift of (hi:lo) left by sh, split in words
             {
                 const uint64_t l2 = sh ? (lo << sh) : lo;
                 const uint64_t h2 = sh ? ((hi << sh) | (lo >> (64 - sh))) : hi;

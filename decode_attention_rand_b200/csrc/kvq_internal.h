@@ -60,7 +60,9 @@ int record_error(int code, const char* msg);
 __host__ __device__ inline int64_t ws_counter_floats(int B, int H_q) {
     return ((int64_t)B * H_q + 3) / 4 * 4;
 }
-__host__ __device__ inline int64_t ws_stat_floats(int B, int H_q, int S) { return (int64_t)B * H_q * S * 2; }
+__host__ __device__ inline int64_t ws_stat_floats(int B, int H_q, int S) {
+    return ((int64_t)B * H_q * S * 2 + 3) / 4 * 4;  // keeps the accumulators 16-byte aligned
+}
 __host__ __device__ inline int64_t ws_acc_floats(int B, int H_q, int S, int d) { return (int64_t)B * H_q * S * d; }
 
 }  // namespace kvq

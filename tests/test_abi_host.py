@@ -57,8 +57,9 @@ def test_split_heuristic():
         assert ctas / (-(-ctas // 148) * 148) >= 0.9, (B, H, ctx, s)
     assert kvq.kvq_decode_num_splits(0, 8, 100, 148) == 1
     # counters (B*H_q int32, rounded to 16 bytes), (m, l) per split, acc per split
+    # (the (m, l) block is rounded to 4 floats so the accumulators stay 16-byte aligned)
     assert kvq.kvq_decode_workspace_bytes(2, 8, 128, 3) == 4 * (16 + 2 * 8 * 3 * 2 + 2 * 8 * 3 * 128)
-    assert kvq.kvq_decode_workspace_bytes(1, 3, 64, 1) == 4 * (4 + 3 * 2 + 3 * 64)
+    assert kvq.kvq_decode_workspace_bytes(1, 3, 64, 1) == 4 * (4 + 8 + 3 * 64)
 
 
 FAKE = 1 << 20  # 16-byte aligned non-NULL addresses; never dereferenced
