@@ -43,12 +43,30 @@ if ROOT not in sys.path:
 DEFAULT_WORKLOAD = "llama7b_layer_b1_hq32_hkv8_d128_ctx4096"
 METRIC = "decode-attn effective HBM GB/s"
 FALLBACK_HBM_GBS = 6650.0
+SM_COUNT_B200 = 148
+FP32_LANES_PER_SM = 128     # FP32 FMA lanes per SM (4 sub-partitions x 32)
+SM_MAX_MHZ = 1965.0
+
+
+def fp32_peak_tflops(sm_mhz, sm_count=SM_COUNT_B200):
+    """FP32 FMA-pipe peak, counting an FMA as two flops."""
+    return 2.0 * FP32_LANES_PER_SM * sm_count * sm_mhz * 1e6 / 1e12
+
+
+def decode_flops_per_token_head(d, G):
+    """FP32-pipe work of decode attention per cached token and KV head, in
+    flops with every pipe operation counted as an FMA (two flops): each pair
+    is scaled by its norm once for K and once for V (2 d multiplies), then
+    every one of the G query heads takes d FMAs for its score and d FMAs for
+    its value accumulation, 2 d (G + 1) operations in all.  A multiply fills
+    an FMA lane slot, so this is the work that meets the FMA-pipe peak."""
+    return 2 * 2 * d * (G + 1)
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=4000)
+    p.add_argument("--steps", type=int, default=20000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -56,6 +74,11 @@ def parse():
                    help="wall time of the bounded oracle sample (cpu_baseline)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-encode", action="store_true")
+    p.add_argument("--case", default=None, choices=["decode_layer", "encode_layer"],
+                   help="run one kernel case only (for profiler captures): the decode of "
+                        "--layer of --workload, or the prefill encode of 8 batch entries of "
+                        "one layer; --steps launches after 3 warm-up launches")
+    p.add_argument("--layer", type=int, default=0)
     return p.parse_args()
 
 
@@ -219,7 +242,7 @@ class DecodeStep:
                                     knew=knew, vnew=vnew, out=out,
                                     cK=[p[0].c() for p in planes], cV=[p[1].c() for p in planes]))
         torch.cuda.synchronize(device)
-        self.kernels_per_step = 4 * w.layers  # 2 encode, decode split, combine
+        self.kernels_per_step = 3 * w.layers  # K append, V append, decode (split + combine)
 
     def step(self, i, ev=None, stream=None):
         kvq, w = self.kvq, self.w
@@ -371,6 +394,120 @@ def time_encode(device, hbm_peak):
     }
 
 
+def time_decode_layers(device, hbm_peak, sm_mhz):
+    """Decode-kernel time on single layers of the large decode workloads
+    (eager launches, CUDA events; each layer's codes exceed L2)."""
+    import torch
+    from decode_attention_rand_b200 import kvq, synth
+    sm = torch.cuda.get_device_properties(device).multi_processor_count
+    fp_peak = fp32_peak_tflops(sm_mhz, sm)
+    res = []
+    for name, layer in (("mistral7b_32layers_b8_hq32_hkv8_d128_ctx32768", 4),
+                        ("mistral7b_32layers_b8_hq32_hkv8_d128_ctx32768", 0),
+                        ("tinyllama_22layers_b4_hq32_hkv4_d64_ctx65536", 2)):
+        w = synth.WORKLOADS[name]
+        sk, sv = synth.layer_signs(w, layer)
+        skd, svd = torch.from_numpy(sk).to(device), torch.from_numpy(sv).to(device)
+        kc = kvq.codec(w.d, w.L_K[layer], w.mode_K)
+        vc = kvq.codec(w.d, w.L_V[layer], w.mode_V)
+        planes = []
+        for kind, c, sg in ((synth.KIND_K, kc, skd), (synth.KIND_V, vc, svd)):
+            p = kvq.alloc_plane(c, w.B, w.H_kv, w.ctx, device)
+            x = synth.kv(w, layer, kind, device=device)
+            kvq.encode(c, sg, x, p, 0)
+            del x
+            planes.append(p)
+        q = synth.queries(w, layer, device=device)
+        ctx = torch.full((w.B,), w.ctx, dtype=torch.int32, device=device)
+        out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float16, device=device)
+        S = kvq.kvq_decode_num_splits(w.B, w.H_kv, w.ctx, sm)
+        ws = kvq.DecodeWorkspace(w.B, w.H_q, w.d, S, device)
+
+        def run():
+            kvq.decode_attn(q, kc, vc, skd, svd, planes[0], planes[1], ctx, w.ctx, None,
+                            num_splits=S, workspace=ws, out=out, out_dtype=kvq.OUT_FP16)
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 20
+        e0.record()
+        for _ in range(n):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / n
+        nb = (w.B * w.H_kv * w.ctx * (row_bytes_total(kvq, w.d, kc.L, kc.norm_mode) +
+                                      row_bytes_total(kvq, w.d, vc.L, vc.norm_mode)) +
+              w.B * w.H_q * w.d * 4)
+        fl = w.B * w.H_kv * w.ctx * decode_flops_per_token_head(w.d, w.G)
+        res.append({"workload": f"{name} layer {layer} (L_K {kc.L}, L_V {vc.L}, {S} splits)",
+                    "us": t * 1e6, "gb_per_s": nb / t / 1e9, "hbm_frac": nb / t / 1e9 / hbm_peak,
+                    "tflop_per_s": fl / t / 1e12, "fp32_frac": fl / t / 1e12 / fp_peak})
+        del planes, q, ws
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_case(args):
+    """One kernel case on cuda:0, for profiler captures of a single launch."""
+    import torch
+    from decode_attention_rand_b200 import build as kbuild
+    from decode_attention_rand_b200 import kvq, synth
+    kbuild.build()
+    kvq.lib()
+    device = torch.device("cuda", 0)
+    steps = max(1, min(args.steps, 20))
+    if args.case == "decode_layer":
+        w = synth.WORKLOADS[args.workload]
+        layer = args.layer
+        sk, sv = synth.layer_signs(w, layer)
+        skd, svd = torch.from_numpy(sk).to(device), torch.from_numpy(sv).to(device)
+        kc = kvq.codec(w.d, w.L_K[layer], w.mode_K)
+        vc = kvq.codec(w.d, w.L_V[layer], w.mode_V)
+        planes = []
+        for kind, c, sg in ((synth.KIND_K, kc, skd), (synth.KIND_V, vc, svd)):
+            p = kvq.alloc_plane(c, w.B, w.H_kv, w.ctx, device)
+            x = synth.kv(w, layer, kind, device=device)
+            kvq.encode(c, sg, x, p, 0)
+            del x
+            planes.append(p)
+        q = synth.queries(w, layer, device=device)
+        ctx = torch.full((w.B,), w.ctx, dtype=torch.int32, device=device)
+        out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float16, device=device)
+        sm = torch.cuda.get_device_properties(device).multi_processor_count
+        S = kvq.kvq_decode_num_splits(w.B, w.H_kv, w.ctx, sm)
+        ws = kvq.DecodeWorkspace(w.B, w.H_q, w.d, S, device)
+
+        def run():
+            kvq.decode_attn(q, kc, vc, skd, svd, planes[0], planes[1], ctx, w.ctx, None,
+                            num_splits=S, workspace=ws, out=out, out_dtype=kvq.OUT_FP16)
+        what = f"decode {w.name} layer {layer}, {S} splits"
+    else:
+        w = synth.WORKLOADS["prefill_32layers_b16_t8192_hkv8_d128"]
+        sk, _ = synth.layer_signs(w, 0)
+        c = kvq.codec(w.d, w.L_K[0], w.mode_K)
+        nb = 8
+        p = kvq.alloc_plane(c, nb, w.H_kv, w.ctx, device)
+        x = synth.kv(w, 0, synth.KIND_K, device=device, b_range=(0, nb))
+        skd = torch.from_numpy(sk).to(device)
+
+        def run():
+            kvq.encode(c, skd, x, p, 0)
+        what = f"encode {w.name} layer 0 K, batch entries 0..{nb - 1}"
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": what, "us_per_launch": e0.elapsed_time(e1) * 1e3 / steps}), flush=True)
+    return 0
+
+
 # --------------------------------------------------------------- oracle --
 
 class OracleSteps:
@@ -516,6 +653,8 @@ def run_reference(args, w):
 
 def main():
     args = parse()
+    if args.case:
+        return run_case(args)
     from decode_attention_rand_b200 import synth
     w = synth.WORKLOADS[args.workload]
     ctx = init_dist(args.gpus)
@@ -550,6 +689,7 @@ def main():
     e2e_ms, e2e_n, h2d, d2h = time_e2e(state, args.steps, ctx)
     e2e_ms = max_over_ranks(ctx, e2e_ms)
     enc = None if args.no_encode else time_encode(device, hbm_peak)
+    big = None if args.no_encode else time_decode_layers(device, hbm_peak, SM_MAX_MHZ)
     t_end = time.time()
     sampler.stop()
     if int(state.err.item()) != 0:
@@ -565,6 +705,14 @@ def main():
     e2e = world * total_bytes * e2e_n / (e2e_ms / 1e3) / 1e9
     dec_bytes = statistics.fmean(per_layer)
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    dec_flops = w.B * w.H_kv * w.ctx * decode_flops_per_token_head(w.d, w.G)
+    sm_mhz = clocks.get("sm_mhz") or SM_MAX_MHZ
+    fp_peak = fp32_peak_tflops(sm_mhz, props.multi_processor_count)
+    fp_achieved = dec_flops / (dec_ms / 1e3) / 1e12
+    traffic = profile_traffic("decode_kernel_llama7b_layer")
+    # the binding roofline of the decode kernel: FP32 FMA pipe when the time
+    # its flops need at peak exceeds the time its bytes need at HBM peak
+    fp_bound = dec_flops / (fp_peak * 1e12) > dec_bytes / (hbm_peak * 1e9)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -578,12 +726,23 @@ def main():
             "timing": "CUDA graph replay, CUDA events, max over ranks",
             "bytes_per_step": total_bytes,
         },
-        "roofline": {
-            "kernel": "decode_split_kernel + decode_combine_kernel (one kvq_decode_attn call)",
+        "roofline": ({
+            "kernel": "decode_kernel (one kvq_decode_attn launch: splits and their combine)",
+            "bound": "alu", "achieved": fp_achieved, "peak": fp_peak, "unit": "TFLOP/s",
+            "frac": fp_achieved / fp_peak,
+            "peak_kind": f"FP32 FMA pipe, derived: {FP32_LANES_PER_SM} lanes/SM x "
+                         f"{props.multi_processor_count} SMs x 2 flop x {sm_mhz:.0f} MHz",
+            "traffic": traffic, "flops_per_launch": dec_flops, "bytes_per_launch": dec_bytes,
+            "us_per_launch": dec_ms * 1e3,
+        } if fp_bound else {
+            "kernel": "decode_kernel (one kvq_decode_attn launch: splits and their combine)",
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
-            "traffic": profile_traffic("decode_split_llama7b_layer"),
-            "bytes_per_launch": dec_bytes, "us_per_launch": dec_ms * 1e3,
+            "traffic": traffic, "bytes_per_launch": dec_bytes, "us_per_launch": dec_ms * 1e3,
+        }),
+        "roofline_hbm": {
+            "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+            "peak_kind": f"{peak_kind} copy bandwidth", "traffic": traffic,
         },
         "e2e": {"value": e2e, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_n},
@@ -592,6 +751,10 @@ def main():
     }
     if enc:
         line["encode"] = enc
+    if big:
+        for r in big:
+            r["fp32_frac"] = r["tflop_per_s"] / fp_peak
+        line["decode_large_layers"] = big
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
