@@ -2,10 +2,11 @@
 """Benchmark of the compressed-KV decode step (one JSON line on rank 0).
 
 A step is one pass of the whole hot path over one batch of synthetic input,
-for every layer of the workload: append the new token's K and V (encode,
-T = 1, at the last cache slot) and run split-K decode attention over the
-whole compressed context (query rotation, scores from codes, online softmax,
-value accumulation in the rotated domain, combine, inverse rotation).
+for every layer of the workload: append the new token's K and V (one encode
+launch for both, T = 1, at the last cache slot) and run split-K decode
+attention over the whole compressed context (query rotation, scores from
+codes, online softmax, value accumulation in the rotated domain, combine,
+inverse rotation), two launches per layer.
 
   value  decode-attention effective HBM GB/s = algorithmic bytes of the step
          (packed K/V codes + fp16 params read, q read, output written, the
@@ -242,15 +243,15 @@ class DecodeStep:
                                     knew=knew, vnew=vnew, out=out,
                                     cK=[p[0].c() for p in planes], cV=[p[1].c() for p in planes]))
         torch.cuda.synchronize(device)
-        self.kernels_per_step = 3 * w.layers  # K append, V append, decode (split + combine)
+        self.kernels_per_step = 2 * w.layers  # K+V append, decode (splits + combine)
 
     def step(self, i, ev=None, stream=None):
         kvq, w = self.kvq, self.w
         b = i % self.nbuf
         st = stream.cuda_stream if stream is not None else self.torch.cuda.current_stream().cuda_stream
         for li, L in enumerate(self.layers):
-            kvq.kvq_encode(L["kc"], L["skd"], L["knew"], w.B, w.H_kv, 1, w.ctx - 1, L["cK"][b], st)
-            kvq.kvq_encode(L["vc"], L["svd"], L["vnew"], w.B, w.H_kv, 1, w.ctx - 1, L["cV"][b], st)
+            kvq.kvq_encode_kv(L["kc"], L["skd"], L["knew"], L["cK"][b], L["vc"], L["svd"],
+                              L["vnew"], L["cV"][b], w.B, w.H_kv, 1, w.ctx - 1, st)
             if ev is not None:
                 ev[li][0].record()
             kvq.kvq_decode_attn(L["q"], L["kc"], L["vc"], L["skd"], L["svd"], L["cK"][b],

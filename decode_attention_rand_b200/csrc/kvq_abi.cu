@@ -115,25 +115,64 @@ int64_t kvq_row_bytes(const kvq_codec* c, int32_t which) {
     }
 }
 
+}  // extern "C"
+
+namespace {
+
+// Argument checks of one encode job; *job->n_vec is 0 when there is nothing
+// to encode.
+int prep_encode(const kvq_codec* codec, const int8_t* signs, const void* x, int32_t B,
+                int32_t H_kv, int32_t T, int64_t pos0, const kvq_plane* out, const char* what,
+                const char* xname, kvq::EncodeJob* job) {
+    int rc = check_codec(codec, what, &job->c);
+    if (rc) return rc;
+    rc = check_plane(out, what, &job->out);
+    if (rc) return rc;
+    if (B < 0 || H_kv < 0 || T < 0) return fail(KVQ_EINVAL, "%s: negative size", what);
+    if (pos0 < 0 || pos0 + (int64_t)T > job->out.capacity)
+        return fail(KVQ_EINVAL, "%s: tokens [%lld, %lld) exceed capacity %lld", what,
+                    (long long)pos0, (long long)(pos0 + T), (long long)job->out.capacity);
+    job->n_vec = (int64_t)B * H_kv * T;
+    job->T = T;
+    job->pos0 = pos0;
+    job->signs = signs;
+    job->x = static_cast<const __half*>(x);
+    if (job->n_vec == 0) return KVQ_OK;
+    if (!signs || !x) return fail(KVQ_EINVAL, "%s: NULL signs or %s", what, xname);
+    if (!aligned16(x)) return fail(KVQ_EINVAL, "%s: %s must be 16-byte aligned", what, xname);
+    return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 int kvq_encode(const kvq_codec* codec, const int8_t* signs, const void* x, int32_t B, int32_t H_kv,
                int32_t T, int64_t pos0, const kvq_plane* out, void* stream) {
-    kvq::CodecDev c;
-    kvq::PlaneDev p;
-    int rc = check_codec(codec, "kvq_encode", &c);
+    kvq::EncodeJob j;
+    const int rc = prep_encode(codec, signs, x, B, H_kv, T, pos0, out, "kvq_encode", "x", &j);
     if (rc) return rc;
-    rc = check_plane(out, "kvq_encode", &p);
-    if (rc) return rc;
-    if (B < 0 || H_kv < 0 || T < 0) return fail(KVQ_EINVAL, "kvq_encode: negative size");
-    if (pos0 < 0 || pos0 + (int64_t)T > p.capacity)
-        return fail(KVQ_EINVAL, "kvq_encode: tokens [%lld, %lld) exceed capacity %lld",
-                    (long long)pos0, (long long)(pos0 + T), (long long)p.capacity);
-    const int64_t n = (int64_t)B * H_kv * T;
-    if (n == 0) return ok();
-    if (!signs || !x) return fail(KVQ_EINVAL, "kvq_encode: NULL signs or x");
-    if (!aligned16(x)) return fail(KVQ_EINVAL, "kvq_encode: x must be 16-byte aligned");
-    return cuda_status(kvq::launch_encode(c, signs, static_cast<const __half*>(x), n, T, pos0, p,
-                                          sm_count_current(), static_cast<cudaStream_t>(stream)),
+    if (j.n_vec == 0) return ok();
+    return cuda_status(kvq::launch_encode_jobs(&j, 1, sm_count_current(),
+                                               static_cast<cudaStream_t>(stream)),
                        "kvq_encode");
+}
+
+int kvq_encode_kv(const kvq_codec* kc, const int8_t* signs_k, const void* k, const kvq_plane* K,
+                  const kvq_codec* vc, const int8_t* signs_v, const void* v, const kvq_plane* V,
+                  int32_t B, int32_t H_kv, int32_t T, int64_t pos0, void* stream) {
+    kvq::EncodeJob j[2];
+    int rc = prep_encode(kc, signs_k, k, B, H_kv, T, pos0, K, "kvq_encode_kv", "k", &j[0]);
+    if (rc) return rc;
+    rc = prep_encode(vc, signs_v, v, B, H_kv, T, pos0, V, "kvq_encode_kv", "v", &j[1]);
+    if (rc) return rc;
+    if (j[0].c.d != j[1].c.d)
+        return fail(KVQ_EINVAL, "kvq_encode_kv: K head_dim %d differs from V head_dim %d",
+                    j[0].c.d, j[1].c.d);
+    if (j[0].n_vec == 0) return ok();
+    return cuda_status(kvq::launch_encode_jobs(j, 2, sm_count_current(),
+                                               static_cast<cudaStream_t>(stream)),
+                       "kvq_encode_kv");
 }
 
 int kvq_dequant(const kvq_codec* codec, const int8_t* signs, const kvq_plane* in, int32_t B,

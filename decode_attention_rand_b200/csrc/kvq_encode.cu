@@ -150,9 +150,16 @@ __device__ __forceinline__ int log4_code_exact(double l, double LO, double HI) {
     return q < 0.0 ? 0 : (q > 15.0 ? 15 : (int)q);
 }
 
+// One launch encodes one tensor (blockIdx.y = 0) or K and V together
+// (blockIdx.y selects the tensor).
+struct EncPair {
+    EncArgs a[2];
+};
+
 template <int D>
 __global__ void __launch_bounds__(kEncWarps * 32)
-encode_kernel(EncArgs A) {
+encode_kernel(EncPair PA) {
+    const EncArgs A = blockIdx.y ? PA.a[1] : PA.a[0];
     using Cfg = EncCfg<D>;
     constexpr int EPL = Cfg::EPL, NL = Cfg::NL, PPL = Cfg::PPL, VPW = Cfg::VPW;
     constexpr int NW = EPL / 2;  // packed pairs per lane (= PPL)
@@ -271,6 +278,11 @@ encode_kernel(EncArgs A) {
         int ncode[PPL];
         uint32_t prm = 0;     // packed fp16 parameter(s)
         bool need_p = false;  // group-uniform
+        // group-wide values the exact path reuses to find the pairs that can
+        // decide a parameter
+        float pmax = 0.f, pmin = 0.f, pband = 0.f;
+        bool unsure = false;  // LOG4: some norm too small for the linearised bound
+        float ll[PPL];        // LOG4: fp32 log2 of each pair norm
         if (A.c.mode == KVQ_NORM_LIN8) {
             float m = 0.f;
 #pragma unroll
@@ -278,6 +290,8 @@ encode_kernel(EncArgs A) {
             m = group_max<NL>(m);
             const float eM = ezr + m * 1e-6f;
             need_p = near_f16_midpoint(m, eM);
+            pmax = m;
+            pband = 2.f * eM;
             const uint16_t Mh = f32_to_f16_sat(m);
             const float Mf = half_bits_to_float(Mh);
             prm = Mh;
@@ -295,8 +309,7 @@ encode_kernel(EncArgs A) {
             }
         } else {
             float lmin = 1e30f, lmax = -1e30f, elmax = 0.f;
-            bool unsure = false;
-            float ll[PPL], el[PPL];
+            float el[PPL];
 #pragma unroll
             for (int i = 0; i < PPL; i++) {
                 const float r = rr[i];
@@ -314,6 +327,9 @@ encode_kernel(EncArgs A) {
             elmax = group_max<NL>(elmax);
             unsure = group_any<NL>(unsure);
             need_p = unsure || near_f16_midpoint(lmin, elmax) || near_f16_midpoint(lmax, elmax);
+            pmin = lmin;
+            pmax = lmax;
+            pband = 2.f * elmax;
             const uint16_t LOh = f32_to_f16_sat(lmin), HIh = f32_to_f16_sat(lmax);
             const float LOf = half_bits_to_float(LOh), HIf = half_bits_to_float(HIh);
             prm = (uint32_t)LOh | ((uint32_t)HIh << 16);
@@ -347,49 +363,52 @@ encode_kernel(EncArgs A) {
 #pragma unroll
             for (int i = 0; i < PPL; i++)
                 if ((need_a >> i) & 1u) acode[i] = exact_angle_code(zd[2 * i], zd[2 * i + 1], L);
+            // A parameter in doubt is decided by the pairs that can hold the
+            // exact extreme: pair i can only if its fp32 value lies within the
+            // two error bounds (its own and the fp32 extreme's) of the fp32
+            // extreme.  Only those pairs get exact norms here; when the exact
+            // parameter equals the fp32 one, the fp32 codes stand except those
+            // already flagged, otherwise (or when the bounds themselves are in
+            // doubt) every code of the group is re-decided.
+            double x64[PPL];  // exact r (LIN8) or log2 r (LOG4) where computed
+            uint32_t have = 0;
             if (__any_sync(KVQ_FULL_MASK, gp)) {
-                // some group's parameter is in doubt: recompute all its norms
-                double r64[PPL];
+                const bool lin8 = A.c.mode == KVQ_NORM_LIN8;
+                double ext_hi = lin8 ? 0.0 : -1e300, ext_lo = 1e300;
 #pragma unroll
-                for (int i = 0; i < PPL; i++) r64[i] = exact_norm(zd[2 * i], zd[2 * i + 1], sqrt_d);
-                if (A.c.mode == KVQ_NORM_LIN8) {
-                    double m = 0.0;
-#pragma unroll
-                    for (int i = 0; i < PPL; i++) m = fmax(m, r64[i]);
-                    m = group_max_d<NL>(m);
-                    if (gp) prm = f64_to_f16_sat(m);
-                    const double M = (double)half_bits_to_float((uint16_t)prm);
-#pragma unroll
-                    for (int i = 0; i < PPL; i++)
-                        if (gp || ((need_n >> i) & 1u)) ncode[i] = lin8_code_exact(r64[i], M);
-                } else {
-                    double l64[PPL];
-                    double lo = 1e300, hi = -1e300;
-#pragma unroll
-                    for (int i = 0; i < PPL; i++) {
-                        l64[i] = exact_log2(r64[i]);
-                        lo = fmin(lo, l64[i]);
-                        hi = fmax(hi, l64[i]);
+                for (int i = 0; i < PPL; i++) {
+                    const float v32 = lin8 ? rr[i] : ll[i];
+                    const bool cand_hi = v32 >= pmax - pband;
+                    const bool cand_lo = !lin8 && v32 <= pmin + pband;
+                    if (gp && (unsure || cand_hi || cand_lo)) {
+                        const double r = exact_norm(zd[2 * i], zd[2 * i + 1], sqrt_d);
+                        x64[i] = lin8 ? r : exact_log2(r);
+                        have |= 1u << i;
+                        if (unsure || cand_hi) ext_hi = fmax(ext_hi, x64[i]);
+                        if (unsure || cand_lo) ext_lo = fmin(ext_lo, x64[i]);
                     }
-                    lo = group_min_d<NL>(lo);
-                    hi = group_max_d<NL>(hi);
-                    if (gp) prm = (uint32_t)f64_to_f16_sat(lo) | ((uint32_t)f64_to_f16_sat(hi) << 16);
-                    const double LO = (double)half_bits_to_float((uint16_t)(prm & 0xFFFF));
-                    const double HI = (double)half_bits_to_float((uint16_t)(prm >> 16));
-#pragma unroll
-                    for (int i = 0; i < PPL; i++)
-                        if (gp || ((need_n >> i) & 1u)) ncode[i] = log4_code_exact(l64[i], LO, HI);
                 }
-            } else if (need_n) {
-                // only single codes in doubt: their norms alone, against the kept parameter
+                ext_hi = group_max_d<NL>(ext_hi);
+                ext_lo = group_min_d<NL>(ext_lo);
+                uint32_t prm_x = lin8 ? (uint32_t)f64_to_f16_sat(ext_hi)
+                                      : ((uint32_t)f64_to_f16_sat(ext_lo) |
+                                         ((uint32_t)f64_to_f16_sat(ext_hi) << 16));
+                const bool redo_all = gp && (unsure || prm_x != prm);
+                if (gp) prm = prm_x;
+                if (redo_all) need_n = (1u << PPL) - 1u;
+            }
+            if (need_n) {
 #pragma unroll
                 for (int i = 0; i < PPL; i++) {
                     if (!((need_n >> i) & 1u)) continue;
-                    const double r = exact_norm(zd[2 * i], zd[2 * i + 1], sqrt_d);
+                    if (!((have >> i) & 1u)) {
+                        const double r = exact_norm(zd[2 * i], zd[2 * i + 1], sqrt_d);
+                        x64[i] = A.c.mode == KVQ_NORM_LIN8 ? r : exact_log2(r);
+                    }
                     if (A.c.mode == KVQ_NORM_LIN8) {
-                        ncode[i] = lin8_code_exact(r, (double)half_bits_to_float((uint16_t)prm));
+                        ncode[i] = lin8_code_exact(x64[i], (double)half_bits_to_float((uint16_t)prm));
                     } else {
-                        ncode[i] = log4_code_exact(exact_log2(r),
+                        ncode[i] = log4_code_exact(x64[i],
                                                    (double)half_bits_to_float((uint16_t)(prm & 0xFFFF)),
                                                    (double)half_bits_to_float((uint16_t)(prm >> 16)));
                     }
@@ -482,40 +501,58 @@ encode_kernel(EncArgs A) {
 }
 
 template <int D>
-static cudaError_t launch_encode_d(const EncArgs& a, int sm_count, cudaStream_t stream) {
+static cudaError_t launch_encode_d(const EncPair& pa, int n_args, int sm_count,
+                                   cudaStream_t stream) {
     constexpr int VPW = EncCfg<D>::VPW;
-    const int64_t tiles = (a.n_vec + VPW - 1) / VPW;
+    int64_t n_max = pa.a[0].n_vec;
+    if (n_args > 1 && pa.a[1].n_vec > n_max) n_max = pa.a[1].n_vec;
+    const int64_t tiles = (n_max + VPW - 1) / VPW;
     int64_t blocks = (tiles + kEncWarps - 1) / kEncWarps;
-    const int64_t cap = (int64_t)sm_count * 8;
+    const int64_t cap = (int64_t)sm_count * 8 / n_args;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    encode_kernel<D><<<(unsigned)blocks, kEncWarps * 32, 0, stream>>>(a);
+    encode_kernel<D><<<dim3((unsigned)blocks, (unsigned)n_args), kEncWarps * 32, 0, stream>>>(pa);
     return cudaGetLastError();
+}
+
+static EncArgs make_args(const EncodeJob& j) {
+    EncArgs a;
+    a.x = j.x;
+    a.signs = j.signs;
+    a.n_vec = j.n_vec;
+    a.T = j.T;
+    a.pos0 = j.pos0;
+    a.c = j.c;
+    a.out = j.out;
+    a.inv_sqrt_d = (float)(1.0 / sqrt((double)j.c.d));
+    a.bins_per_rad = (float)((double)j.c.L / (2.0 * kPi));
+    return a;
+}
+
+cudaError_t launch_encode_jobs(const EncodeJob* jobs, int n_jobs, int sm_count,
+                               cudaStream_t stream) {
+    if (n_jobs < 1 || n_jobs > 2) return cudaErrorInvalidValue;
+    if (n_jobs == 2 && jobs[0].c.d != jobs[1].c.d) return cudaErrorInvalidValue;
+    EncPair pa;
+    pa.a[0] = make_args(jobs[0]);
+    pa.a[1] = n_jobs == 2 ? make_args(jobs[1]) : pa.a[0];
+    switch (jobs[0].c.d) {
+        case 4: return launch_encode_d<4>(pa, n_jobs, sm_count, stream);
+        case 8: return launch_encode_d<8>(pa, n_jobs, sm_count, stream);
+        case 16: return launch_encode_d<16>(pa, n_jobs, sm_count, stream);
+        case 32: return launch_encode_d<32>(pa, n_jobs, sm_count, stream);
+        case 64: return launch_encode_d<64>(pa, n_jobs, sm_count, stream);
+        case 128: return launch_encode_d<128>(pa, n_jobs, sm_count, stream);
+        case 256: return launch_encode_d<256>(pa, n_jobs, sm_count, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_encode(const CodecDev& c, const int8_t* signs, const __half* x, int64_t n_vec,
                           int64_t T, int64_t pos0, const PlaneDev& out, int sm_count,
                           cudaStream_t stream) {
-    EncArgs a;
-    a.x = x;
-    a.signs = signs;
-    a.n_vec = n_vec;
-    a.T = T;
-    a.pos0 = pos0;
-    a.c = c;
-    a.out = out;
-    a.inv_sqrt_d = (float)(1.0 / sqrt((double)c.d));
-    a.bins_per_rad = (float)((double)c.L / (2.0 * kPi));
-    switch (c.d) {
-        case 4: return launch_encode_d<4>(a, sm_count, stream);
-        case 8: return launch_encode_d<8>(a, sm_count, stream);
-        case 16: return launch_encode_d<16>(a, sm_count, stream);
-        case 32: return launch_encode_d<32>(a, sm_count, stream);
-        case 64: return launch_encode_d<64>(a, sm_count, stream);
-        case 128: return launch_encode_d<128>(a, sm_count, stream);
-        case 256: return launch_encode_d<256>(a, sm_count, stream);
-        default: return cudaErrorInvalidValue;
-    }
+    const EncodeJob j{c, signs, x, n_vec, T, pos0, out};
+    return launch_encode_jobs(&j, 1, sm_count, stream);
 }
 
 }  // namespace kvq

@@ -10,6 +10,22 @@ cudaError_t launch_encode(const CodecDev& c, const int8_t* signs, const __half* 
                           int64_t T, int64_t pos0, const PlaneDev& out, int sm_count,
                           cudaStream_t stream);
 
+// One tensor's share of an encode launch.
+struct EncodeJob {
+    CodecDev c;
+    const int8_t* signs;
+    const __half* x;
+    int64_t n_vec;  // B * H_kv * T
+    int64_t T;
+    int64_t pos0;
+    PlaneDev out;
+};
+
+// One launch for one or two jobs of the same head_dim (K and V appended
+// together); a job with n_vec 0 is skipped.
+cudaError_t launch_encode_jobs(const EncodeJob* jobs, int n_jobs, int sm_count,
+                               cudaStream_t stream);
+
 cudaError_t launch_dequant(const CodecDev& c, const int8_t* signs, const PlaneDev& in,
                            int64_t n_vec, int64_t T, int64_t pos0, __half* y, int sm_count,
                            cudaStream_t stream);

@@ -52,6 +52,9 @@ _SIGNATURES = {
     "kvq_row_bytes": (C.c_int64, [C.POINTER(kvq_codec), C.c_int32]),
     "kvq_encode": (C.c_int, [C.POINTER(kvq_codec), C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
                              C.c_int32, C.c_int64, C.POINTER(kvq_plane), C.c_void_p]),
+    "kvq_encode_kv": (C.c_int, [C.POINTER(kvq_codec), C.c_void_p, C.c_void_p, C.POINTER(kvq_plane),
+                                C.POINTER(kvq_codec), C.c_void_p, C.c_void_p, C.POINTER(kvq_plane),
+                                C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_void_p]),
     "kvq_dequant": (C.c_int, [C.POINTER(kvq_codec), C.c_void_p, C.POINTER(kvq_plane), C.c_int32,
                               C.c_int32, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]),
     "kvq_decode_num_splits": (C.c_int32, [C.c_int32, C.c_int32, C.c_int64, C.c_int32]),
@@ -140,6 +143,13 @@ def kvq_encode(codec: kvq_codec, signs, x, B: int, H_kv: int, T: int, pos0: int,
                             C.byref(out), _stream(stream)))
 
 
+def kvq_encode_kv(kc: kvq_codec, signs_k, k, K: kvq_plane, vc: kvq_codec, signs_v, v,
+                  V: kvq_plane, B: int, H_kv: int, T: int, pos0: int, stream=None):
+    _check(lib().kvq_encode_kv(C.byref(kc), _ptr(signs_k), _ptr(k), C.byref(K), C.byref(vc),
+                               _ptr(signs_v), _ptr(v), C.byref(V), B, H_kv, T, pos0,
+                               _stream(stream)))
+
+
 def kvq_dequant(codec: kvq_codec, signs, plane: kvq_plane, B: int, H_kv: int, T: int,
                 pos0: int, y, stream=None):
     _check(lib().kvq_dequant(C.byref(codec), _ptr(signs), C.byref(plane), B, H_kv, T, pos0,
@@ -218,6 +228,16 @@ def encode(c: kvq_codec, signs, x, plane: Plane, pos0: int = 0, stream=None):
     """Encode x [B, H_kv, T, d] (fp16, contiguous) into plane tokens pos0.."""
     B, H, T, d = x.shape
     kvq_encode(c, signs, x, B, H, T, pos0, plane.c(), stream)
+
+
+def encode_kv(kc: kvq_codec, signs_k, k, K: Plane, vc: kvq_codec, signs_v, v, V: Plane,
+              pos0: int = 0, stream=None):
+    """Encode k and v [B, H_kv, T, d] (fp16, contiguous) into K and V tokens
+    pos0.. in one launch."""
+    if tuple(k.shape) != tuple(v.shape):
+        raise ValueError("k and v must have the same shape")
+    B, H, T, d = k.shape
+    kvq_encode_kv(kc, signs_k, k, K.c(), vc, signs_v, v, V.c(), B, H, T, pos0, stream)
 
 
 def dequant(c: kvq_codec, signs, plane: Plane, T: int, pos0: int = 0, out=None, stream=None):

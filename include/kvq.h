@@ -152,6 +152,20 @@ int kvq_encode(const kvq_codec* codec, const int8_t* signs, const void* x,
                int32_t B, int32_t H_kv, int32_t T, int64_t pos0,
                const kvq_plane* out, void* stream);
 
+/* Encode the same token range of a layer's K and V in one launch: the same
+ * result as kvq_encode(kc, signs_k, k, B, H_kv, T, pos0, K) followed by
+ * kvq_encode(vc, signs_v, v, B, H_kv, T, pos0, V).  The per-token append of
+ * a decode step writes one K and one V row per (b, h); one launch instead of
+ * two halves the fixed cost of that step (the TurboAngle abstract encodes K
+ * and V independently, so nothing ties the two halves together but the
+ * launch).  Requires kc->head_dim == vc->head_dim; the codecs may differ in
+ * L and norm mode.  Arguments as for kvq_encode; argument errors are
+ * reported before anything is launched.  T == 0 is a no-op. */
+int kvq_encode_kv(const kvq_codec* kc, const int8_t* signs_k, const void* k,
+                  const kvq_plane* K, const kvq_codec* vc, const int8_t* signs_v,
+                  const void* v, const kvq_plane* V, int32_t B, int32_t H_kv,
+                  int32_t T, int64_t pos0, void* stream);
+
 /* Dequantize tokens pos0 .. pos0+T-1 of a plane back to fp16:
  *   y  device fp16 [B][H_kv][T][head_dim], 16-byte aligned (x^ above). */
 int kvq_dequant(const kvq_codec* codec, const int8_t* signs,

@@ -90,6 +90,32 @@ def test_encode_rejects_bad_arguments(case):
     assert case["msg"] in kvq.kvq_last_error()
 
 
+@pytest.mark.parametrize("case", [
+    dict(vc=(64, 64, 1), msg="head_dim"),
+    dict(k=FAKE + 2, msg="k must be 16-byte aligned"),
+    dict(v=FAKE + 8, msg="v must be 16-byte aligned"),
+    dict(vc=(128, 1, 1), msg="L = 1"),
+    dict(T=40, msg="exceed capacity"),
+])
+def test_encode_kv_rejects_bad_arguments(case):
+    kc = kvq.codec(*case.get("kc", (128, 128, 0)))
+    vc = kvq.codec(*case.get("vc", (128, 64, 1)))
+    K, V = _plane(), _plane(base=FAKE + (1 << 16))
+    rc = kvq.lib().kvq_encode_kv(C.byref(kc), FAKE, case.get("k", FAKE), C.byref(K), C.byref(vc),
+                                 FAKE, case.get("v", FAKE), C.byref(V), 1, 2, case.get("T", 4), 0,
+                                 None)
+    assert rc in (kvq.KVQ_EINVAL, kvq.KVQ_EUNSUPPORTED)
+    assert case["msg"] in kvq.kvq_last_error()
+
+
+def test_encode_kv_empty_is_ok_without_gpu():
+    kc, vc = kvq.codec(128, 128, 0), kvq.codec(128, 64, 1)
+    K, V = _plane(), _plane()
+    assert kvq.lib().kvq_encode_kv(C.byref(kc), None, None, C.byref(K), C.byref(vc), None, None,
+                                   C.byref(V), 0, 2, 4, 0, None) == 0
+    assert kvq.kvq_last_error() == ""
+
+
 def test_encode_and_dequant_empty_is_ok_without_gpu():
     c = kvq.codec(128, 128, 0)
     p = _plane()

@@ -126,6 +126,42 @@ def test_encode_append_one_token(dev):
     compare_codes(plane_rows(plane, t_range=(0, 40)), O.encode(x, s, L, O.MODE_LIN8))
 
 
+@pytest.mark.parametrize("T,pos0", [(37, 5), (1, 47)])
+def test_encode_kv_equals_two_encodes(dev, T, pos0):
+    """kvq_encode_kv writes exactly what kvq_encode writes for K and V
+    separately (a prefill slice and a one-token append), and both match the
+    oracle."""
+    d, B, H, cap = 128, 2, 3, 48
+    sk, sv = _signs(11, d), _signs(12, d)
+    k = _rand_x(B, H, T, d, seed=13)
+    v = _rand_x(B, H, T, d, seed=14, outliers=False)
+    kc, vc = kvq.codec(d, 128, O.MODE_LIN8), kvq.codec(d, 64, O.MODE_LOG4)
+    skd, svd = _dev_signs(sk), _dev_signs(sv)
+    kd, vd = torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda()
+    K1, V1 = kvq.alloc_plane(kc, B, H, cap), kvq.alloc_plane(vc, B, H, cap)
+    K2, V2 = kvq.alloc_plane(kc, B, H, cap), kvq.alloc_plane(vc, B, H, cap)
+    kvq.encode_kv(kc, skd, kd, K1, vc, svd, vd, V1, pos0)
+    kvq.encode(kc, skd, kd, K2, pos0)
+    kvq.encode(vc, svd, vd, V2, pos0)
+    torch.cuda.synchronize()
+    for w in range(3):
+        assert torch.equal(K1.rows(w), K2.rows(w))
+        assert torch.equal(V1.rows(w), V2.rows(w))
+    compare_codes(plane_rows(K1, t_range=(pos0, pos0 + T)), O.encode(k, sk, 128, O.MODE_LIN8))
+    compare_codes(plane_rows(V1, t_range=(pos0, pos0 + T)), O.encode(v, sv, 64, O.MODE_LOG4))
+
+
+def test_encode_kv_rejects_mismatched_head_dims(dev):
+    kc, vc = kvq.codec(128, 128, O.MODE_LIN8), kvq.codec(64, 64, O.MODE_LOG4)
+    K, V = kvq.alloc_plane(kc, 1, 1, 16), kvq.alloc_plane(vc, 1, 1, 16)
+    k = torch.zeros((1, 1, 1, 128), dtype=torch.float16, device="cuda")
+    v = torch.zeros((1, 1, 1, 64), dtype=torch.float16, device="cuda")
+    s = torch.ones(128, dtype=torch.int8, device="cuda")
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_encode_kv(kc, s, k, K.c(), vc, s, v, V.c(), 1, 1, 1, 0)
+    assert "head_dim" in str(e.value)
+
+
 def test_encode_edge_cases(dev):
     d = 128
     s = _signs(3, d)
