@@ -338,20 +338,22 @@ decode_kernel(DecodeArgs A) {
         for (; issued < NST - 1 && issued < ntiles_max; issued++) issue_tile(issued);
 
     // ---- everyone: tables and q' (overlaps the first copies) -----------------
-    // consecutive threads write consecutive replicas (no bank conflicts); the
-    // 16 threads of an entry compute the same value in the same instruction
+    // tabV follows tabK, so both tables are one array of nK + nV entries of
+    // kTabRep replicas.  Each bin centre is computed once, into replica 0;
+    // the other replicas are then copied by consecutive threads writing
+    // consecutive addresses (no bank conflicts).
 #pragma unroll 1
-    for (int idx = tid; idx < nK * kTabRep; idx += CONSUMERS) {
+    for (int e = tid; e < nK + nV; e += CONSUMERS) {
+        const bool isK = e < nK;
+        const int a = isK ? e : e - nK;
         float s, c;
-        sincospif((float)(2 * (idx / kTabRep) + 1) / (float)A.kc.L - 1.f, &s, &c);
-        tabK[idx] = make_float2(c, s);
+        sincospif((float)(2 * a + 1) / (float)(isK ? A.kc.L : A.vc.L) - 1.f, &s, &c);
+        tabK[e * kTabRep] = make_float2(c, s);
     }
+    __syncthreads();
 #pragma unroll 1
-    for (int idx = tid; idx < nV * kTabRep; idx += CONSUMERS) {
-        float s, c;
-        sincospif((float)(2 * (idx / kTabRep) + 1) / (float)A.vc.L - 1.f, &s, &c);
-        tabV[idx] = make_float2(c, s);
-    }
+    for (int idx = tid; idx < (nK + nV) * kTabRep; idx += CONSUMERS)
+        if (idx % kTabRep) tabK[idx] = tabK[idx - idx % kTabRep];
     for (int h = warp; h < G; h += WARPS) {
         const __half* qh = A.q + ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * D;
         float v[EPQ];
