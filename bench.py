@@ -80,6 +80,8 @@ def parse():
                         "--layer of --workload, or the prefill encode of 8 batch entries of "
                         "one layer; --steps launches after 3 warm-up launches")
     p.add_argument("--layer", type=int, default=0)
+    p.add_argument("--tensor", default="k", choices=["k", "v"],
+                   help="encode_layer case: encode the layer's K (8-bit linear norms) or V (4-bit log)")
     return p.parse_args()
 
 
@@ -486,16 +488,17 @@ def run_case(args):
         what = f"decode {w.name} layer {layer}, {S} splits"
     else:
         w = synth.WORKLOADS["prefill_32layers_b16_t8192_hkv8_d128"]
-        sk, _ = synth.layer_signs(w, 0)
-        c = kvq.codec(w.d, w.L_K[0], w.mode_K)
+        sk, sv = synth.layer_signs(w, 0)
+        isk = args.tensor == "k"
+        c = (kvq.codec(w.d, w.L_K[0], w.mode_K) if isk else kvq.codec(w.d, w.L_V[0], w.mode_V))
         nb = 8
         p = kvq.alloc_plane(c, nb, w.H_kv, w.ctx, device)
-        x = synth.kv(w, 0, synth.KIND_K, device=device, b_range=(0, nb))
-        skd = torch.from_numpy(sk).to(device)
+        x = synth.kv(w, 0, synth.KIND_K if isk else synth.KIND_V, device=device, b_range=(0, nb))
+        skd = torch.from_numpy(sk if isk else sv).to(device)
 
         def run():
             kvq.encode(c, skd, x, p, 0)
-        what = f"encode {w.name} layer 0 K, batch entries 0..{nb - 1}"
+        what = f"encode {w.name} layer 0 {'K' if isk else 'V'}, batch entries 0..{nb - 1}"
     for _ in range(3):
         run()
     torch.cuda.synchronize()
