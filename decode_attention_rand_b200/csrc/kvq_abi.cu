@@ -197,29 +197,27 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs, const kvq_plane* in
 }
 
 int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx, int32_t sm_count) {
-    // One CTA runs per SM.  Pick the fewest waves whose split count keeps at
-    // least 90% of the CTA slots busy, with at least 128 tokens per split;
-    // otherwise the most balanced choice within 8 waves.
+    // One CTA runs per SM, streaming tiles of about 128 tokens, and every CTA
+    // pays a fixed cost (prologue, merge, combine) of about three tiles.  The
+    // launch takes waves x (tiles per CTA + 3) tile times; pick the split
+    // count that minimises it, the fewer CTAs on ties.
     if (B <= 0 || H_kv <= 0 || max_ctx <= 0 || sm_count <= 0) return 1;
     const int64_t units = (int64_t)B * H_kv;
-    int64_t max_s = (max_ctx + 127) / 128;
-    if (max_s > 65535) max_s = 65535;
+    const int64_t tiles = (max_ctx + 127) / 128;
+    int64_t max_s = tiles < 65535 ? tiles : 65535;
+    // beyond eight waves the model's gains are noise
+    const int64_t wave_cap = (8 * (int64_t)sm_count + units - 1) / units;
+    if (max_s > wave_cap) max_s = wave_cap;
     if (max_s < 1) max_s = 1;
-    int64_t best = 1;
-    double best_eff = -1.0;
-    for (int64_t w = 1; w <= 8; w++) {
-        int64_t s = w * sm_count / units;
-        if (s < 1) s = 1;
-        if (s > max_s) s = max_s;
-        const int64_t ctas = units * s;
-        const int64_t waves = (ctas + sm_count - 1) / sm_count;
-        const double eff = (double)ctas / (double)(waves * sm_count);
-        if (eff >= 0.9) return (int32_t)s;
-        if (eff > best_eff + 1e-9) {
-            best_eff = eff;
+    int64_t best = 1, best_cost = -1;
+    for (int64_t s = 1; s <= max_s; s++) {
+        const int64_t waves = (units * s + sm_count - 1) / sm_count;
+        const int64_t per_cta = (tiles + s - 1) / s;
+        const int64_t cost = waves * (per_cta + 3);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
             best = s;
         }
-        if (s == max_s) break;
     }
     return (int32_t)best;
 }

@@ -149,6 +149,45 @@ __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
     return d;
 }
 
+// ---------------------------------------------------------- clusters ----
+
+// Barrier over every thread of every CTA of the cluster; release/acquire
+// make each CTA's shared-memory writes before it visible to the others after.
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile(
+        "barrier.cluster.arrive.release.aligned;\n\t"
+        "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory offset in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float dsmem_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float2 dsmem_f32x2(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float4 dsmem_f32x4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 // ------------------------------------------------------- group exchange --
 
 // Transpose-reduce over the NL lanes of a group: on return v[0..VF) holds the
@@ -641,6 +680,9 @@ decode_kernel(DecodeArgs A) {
     const int S = A.num_splits;
     float* stats = A.ws + ws_counter_floats(A.B, A.H_q);
     float* accs = stats + ws_stat_floats(A.B, A.H_q, S);
+    // clustered launch: this CTA's partial stays in its own shared memory,
+    // [G][D + 4] = acc[D], m, l (16-byte aligned rows)
+    float* part = hml + (2 * G + 3) / 4 * 4;
     // thread -> (h, k, lg, c) with (lg, c) fastest: consecutive threads read
     // consecutive floats of a row; element j = 2 (lg PP + k) + c
     for (int idx = tid; idx < G * D; idx += CONSUMERS) {
@@ -655,12 +697,79 @@ decode_kernel(DecodeArgs A) {
             a1 = fmaf(gl[(g + 1) * G + h], row[(g + 1) * 2 * NL], a1);
         }
         for (; g < NG; g++) a0 = fmaf(gl[g * G + h], row[g * 2 * NL], a0);
-        const int64_t slot = ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * S + split;
-        accs[slot * D + j] = a0 + a1;
-        if (j == 0) {
-            stats[slot * 2] = hml[2 * h];
-            stats[slot * 2 + 1] = hml[2 * h + 1];
+        if (A.cluster) {
+            part[h * (D + 4) + j] = a0 + a1;
+            if (j == 0) {
+                part[h * (D + 4) + D] = hml[2 * h];
+                part[h * (D + 4) + D + 1] = hml[2 * h + 1];
+            }
+        } else {
+            const int64_t slot = ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * S + split;
+            accs[slot * D + j] = a0 + a1;
+            if (j == 0) {
+                stats[slot * 2] = hml[2 * h];
+                stats[slot * 2 + 1] = hml[2 * h + 1];
+            }
         }
+    }
+
+    // ---- clustered launch: the splits of this (b, KV head) are one cluster
+    // and merge through distributed shared memory: cluster CTA r takes heads
+    // r, r + S, ... (one warp per head), reading every split's partial
+    if (A.cluster) {
+        cluster_barrier();
+        const uint32_t part_s = smem_u32(part);
+        for (int h = split + S * warp; h < G; h += S * WARPS) {
+            const int64_t hq = (int64_t)b * A.H_q + (int64_t)kvh * G + h;
+            const uint32_t row = part_s + (uint32_t)(h * (D + 4)) * 4u;
+            float m_l = -INFINITY, l_l = 0.f;  // lane s holds split s (S <= 32)
+            if (lane < S) {
+                const uint32_t rr = dsmem_addr(row, (uint32_t)lane);
+                m_l = dsmem_f32(rr + 4u * D);
+                l_l = dsmem_f32(rr + 4u * (D + 1));
+            }
+            const float mx = group_max<32>(m_l);
+            const float w_l = (lane < S && mx != -INFINITY) ? ex2(m_l - mx) : 0.f;
+            const float sl = group_sum<32>(w_l * l_l);
+            float v[EPQ];
+#pragma unroll
+            for (int e = 0; e < EPQ; e++) v[e] = 0.f;
+#pragma unroll 4
+            for (int sp = 0; sp < S; sp++) {
+                const float w = __shfl_sync(KVQ_FULL_MASK, w_l, sp);
+                const uint32_t ra = dsmem_addr(row, (uint32_t)sp) + 4u * (uint32_t)(lane * EPQ);
+                if constexpr (EPQ == 4) {
+                    const float4 x = dsmem_f32x4(ra);
+                    v[0] = fmaf(w, x.x, v[0]);
+                    v[1] = fmaf(w, x.y, v[1]);
+                    v[2] = fmaf(w, x.z, v[2]);
+                    v[3] = fmaf(w, x.w, v[3]);
+                } else {
+                    const float2 x = dsmem_f32x2(ra);
+                    v[0] = fmaf(w, x.x, v[0]);
+                    v[1] = fmaf(w, x.y, v[1]);
+                }
+            }
+            const float inv = sl > 0.f ? 1.f / sl : 0.f;
+#pragma unroll
+            for (int e = 0; e < EPQ; e++) v[e] *= inv;
+            fwht_local<EPQ>(v);
+            fwht_cross<EPQ, 32>(v, lane);
+            const float isd = rsqrtf((float)D);
+#pragma unroll
+            for (int e = 0; e < EPQ; e++) {
+                const int j = lane * EPQ + e;
+                float o = v[e] * isd;
+                o = A.signs_v[j] < 0 ? -o : o;
+                if (A.out_dtype == 0)
+                    reinterpret_cast<__half*>(A.out)[hq * D + j] = __float2half_rn(o);
+                else
+                    reinterpret_cast<float*>(A.out)[hq * D + j] = o;
+            }
+        }
+        // no CTA leaves while another may still read its partial
+        cluster_barrier();
+        return;
     }
 
     // ---- the last CTA of this (b, KV head) merges the splits ----------------
@@ -761,7 +870,8 @@ inline size_t decode_smem_plan(DecodeArgs& a) {
     a.stage_bytes = sb;
     const size_t merge =
         sizeof(float) * ((size_t)2 * Cfg::NG * G +
-                         (size_t)G * Cfg::PP * (Cfg::NG * 2 * Cfg::NL + 16) + 2 * (size_t)G);
+                         (size_t)G * Cfg::PP * (Cfg::NG * 2 * Cfg::NL + 16) +
+                         (size_t)(2 * G + 3) / 4 * 4 + (size_t)G * (D + 4));
     for (int ns = kMaxStages; ns >= 2; ns--) {
         size_t ring = (size_t)ns * sb;
         if (ring < merge) ring = merge;
@@ -773,23 +883,78 @@ inline size_t decode_smem_plan(DecodeArgs& a) {
     return 0;
 }
 
+// Largest cluster the combine uses (non-portable beyond 8 CTAs).
+constexpr int kMaxClusterSplits = 16;
+
 template <int D, int G, int BK, int BV>
 inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
     using Cfg = DecCfg<D, G>;
+    auto kernel = decode_kernel<D, G, BK, BV>;
     const size_t smem = decode_smem_plan<D, G>(a);
     if (smem == 0) return cudaErrorInvalidConfiguration;
     static bool attr_done[64] = {};
+    static int sm_count[64] = {};
+    // per device and split count: how many clusters of that many CTAs can be
+    // resident at once (-1 unknown)
+    static int cluster_max[64][kMaxClusterSplits + 1];
+    static bool cluster_init[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(decode_kernel<D, G, BK, BV>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    const bool cache = dev >= 0 && dev < 64;
+    if (!cache || !attr_done[dev]) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[dev] = true;
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        if (cache) {
+            sm_count[dev] = n;
+            if (!cluster_init[dev]) {
+                for (int k = 0; k <= kMaxClusterSplits; k++) cluster_max[dev][k] = -1;
+                cluster_init[dev] = true;
+            }
+            attr_done[dev] = true;
+        }
     }
     dim3 grid((unsigned)a.num_splits, (unsigned)a.H_kv, (unsigned)a.B);
-    decode_kernel<D, G, BK, BV><<<grid, Cfg::THREADS, smem, stream>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)a.num_splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    // the cluster combine pays off only when every cluster of the launch is
+    // resident at once (it saves the L2 round trip of the last-CTA combine);
+    // the GPC layout admits only a few large clusters at a time, so ask the
+    // occupancy calculator rather than count SMs
+    const int S = a.num_splits;
+    a.cluster = 0;
+    if (cache && S <= kMaxClusterSplits &&
+        (int64_t)a.B * a.H_kv * S <= (int64_t)sm_count[dev]) {
+        if (cluster_max[dev][S] < 0) {
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            const cudaError_t q = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+            if (q != cudaSuccess) {
+                (void)cudaGetLastError();
+                n = 0;
+            }
+            cluster_max[dev][S] = n;
+        }
+        a.cluster = (int64_t)a.B * a.H_kv <= (int64_t)cluster_max[dev][S];
+    }
+    cfg.attrs = a.cluster ? attr : nullptr;
+    cfg.numAttrs = a.cluster ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kernel, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

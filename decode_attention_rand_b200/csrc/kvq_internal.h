@@ -51,6 +51,8 @@ struct DecodeArgs {
     int stage_bytes;
     int stage_offset;
     int nstages;             // ring depth
+    int cluster;             // 1: the splits of a (b, KV head) form one thread-block
+                             // cluster and combine through distributed shared memory
 };
 
 // True when the decode kernels are built for this (head_dim, G, L_K, L_V)

@@ -173,8 +173,10 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs,
                 int64_t pos0, void* y, void* stream);
 
 /* Split count the library would choose for a decode launch (host logic,
- * deterministic): spreads B*H_kv*max_ctx over about two waves of CTAs on
- * sm_count SMs, at least 1 and at most ceil(max_ctx / 16). */
+ * deterministic).  One CTA per SM streams tiles of about 128 tokens and
+ * pays a fixed cost of about three tiles; the split count minimises
+ * waves x (tiles per CTA + 3) over at most eight waves on sm_count SMs,
+ * the fewer CTAs on ties.  At least 1, at most ceil(max_ctx / 128). */
 int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx,
                               int32_t sm_count);
 
@@ -207,7 +209,11 @@ int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim,
  * One kernel runs on `stream`: each CTA handles one (split, KV head, batch
  * entry); the last CTA of a (batch entry, KV head) to finish merges the
  * per-split softmax states, applies the inverse FWHT and D_V / sqrt(d) and
- * writes the output. */
+ * writes the output.  When num_splits <= 16 and every (batch entry, KV head)
+ * cluster of num_splits CTAs fits on the GPU at once, the splits of each
+ * (batch entry, KV head) run as one thread-block cluster instead and merge
+ * through distributed shared memory; the workspace is then not touched
+ * (it must still be passed). */
 int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc,
                     const int8_t* signs_k, const int8_t* signs_v,
                     const kvq_plane* K, const kvq_plane* V,
