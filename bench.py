@@ -265,7 +265,11 @@ class DecodeStep:
 
 def time_graph(state, K, W, dist_ctx):
     """Device time of exactly K steps replayed from CUDA graphs, plus the
-    average decode-launch duration from events captured in the graph."""
+    average decode-launch duration from events captured in a separate graph.
+
+    The timed graphs hold the steps' kernels only: an event node between the
+    append and the decode would cut the programmatic dependency that lets the
+    decode's setup overlap the append."""
     import torch
     stream = torch.cuda.Stream()
     for i in range(W):
@@ -273,25 +277,31 @@ def time_graph(state, K, W, dist_ctx):
     torch.cuda.synchronize()
     unit = max(1, min(K, state.nbuf * max(1, math.ceil(64 / state.nbuf))))
     n_full, rem = divmod(K, unit)
-    # external events become event-record nodes of the graph, so each decode
-    # launch is timed inside the replay
-    evs = [[[torch.cuda.Event(enable_timing=True, external=True),
-             torch.cuda.Event(enable_timing=True, external=True)]
-            for _ in state.layers] for _ in range(unit)]
     g_unit = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_unit, stream=stream):
         for i in range(unit):
-            state.step(i, evs[i], stream=torch.cuda.current_stream())
+            state.step(i, stream=torch.cuda.current_stream())
     g_rem = None
     if rem:
         g_rem = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_rem, stream=stream):
             for i in range(rem):
                 state.step(n_full * unit + i, stream=torch.cuda.current_stream())
+    # external events become event-record nodes of the graph, so each decode
+    # launch is timed inside the replay
+    n_ev = min(unit, 16)
+    evs = [[[torch.cuda.Event(enable_timing=True, external=True),
+             torch.cuda.Event(enable_timing=True, external=True)]
+            for _ in state.layers] for _ in range(n_ev)]
+    g_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ev, stream=stream):
+        for i in range(n_ev):
+            state.step(i, evs[i], stream=torch.cuda.current_stream())
     # one untimed replay uploads the graphs (extra warm-up)
     g_unit.replay()
     if g_rem:
         g_rem.replay()
+    g_ev.replay()
     torch.cuda.synchronize()
     barrier(dist_ctx)
     t_wall0 = time.time()
@@ -307,8 +317,12 @@ def time_graph(state, K, W, dist_ctx):
     t_wall1 = time.time()
     barrier(dist_ctx)
     ms = start.elapsed_time(end)
-    dec_ms = [evs[i][li][0].elapsed_time(evs[i][li][1]) for i in range(unit)
-              for li in range(len(state.layers))]
+    dec_ms = []
+    for _ in range(4):
+        g_ev.replay()
+        torch.cuda.synchronize()
+        dec_ms += [evs[i][li][0].elapsed_time(evs[i][li][1]) for i in range(n_ev)
+                   for li in range(len(state.layers))]
     return ms, statistics.fmean(dec_ms), (t_wall0, t_wall1)
 
 

@@ -118,6 +118,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// Wait until the grids this one depends on have completed and their memory
+// is visible (a no-op without a programmatic dependency).
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -333,8 +339,6 @@ decode_kernel(DecodeArgs A) {
     const int64_t t0 = (int64_t)split * A.split_len;
     const int64_t t1m = (t0 + A.split_len < lim) ? t0 + A.split_len : lim;
     const int ntiles_max = t1m > t0 ? (int)((t1m - t0 + kTT - 1) / kTT) : 0;
-    const int64_t ctx_in = A.ctx_len[b];
-
     if (tid == 0) {
         for (int s = 0; s < NST; s++) {
             mbar_init(&full[s], 1);
@@ -373,8 +377,15 @@ decode_kernel(DecodeArgs A) {
     };
     // tile t + NST - 1 is issued once tile t - 1 is released, so NST - 1 tiles
     // are in flight ahead of the one being consumed
-    if (tid == 0)
+    // Launched as a programmatic dependent of the previous kernel on the
+    // stream (typically the append of this step), the kernel may start
+    // before that one ends: nothing it reads from global memory (codes, q,
+    // ctx_len, signs) is touched before griddepcontrol.wait; the barrier setup
+    // and the cos/sin tables overlap the previous kernel's tail.
+    if (tid == 0) {
+        griddep_wait();
         for (; issued < NST - 1 && issued < ntiles_max; issued++) issue_tile(issued);
+    }
 
     // ---- everyone: tables and q' (overlaps the first copies) -----------------
     // tabV follows tabK, so both tables are one array of nK + nV entries of
@@ -393,6 +404,8 @@ decode_kernel(DecodeArgs A) {
 #pragma unroll 1
     for (int idx = tid; idx < (nK + nV) * kTabRep; idx += CONSUMERS)
         if (idx % kTabRep) tabK[idx] = tabK[idx - idx % kTabRep];
+    griddep_wait();
+    const int64_t ctx_in = A.ctx_len[b];
     for (int h = warp; h < G; h += WARPS) {
         const __half* qh = A.q + ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * D;
         float v[EPQ];
@@ -925,11 +938,14 @@ inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
     cfg.blockDim = dim3(Cfg::THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)a.num_splits;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch: see griddep_wait in the kernel
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     // the cluster combine pays off only when every cluster of the launch is
     // resident at once (it saves the L2 round trip of the last-CTA combine);
     // the GPC layout admits only a few large clusters at a time, so ask the
@@ -951,8 +967,8 @@ inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
         }
         a.cluster = (int64_t)a.B * a.H_kv <= (int64_t)cluster_max[dev][S];
     }
-    cfg.attrs = a.cluster ? attr : nullptr;
-    cfg.numAttrs = a.cluster ? 1 : 0;
+    cfg.attrs = a.cluster ? attr : attr + 1;
+    cfg.numAttrs = a.cluster ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kernel, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -728,6 +728,10 @@ __device__ __forceinline__ float angle_margin(const EncArgs& A) {
 template <int D>
 __global__ void __launch_bounds__(kEncWarps * 32, kEncBlocksPerSM)
 encode_kernel(EncPair PA) {
+    // a kernel launched as this one's programmatic dependent (the decode of
+    // the same step) may start its own setup now; it waits for this grid to
+    // finish before reading anything this grid writes
+    asm volatile("griddepcontrol.launch_dependents;");
     const EncArgs A = blockIdx.y ? PA.a[1] : PA.a[0];
     using Cfg = EncCfg<D>;
     constexpr int NL = Cfg::NL, PPL = Cfg::PPL, VPW = Cfg::VPW;
