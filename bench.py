@@ -2,11 +2,11 @@
 """Benchmark of the compressed-KV decode step (one JSON line on rank 0).
 
 A step is one pass of the whole hot path over one batch of synthetic input,
-for every layer of the workload: append the new token's K and V (one encode
-launch for both, T = 1, at the last cache slot) and run split-K decode
-attention over the whole compressed context (query rotation, scores from
-codes, online softmax, value accumulation in the rotated domain, combine,
-inverse rotation), two launches per layer.
+for every layer of the workload: append the new token's K and V (encode,
+T = 1, at the last cache slot) and run split-K decode attention over the
+whole compressed context (query rotation, scores from codes, online softmax,
+value accumulation in the rotated domain, combine, inverse rotation), in one
+kvq_decode_step launch per layer.
 
   value  decode-attention effective HBM GB/s = algorithmic bytes of the step
          (packed K/V codes + fp16 params read, q read, output written, the
@@ -245,20 +245,20 @@ class DecodeStep:
                                     knew=knew, vnew=vnew, out=out,
                                     cK=[p[0].c() for p in planes], cV=[p[1].c() for p in planes]))
         torch.cuda.synchronize(device)
-        self.kernels_per_step = 2 * w.layers  # K+V append, decode (splits + combine)
+        self.kernels_per_step = w.layers  # one fused append + decode launch per layer
 
     def step(self, i, ev=None, stream=None):
         kvq, w = self.kvq, self.w
         b = i % self.nbuf
         st = stream.cuda_stream if stream is not None else self.torch.cuda.current_stream().cuda_stream
         for li, L in enumerate(self.layers):
-            kvq.kvq_encode_kv(L["kc"], L["skd"], L["knew"], L["cK"][b], L["vc"], L["svd"],
-                              L["vnew"], L["cV"][b], w.B, w.H_kv, 1, w.ctx - 1, st)
             if ev is not None:
                 ev[li][0].record()
-            kvq.kvq_decode_attn(L["q"], L["kc"], L["vc"], L["skd"], L["svd"], L["cK"][b],
-                                L["cV"][b], self.ctx, w.B, w.H_q, w.H_kv, w.ctx, self.tau, self.S,
-                                self.ws.buf, self.ws.nbytes, self.err, L["out"], kvq.OUT_FP16, st)
+            # one kernel: append the new K and V at position ctx - 1, then attend
+            kvq.kvq_decode_step(L["q"], L["knew"], L["vnew"], L["kc"], L["vc"], L["skd"],
+                                L["svd"], L["cK"][b], L["cV"][b], self.ctx, w.B, w.H_q, w.H_kv,
+                                w.ctx, self.tau, self.S, self.ws.buf, self.ws.nbytes, self.err,
+                                L["out"], kvq.OUT_FP16, st)
             if ev is not None:
                 ev[li][1].record()
 
@@ -745,7 +745,7 @@ def main():
             "bytes_per_step": total_bytes,
         },
         "roofline": ({
-            "kernel": "decode_kernel (one kvq_decode_attn launch: splits and their combine)",
+            "kernel": "decode_kernel (one kvq_decode_step launch: append, splits and their combine)",
             "bound": "alu", "achieved": fp_achieved, "peak": fp_peak, "unit": "TFLOP/s",
             "frac": fp_achieved / fp_peak,
             "peak_kind": f"FP32 FMA pipe, derived: {FP32_LANES_PER_SM} lanes/SM x "
@@ -753,7 +753,7 @@ def main():
             "traffic": traffic, "flops_per_launch": dec_flops, "bytes_per_launch": dec_bytes,
             "us_per_launch": dec_ms * 1e3,
         } if fp_bound else {
-            "kernel": "decode_kernel (one kvq_decode_attn launch: splits and their combine)",
+            "kernel": "decode_kernel (one kvq_decode_step launch: append, splits and their combine)",
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
             "traffic": traffic, "bytes_per_launch": dec_bytes, "us_per_launch": dec_ms * 1e3,

@@ -229,49 +229,59 @@ int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim, int
                                      kvq::ws_acc_floats(B, H_q, num_splits, head_dim));
 }
 
-int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc, const int8_t* signs_k,
-                    const int8_t* signs_v, const kvq_plane* K, const kvq_plane* V,
-                    const int32_t* ctx_len, int32_t B, int32_t H_q, int32_t H_kv, int64_t max_ctx,
-                    float softmax_scale, int32_t num_splits, void* workspace, int64_t ws_bytes,
-                    int32_t* err_word, void* out, int32_t out_dtype, void* stream) {
-    kvq::DecodeArgs a;
-    int rc = check_codec(kc, "kvq_decode_attn (K)", &a.kc);
+}  // extern "C"
+
+namespace {
+
+// Argument checks and launch of a decode, with (kvq_decode_step) or without
+// (kvq_decode_attn) the fused append of the new token.
+int decode_impl(const char* what, const void* q, const void* k_new, const void* v_new,
+                const kvq_codec* kc, const kvq_codec* vc, const int8_t* signs_k,
+                const int8_t* signs_v, const kvq_plane* K, const kvq_plane* V,
+                const int32_t* ctx_len, int32_t B, int32_t H_q, int32_t H_kv, int64_t max_ctx,
+                float softmax_scale, int32_t num_splits, void* workspace, int64_t ws_bytes,
+                int32_t* err_word, void* out, int32_t out_dtype, void* stream) {
+    char wk[64], wv[64];
+    snprintf(wk, sizeof(wk), "%s (K)", what);
+    snprintf(wv, sizeof(wv), "%s (V)", what);
+    kvq::DecodeArgs a = {};
+    int rc = check_codec(kc, wk, &a.kc);
     if (rc) return rc;
-    rc = check_codec(vc, "kvq_decode_attn (V)", &a.vc);
+    rc = check_codec(vc, wv, &a.vc);
     if (rc) return rc;
-    rc = check_plane(K, "kvq_decode_attn (K)", &a.K);
+    rc = check_plane(K, wk, &a.K);
     if (rc) return rc;
-    rc = check_plane(V, "kvq_decode_attn (V)", &a.V);
+    rc = check_plane(V, wv, &a.V);
     if (rc) return rc;
-    if (a.kc.d != a.vc.d) return fail(KVQ_EINVAL, "kvq_decode_attn: K and V head_dim differ");
+    if (a.kc.d != a.vc.d) return fail(KVQ_EINVAL, "%s: K and V head_dim differ", what);
     if (a.K.capacity != a.V.capacity)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: K and V capacity differ");
+        return fail(KVQ_EINVAL, "%s: K and V capacity differ", what);
     if (B < 0 || H_q < 0 || H_kv < 0 || max_ctx < 0)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: negative size");
+        return fail(KVQ_EINVAL, "%s: negative size", what);
     if (B == 0 || H_q == 0) return ok();
     if (B > 65535 || H_kv > 65535)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: B and H_kv must be at most 65535");
+        return fail(KVQ_EINVAL, "%s: B and H_kv must be at most 65535", what);
     if (H_kv <= 0 || H_q % H_kv != 0)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: H_q %d is not a multiple of H_kv %d", H_q, H_kv);
+        return fail(KVQ_EINVAL, "%s: H_q %d is not a multiple of H_kv %d", what, H_q, H_kv);
     if (num_splits < 1 || num_splits > 65535)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: num_splits %d outside 1..65535", num_splits);
+        return fail(KVQ_EINVAL, "%s: num_splits %d outside 1..65535", what, num_splits);
     if (out_dtype != 0 && out_dtype != 1)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: out_dtype must be 0 (fp16) or 1 (fp32)");
+        return fail(KVQ_EINVAL, "%s: out_dtype must be 0 (fp16) or 1 (fp32)", what);
     if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: softmax_scale is not finite");
+        return fail(KVQ_EINVAL, "%s: softmax_scale is not finite", what);
     const int G = H_q / H_kv;
     if (!kvq::decode_supported(a.kc.d, G, a.kc.L, a.vc.L, a.kc.mode, a.vc.mode))
         return fail(KVQ_EUNSUPPORTED,
-                    "kvq_decode_attn: no kernel for head_dim %d, G %d, L_K %d, L_V %d "
+                    "%s: no kernel for head_dim %d, G %d, L_K %d, L_V %d "
                     "(built: head_dim 64/128, G 1/2/4/8, L <= 256)",
-                    a.kc.d, G, a.kc.L, a.vc.L);
+                    what, a.kc.d, G, a.kc.L, a.vc.L);
     const int64_t need = kvq_decode_workspace_bytes(B, H_q, a.kc.d, num_splits);
     if (!workspace || ws_bytes < need)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: workspace of %lld bytes is below the %lld needed",
+        return fail(KVQ_EINVAL, "%s: workspace of %lld bytes is below the %lld needed", what,
                     (long long)ws_bytes, (long long)need);
-    if (!aligned16(workspace)) return fail(KVQ_EINVAL, "kvq_decode_attn: workspace not 16-byte aligned");
+    if (!aligned16(workspace)) return fail(KVQ_EINVAL, "%s: workspace not 16-byte aligned", what);
     if (!q || !signs_k || !signs_v || !ctx_len || !out)
-        return fail(KVQ_EINVAL, "kvq_decode_attn: NULL q, signs, ctx_len or out");
+        return fail(KVQ_EINVAL, "%s: NULL q, signs, ctx_len or out", what);
     a.q = static_cast<const __half*>(q);
     a.signs_k = signs_k;
     a.signs_v = signs_v;
@@ -289,7 +299,41 @@ int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc, con
     a.err_word = err_word;
     a.out = out;
     a.out_dtype = out_dtype;
-    return cuda_status(kvq::launch_decode(a, static_cast<cudaStream_t>(stream)), "kvq_decode_attn");
+    a.k_new = static_cast<const __half*>(k_new);
+    a.v_new = static_cast<const __half*>(v_new);
+    if (k_new) {
+        a.enc_k = kvq::encode_args(a.kc, signs_k);
+        a.enc_v = kvq::encode_args(a.vc, signs_v);
+    }
+    return cuda_status(kvq::launch_decode(a, static_cast<cudaStream_t>(stream)), what);
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc, const int8_t* signs_k,
+                    const int8_t* signs_v, const kvq_plane* K, const kvq_plane* V,
+                    const int32_t* ctx_len, int32_t B, int32_t H_q, int32_t H_kv, int64_t max_ctx,
+                    float softmax_scale, int32_t num_splits, void* workspace, int64_t ws_bytes,
+                    int32_t* err_word, void* out, int32_t out_dtype, void* stream) {
+    return decode_impl("kvq_decode_attn", q, nullptr, nullptr, kc, vc, signs_k, signs_v, K, V,
+                       ctx_len, B, H_q, H_kv, max_ctx, softmax_scale, num_splits, workspace,
+                       ws_bytes, err_word, out, out_dtype, stream);
+}
+
+int kvq_decode_step(const void* q, const void* k_new, const void* v_new, const kvq_codec* kc,
+                    const kvq_codec* vc, const int8_t* signs_k, const int8_t* signs_v,
+                    const kvq_plane* K, const kvq_plane* V, const int32_t* ctx_len, int32_t B,
+                    int32_t H_q, int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                    int32_t num_splits, void* workspace, int64_t ws_bytes, int32_t* err_word,
+                    void* out, int32_t out_dtype, void* stream) {
+    if (!k_new || !v_new) return fail(KVQ_EINVAL, "kvq_decode_step: NULL k_new or v_new");
+    if (!aligned16(k_new) || !aligned16(v_new))
+        return fail(KVQ_EINVAL, "kvq_decode_step: k_new and v_new must be 16-byte aligned");
+    return decode_impl("kvq_decode_step", q, k_new, v_new, kc, vc, signs_k, signs_v, K, V,
+                       ctx_len, B, H_q, H_kv, max_ctx, softmax_scale, num_splits, workspace,
+                       ws_bytes, err_word, out, out_dtype, stream);
 }
 
 }  // extern "C"

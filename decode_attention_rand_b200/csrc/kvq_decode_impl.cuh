@@ -39,6 +39,7 @@
 //     splits, divides by l, applies the inverse FWHT and D_V / sqrt(d).
 #pragma once
 
+#include "kvq_encode_impl.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -124,6 +125,22 @@ __device__ __forceinline__ void griddep_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Arrive on named barrier `id` without waiting (the producer side).
+__device__ __forceinline__ void named_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Barrier over `count` threads (a multiple of 32) of the CTA, id 1..15.
+__device__ __forceinline__ void named_barrier(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Orders this thread's generic-proxy global writes before later async-proxy
+// (bulk copy) reads of them.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -132,27 +149,6 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-typedef unsigned long long f32x2;  // two packed fp32 lanes
-
-__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
-    f32x2 v;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
-    return v;
-}
-__device__ __forceinline__ float lo2(f32x2 v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float hi2(f32x2 v) { return __uint_as_float((uint32_t)(v >> 32)); }
-
-__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
-    f32x2 d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
-    f32x2 d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
 }
 
 // ---------------------------------------------------------- clusters ----
@@ -327,6 +323,7 @@ decode_kernel(DecodeArgs A) {
     float2* tabK = reinterpret_cast<float2*>(smem + 16 * kMaxStages + 16);  // [2^bK][16]
     float2* tabV = tabK + nK * kTabRep;                           // [2^bV][16]
     float* qs = reinterpret_cast<float*>(tabV + nV * kTabRep);    // [G][D]
+    uint32_t* encst = reinterpret_cast<uint32_t*>(qs + G * D);    // [2][kEncStageWords]
     unsigned char* stages = smem + A.stage_offset;                // [kStages][stage]
 
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -382,48 +379,94 @@ decode_kernel(DecodeArgs A) {
     // before that one ends: nothing it reads from global memory (codes, q,
     // ctx_len, signs) is touched before griddepcontrol.wait; the barrier setup
     // and the cos/sin tables overlap the previous kernel's tail.
+    // Fused append (kvq_decode_step): the split holding the new token (position
+    // ctx_len[b] - 1) encodes it with warps 0 and 1 while the other warps build
+    // the tables and rotate q; the tile holding it, and the ones after, are
+    // copied in only after it is written.  Without an append all warps share
+    // the tables and q.
+    const bool fused = A.k_new != nullptr;
+    const int w0 = fused ? 2 : 0;  // first warp of the table / q' work
+    int64_t ctx_in = 0;
+    bool append = false;           // warps 0 and 1 of a fused launch
+    if (fused && warp < 2) {
+        griddep_wait();
+        ctx_in = A.ctx_len[b];
+        append = ctx_in >= 1 && ctx_in <= lim && ctx_in - 1 >= t0 && ctx_in - 1 < t1m;
+    }
     if (tid == 0) {
         griddep_wait();
-        for (; issued < NST - 1 && issued < ntiles_max; issued++) issue_tile(issued);
+        const int hold = append ? (int)((ctx_in - 1 - t0) / kTT) : ntiles_max;
+        for (; issued < NST - 1 && issued < ntiles_max && issued < hold; issued++) issue_tile(issued);
+    }
+    if (fused && warp < 2) {
+        if (append) {
+            // the same encode_tile as kvq_encode, one vector per warp
+            using ECfg = EncCfg<D>;
+            EncArgs E = warp == 0 ? A.enc_k : A.enc_v;
+            const PlaneDev& pl = warp == 0 ? A.K : A.V;
+            const int64_t bh = (int64_t)b * A.H_kv + kvh;
+            E.x = (warp == 0 ? A.k_new : A.v_new) + bh * D;
+            E.n_vec = 1;
+            E.T = 1;
+            E.pos0 = ctx_in - 1;
+            E.out.angles = pl.angles + bh * pl.capacity * (int64_t)E.c.angle_words * 4;
+            E.out.norms = pl.norms + bh * pl.capacity * (int64_t)E.c.norm_bytes;
+            E.out.params = pl.params + bh * pl.capacity * (int64_t)E.c.param_bytes;
+            E.out.capacity = pl.capacity;
+            uint32_t* est = encst + warp * kEncStageWords;
+            for (int i = lane; i < kEncStageWords; i += 32) est[i] = 0u;
+            __syncwarp();
+            const int elg = lane % ECfg::NL, egrp = lane / ECfg::NL;
+            uint32_t smask[ECfg::PPL];
+            lane_sign_masks<D>(E.signs, elg, smask);
+            (void)encode_tile<D, true>(E, 0, smask, est, angle_margin(E), lane, egrp, elg);
+            fence_proxy_async_global();
+        }
+        named_barrier(1, 64);
+        if (tid == 0 && append)
+            for (; issued < NST - 1 && issued < ntiles_max; issued++) issue_tile(issued);
     }
 
-    // ---- everyone: tables and q' (overlaps the first copies) -----------------
+    // ---- tables and q' (overlap the first copies and the append) -------------
     // tabV follows tabK, so both tables are one array of nK + nV entries of
     // kTabRep replicas.  Each bin centre is computed once, into replica 0;
     // the other replicas are then copied by consecutive threads writing
     // consecutive addresses (no bank conflicts).
+    if (warp >= w0) {
+        const int nthr = CONSUMERS - 32 * w0, t = tid - 32 * w0;
 #pragma unroll 1
-    for (int e = tid; e < nK + nV; e += CONSUMERS) {
-        const bool isK = e < nK;
-        const int a = isK ? e : e - nK;
-        float s, c;
-        sincospif((float)(2 * a + 1) / (float)(isK ? A.kc.L : A.vc.L) - 1.f, &s, &c);
-        tabK[e * kTabRep] = make_float2(c, s);
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int idx = tid; idx < (nK + nV) * kTabRep; idx += CONSUMERS)
-        if (idx % kTabRep) tabK[idx] = tabK[idx - idx % kTabRep];
-    griddep_wait();
-    const int64_t ctx_in = A.ctx_len[b];
-    for (int h = warp; h < G; h += WARPS) {
-        const __half* qh = A.q + ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * D;
-        float v[EPQ];
-#pragma unroll
-        for (int e = 0; e < EPQ; e++) {
-            const int j = lane * EPQ + e;
-            const float f = __half2float(qh[j]);
-            v[e] = A.signs_k[j] < 0 ? -f : f;
+        for (int e = t; e < nK + nV; e += nthr) {
+            const bool isK = e < nK;
+            const int a = isK ? e : e - nK;
+            float s, c;
+            sincospif((float)(2 * a + 1) / (float)(isK ? A.kc.L : A.vc.L) - 1.f, &s, &c);
+            tabK[e * kTabRep] = make_float2(c, s);
         }
-        fwht_local<EPQ>(v);
-        fwht_cross<EPQ, 32>(v, lane);
-        const float isd = rsqrtf((float)D);
-        if constexpr (EPQ == 4) {
-            reinterpret_cast<float4*>(qs + h * D)[lane] =
-                make_float4(v[0] * isd, v[1] * isd, v[2] * isd, v[3] * isd);
-        } else {
+        named_barrier(2, nthr);
+#pragma unroll 1
+        for (int idx = t; idx < (nK + nV) * kTabRep; idx += nthr)
+            if (idx % kTabRep) tabK[idx] = tabK[idx - idx % kTabRep];
+        griddep_wait();
+        ctx_in = A.ctx_len[b];
+        for (int h = warp - w0; h < G; h += WARPS - w0) {
+            const __half* qh = A.q + ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * D;
+            float v[EPQ];
 #pragma unroll
-            for (int e = 0; e < EPQ; e++) qs[h * D + lane * EPQ + e] = v[e] * isd;
+            for (int e = 0; e < EPQ; e++) {
+                const int j = lane * EPQ + e;
+                const float f = __half2float(qh[j]);
+                v[e] = A.signs_k[j] < 0 ? -f : f;
+            }
+            fwht_local<EPQ>(v);
+            fwht_cross<EPQ, 32>(v, lane);
+            const float isd = rsqrtf((float)D);
+            if constexpr (EPQ == 4) {
+                reinterpret_cast<float4*>(qs + h * D)[lane] =
+                    make_float4(v[0] * isd, v[1] * isd, v[2] * isd, v[3] * isd);
+            } else {
+#pragma unroll
+                for (int e = 0; e < EPQ; e++) qs[h * D + lane * EPQ + e] = v[e] * isd;
+            }
         }
     }
     int64_t ctx = ctx_in;
@@ -437,7 +480,18 @@ decode_kernel(DecodeArgs A) {
     const int nloop = ntiles > (NST - 1 < ntiles_max ? NST - 1 : ntiles_max)
                           ? ntiles
                           : (NST - 1 < ntiles_max ? NST - 1 : ntiles_max);
-    __syncthreads();
+    if (fused) {
+        // the table / q' warps start on the tiles at once; the append warps
+        // join when done (barrier 3: the others only arrive, they do not wait)
+        if (warp >= w0) {
+            named_barrier(2, CONSUMERS - 32 * w0);
+            named_arrive(3, CONSUMERS);
+        } else {
+            named_barrier(3, CONSUMERS);
+        }
+    } else {
+        __syncthreads();
+    }
 
     const int grp = lane / NL, lg = lane % NL;
     const int gidx = warp * GPW + grp;
@@ -869,7 +923,7 @@ inline size_t decode_smem_plan(DecodeArgs& a) {
     using Cfg = DecCfg<D, G>;
     size_t off = 16 * kMaxStages + 16 +
                  sizeof(float2) * kTabRep * (size_t)((1 << a.kc.bits) + (1 << a.vc.bits)) +
-                 sizeof(float) * G * D;
+                 sizeof(float) * G * D + sizeof(uint32_t) * 2 * kEncStageWords;
     off = (off + 15) / 16 * 16;
     a.stage_offset = (int)off;
     const int rb[6] = {a.kc.angle_words * 4, a.kc.norm_bytes, a.kc.param_bytes,

@@ -30,6 +30,22 @@ cudaError_t launch_dequant(const CodecDev& c, const int8_t* signs, const PlaneDe
                            int64_t n_vec, int64_t T, int64_t pos0, __half* y, int sm_count,
                            cudaStream_t stream);
 
+// One encode job as the kernels see it (built on the host by make_args).
+struct EncArgs {
+    const __half* x;
+    const int8_t* signs;
+    int64_t n_vec;
+    int64_t T;
+    int64_t pos0;
+    CodecDev c;
+    PlaneDev out;
+    float inv_sqrt_d;
+    float bins_per_rad;  // L / (2 pi)
+};
+
+// Codec-wide part of an encode job (x, n_vec, T, pos0 and out left empty).
+EncArgs encode_args(const CodecDev& c, const int8_t* signs);
+
 struct DecodeArgs {
     const __half* q;        // [B][H_q][d]
     CodecDev kc, vc;
@@ -53,6 +69,11 @@ struct DecodeArgs {
     int nstages;             // ring depth
     int cluster;             // 1: the splits of a (b, KV head) form one thread-block
                              // cluster and combine through distributed shared memory
+    // fused append (kvq_decode_step): the new token of every (b, KV head),
+    // encoded by the CTA whose split holds position ctx_len[b] - 1
+    const __half* k_new;     // [B][H_kv][d] or NULL (no append)
+    const __half* v_new;     // [B][H_kv][d]
+    EncArgs enc_k, enc_v;    // codec, signs and constants of the two encodes
 };
 
 // True when the decode kernels are built for this (head_dim, G, L_K, L_V)

@@ -64,6 +64,12 @@ _SIGNATURES = {
                                           C.POINTER(kvq_plane), C.c_void_p, C.c_int32, C.c_int32,
                                           C.c_int32, C.c_int64, C.c_float, C.c_int32, C.c_void_p,
                                           C.c_void_p, C.c_int32, C.c_void_p]),
+    "kvq_decode_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.POINTER(kvq_codec),
+                                  C.POINTER(kvq_codec), C.c_void_p, C.c_void_p,
+                                  C.POINTER(kvq_plane), C.POINTER(kvq_plane), C.c_void_p,
+                                  C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_float, C.c_int32,
+                                  C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int32,
+                                  C.c_void_p]),
     "kvq_decode_attn": (C.c_int, [C.c_void_p, C.POINTER(kvq_codec), C.POINTER(kvq_codec),
                                   C.c_void_p, C.c_void_p, C.POINTER(kvq_plane),
                                   C.POINTER(kvq_plane), C.c_void_p, C.c_int32, C.c_int32,
@@ -162,6 +168,17 @@ def kvq_decode_num_splits(B: int, H_kv: int, max_ctx: int, sm_count: int) -> int
 
 def kvq_decode_workspace_bytes(B: int, H_q: int, head_dim: int, num_splits: int) -> int:
     return lib().kvq_decode_workspace_bytes(B, H_q, head_dim, num_splits)
+
+
+def kvq_decode_step(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v,
+                    K: kvq_plane, V: kvq_plane, ctx_len, B: int, H_q: int, H_kv: int,
+                    max_ctx: int, softmax_scale: float, num_splits: int, workspace, ws_bytes: int,
+                    err_word, out, out_dtype: int, stream=None):
+    _check(lib().kvq_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), C.byref(kc), C.byref(vc),
+                                 _ptr(signs_k), _ptr(signs_v), C.byref(K), C.byref(V),
+                                 _ptr(ctx_len), B, H_q, H_kv, max_ctx, softmax_scale, num_splits,
+                                 _ptr(workspace), ws_bytes, _ptr(err_word), _ptr(out), out_dtype,
+                                 _stream(stream)))
 
 
 def kvq_decode_attn(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: kvq_plane,
@@ -279,4 +296,28 @@ def decode_attn(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: Plane, V: 
     kvq_decode_attn(q, kc, vc, signs_k, signs_v, K.c(), V.c(), ctx_len, B, H_q, K.H_kv, max_ctx,
                     softmax_scale, num_splits, workspace.buf, workspace.nbytes, err_word, out,
                     out_dtype, stream)
+    return out
+
+
+def decode_step(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: Plane,
+                V: Plane, ctx_len, max_ctx: int, softmax_scale: float | None = None,
+                num_splits=None, workspace: DecodeWorkspace | None = None, err_word=None, out=None,
+                out_dtype: int = OUT_FP32, stream=None):
+    """Append k_new / v_new [B, H_kv, d] at position ctx_len[b] - 1 and attend
+    q over positions 0 .. ctx_len[b] - 1, in one kernel."""
+    import torch
+    B, H_q, d = q.shape
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    if num_splits is None:
+        sm = torch.cuda.get_device_properties(q.device).multi_processor_count
+        num_splits = kvq_decode_num_splits(B, K.H_kv, max_ctx, sm)
+    if workspace is None or workspace.num_splits != num_splits:
+        workspace = DecodeWorkspace(B, H_q, d, num_splits, q.device)
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.float16 if out_dtype == OUT_FP16
+                          else torch.float32, device=q.device)
+    kvq_decode_step(q, k_new, v_new, kc, vc, signs_k, signs_v, K.c(), V.c(), ctx_len, B, H_q,
+                    K.H_kv, max_ctx, softmax_scale, num_splits, workspace.buf, workspace.nbytes,
+                    err_word, out, out_dtype, stream)
     return out

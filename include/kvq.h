@@ -223,6 +223,30 @@ int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc,
                     int32_t* err_word, void* out, int32_t out_dtype,
                     void* stream);
 
+/* One decode step of one layer in one kernel: the append of each sequence's
+ * new token fused into kvq_decode_attn.  For every b with 1 <= ctx_len[b]
+ * <= min(max_ctx, capacity), the token at position ctx_len[b] - 1 of every
+ * KV head is first written as
+ *   kvq_encode_kv(kc, signs_k, k_new[b], K, vc, signs_v, v_new[b], V, ...)
+ * would write it (same codes, byte for byte), then attention runs over
+ * positions 0 .. ctx_len[b] - 1, the new token included, exactly as
+ * kvq_decode_attn.  The TurboAngle abstract encodes K and V on arrival and
+ * attends from codes; doing both in one launch is this library's choice:
+ * the split that holds the new token encodes it while its first tiles are
+ * in flight, the other splits never wait for it.
+ *   k_new, v_new  device fp16 [B][H_kv][head_dim], 16-byte aligned
+ * Everything else as for kvq_decode_attn.  A ctx_len outside the range
+ * above appends nothing (and is clipped and reported as there). */
+int kvq_decode_step(const void* q, const void* k_new, const void* v_new,
+                    const kvq_codec* kc, const kvq_codec* vc,
+                    const int8_t* signs_k, const int8_t* signs_v,
+                    const kvq_plane* K, const kvq_plane* V,
+                    const int32_t* ctx_len, int32_t B, int32_t H_q,
+                    int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                    int32_t num_splits, void* workspace, int64_t ws_bytes,
+                    int32_t* err_word, void* out, int32_t out_dtype,
+                    void* stream);
+
 /* Size of the scratch array built into the library for
  * kvq_decode_attn_noalloc (4 MiB of device memory per GPU that loads it). */
 #define KVQ_NOALLOC_SCRATCH_BYTES (4u << 20)

@@ -165,6 +165,32 @@ def test_decode_rejects_bad_arguments(kw, status, msg):
     assert msg in kvq.kvq_last_error()
 
 
+@pytest.mark.parametrize("k,v,msg", [
+    (None, FAKE, "NULL k_new"),
+    (FAKE + 8, FAKE, "16-byte aligned"),
+    (FAKE, FAKE + 4, "16-byte aligned"),
+])
+def test_decode_step_rejects_bad_new_tokens(k, v, msg):
+    kc, vc = kvq.codec(128, 128, 0), kvq.codec(128, 64, 1)
+    K, V = _plane(), _plane()
+    ws = kvq.kvq_decode_workspace_bytes(1, 8, 128, 2)
+    rc = kvq.lib().kvq_decode_step(FAKE, k, v, C.byref(kc), C.byref(vc), FAKE, FAKE, C.byref(K),
+                                   C.byref(V), FAKE, 1, 8, 2, 32, 0.1, 2, FAKE, ws, None, FAKE, 0,
+                                   None)
+    assert rc == kvq.KVQ_EINVAL
+    assert msg in kvq.kvq_last_error()
+
+
+def test_decode_step_shares_the_decode_checks():
+    kc, vc = kvq.codec(128, 128, 0), kvq.codec(64, 64, 1)
+    K, V = _plane(), _plane()
+    rc = kvq.lib().kvq_decode_step(FAKE, FAKE, FAKE, C.byref(kc), C.byref(vc), FAKE, FAKE,
+                                   C.byref(K), C.byref(V), FAKE, 1, 8, 2, 32, 0.1, 2, FAKE, 1 << 20,
+                                   None, FAKE, 0, None)
+    assert rc == kvq.KVQ_EINVAL
+    assert "kvq_decode_step: K and V head_dim differ" in kvq.kvq_last_error()
+
+
 def test_error_state_is_per_thread():
     import threading
     c = kvq.codec(128, 1, 0)

@@ -292,6 +292,73 @@ def test_decode_split_invariance(dev):
         assert rel_l2(o, outs[0]).max() < 1e-5
 
 
+@pytest.mark.parametrize("ctx_lens,splits,H_kv,G", [
+    ([300, 129, 1, 0], None, 2, 4),   # ragged, a one-token sequence, an empty one
+    ([256, 128], 2, 2, 4),            # new token on the first row of a tile / of a split
+    ([257, 200], 3, 2, 4),
+    ([4096], None, 8, 4),             # the Llama-shaped layer
+    ([1000, 513], 1, 1, 8),           # one split: the held tile is not the first
+])
+def test_decode_step_equals_append_then_decode(dev, ctx_lens, splits, H_kv, G):
+    """kvq_decode_step writes the new token's codes exactly as kvq_encode_kv
+    does and returns exactly what kvq_decode_attn returns on the appended
+    cache; the appended cache also matches the oracle."""
+    d, B = 128, len(ctx_lens)
+    H_q = G * H_kv
+    cap = (max(ctx_lens) + 16 + 15) // 16 * 16
+    sk, sv = _signs(31, d), _signs(32, d)
+    k = _rand_x(B, H_kv, cap, d, seed=33)
+    v = _rand_x(B, H_kv, cap, d, seed=34, outliers=False)
+    kc, vc = kvq.codec(d, 128, O.MODE_LIN8), kvq.codec(d, 64, O.MODE_LOG4)
+    skd, svd = _dev_signs(sk), _dev_signs(sv)
+    kd, vd = torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda()
+    # reference: every position encoded; step: the new positions blanked first
+    Kr, Vr = kvq.alloc_plane(kc, B, H_kv, cap), kvq.alloc_plane(vc, B, H_kv, cap)
+    Ks, Vs = kvq.alloc_plane(kc, B, H_kv, cap), kvq.alloc_plane(vc, B, H_kv, cap)
+    for P, c, x, sg in ((Kr, kc, kd, skd), (Vr, vc, vd, svd), (Ks, kc, kd, skd), (Vs, vc, vd, svd)):
+        kvq.encode(c, sg, x, P, 0)
+    k_new = torch.zeros((B, H_kv, d), dtype=torch.float16, device="cuda")
+    v_new = torch.zeros_like(k_new)
+    for b, n in enumerate(ctx_lens):
+        if n >= 1:
+            k_new[b] = kd[b, :, n - 1]
+            v_new[b] = vd[b, :, n - 1]
+            for P in (Ks, Vs):
+                for w in range(3):
+                    P.rows(w)[b, :, n - 1] = 0xA5
+    ctx = torch.tensor(ctx_lens, dtype=torch.int32, device="cuda")
+    q = torch.from_numpy(np.random.default_rng(35).standard_normal((B, H_q, d)).astype(np.float16)).cuda()
+    maxc = max(ctx_lens)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out_s = kvq.decode_step(q, k_new, v_new, kc, vc, skd, svd, Ks, Vs, ctx, maxc, num_splits=splits,
+                            err_word=err)
+    out_r = kvq.decode_attn(q, kc, vc, skd, svd, Kr, Vr, ctx, maxc, num_splits=splits)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for w in range(3):
+        assert torch.equal(Ks.rows(w), Kr.rows(w)), ("K", w)
+        assert torch.equal(Vs.rows(w), Vr.rows(w)), ("V", w)
+    assert torch.equal(out_s, out_r)
+    compare_codes(plane_rows(Ks, t_range=(0, cap)), O.encode(k, sk, 128, O.MODE_LIN8))
+    compare_codes(plane_rows(Vs, t_range=(0, cap)), O.encode(v, sv, 64, O.MODE_LOG4))
+
+
+def test_decode_step_clipped_context_appends_nothing(dev):
+    d, B, H_kv, cap = 128, 1, 2, 64
+    kc, vc = kvq.codec(d, 128, O.MODE_LIN8), kvq.codec(d, 64, O.MODE_LOG4)
+    K, V = kvq.alloc_plane(kc, B, H_kv, cap), kvq.alloc_plane(vc, B, H_kv, cap)
+    s = _dev_signs(_signs(36, d))
+    k_new = torch.ones((B, H_kv, d), dtype=torch.float16, device="cuda")
+    q = torch.ones((B, 4 * H_kv, d), dtype=torch.float16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ctx = torch.tensor([cap + 5], dtype=torch.int32, device="cuda")
+    kvq.decode_step(q, k_new, k_new, kc, vc, s, s, K, V, ctx, cap, err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & kvq.KVQ_DEVERR_CTX_RANGE
+    for w in range(3):
+        assert int(K.rows(w).count_nonzero()) == 0 and int(V.rows(w).count_nonzero()) == 0
+
+
 def test_decode_fp16_output_and_scale(dev):
     got, want, _ = run_decode_case(2, 16, 2, 128, [250, 99], 128, 64, seed=6,
                                    out_dtype=kvq.OUT_FP16, q_scale=3.0, tau=0.2)
