@@ -721,6 +721,12 @@ def main():
     world = ctx["world"]
     value = world * total_bytes * args.steps / (ms / 1e3) / 1e9
     e2e = world * total_bytes * e2e_n / (e2e_ms / 1e3) / 1e9
+    # the step is one kvq_decode_step launch per layer, so the timed region's
+    # device time over its launches is the kernel's average launch duration;
+    # dec_ms (event nodes around each launch, which add their own dispatch
+    # gaps) is reported beside it
+    dec_ms_isolated = dec_ms
+    dec_ms = ms / (args.steps * w.layers)
     dec_bytes = statistics.fmean(per_layer)
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
     dec_flops = w.B * w.H_kv * w.ctx * decode_flops_per_token_head(w.d, w.G)
@@ -751,12 +757,13 @@ def main():
             "peak_kind": f"FP32 FMA pipe, derived: {FP32_LANES_PER_SM} lanes/SM x "
                          f"{props.multi_processor_count} SMs x 2 flop x {sm_mhz:.0f} MHz",
             "traffic": traffic, "flops_per_launch": dec_flops, "bytes_per_launch": dec_bytes,
-            "us_per_launch": dec_ms * 1e3,
+            "us_per_launch": dec_ms * 1e3, "us_per_launch_event_bracketed": dec_ms_isolated * 1e3,
         } if fp_bound else {
             "kernel": "decode_kernel (one kvq_decode_step launch: append, splits and their combine)",
             "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
             "traffic": traffic, "bytes_per_launch": dec_bytes, "us_per_launch": dec_ms * 1e3,
+            "us_per_launch_event_bracketed": dec_ms_isolated * 1e3,
         }),
         "roofline_hbm": {
             "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
