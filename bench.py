@@ -648,6 +648,13 @@ def max_over_ranks(ctx, value):
     return float(t.item())
 
 
+def workload_config(w) -> dict:
+    """The workload part of the JSON line's config, shared by both arms."""
+    return {"workload": w.name, "layers": w.layers, "batch": w.B, "H_q": w.H_q, "H_kv": w.H_kv,
+            "head_dim": w.d, "ctx": w.ctx, "L_K": sorted(set(w.L_K)), "L_V": sorted(set(w.L_V)),
+            "norms": "K lin8, V log4"}
+
+
 def run_reference(args, w):
     """The reference arm: the fp64 oracle on the host cores, K timed steps of
     a bounded sample each, the whole run kept to a few minutes."""
@@ -661,7 +668,7 @@ def run_reference(args, w):
         "metric": METRIC, "value": gbs, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(args.steps, 1) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name},
+        "data": "synthetic", "config": workload_config(w),
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": ors.threads, "kind": "oracle",
                          "sample": ors.describe(args.steps)},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -742,9 +749,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {
-            "workload": w.name, "layers": w.layers, "batch": w.B, "H_q": w.H_q, "H_kv": w.H_kv,
-            "head_dim": w.d, "ctx": w.ctx, "L_K": sorted(set(w.L_K)), "L_V": sorted(set(w.L_V)),
-            "norms": "K lin8, V log4", "num_splits": state.S, "out": "fp16",
+            **workload_config(w), "num_splits": state.S, "out": "fp16",
             "l2": f"inputs larger than L2: {state.nbuf} rotated cache copies "
                   f"({state.nbuf * sum(per_layer) / 2**20:.0f} MiB per cycle, L2 {l2 / 2**20:.0f} MiB)",
             "timing": "CUDA graph replay, CUDA events, max over ranks",
