@@ -68,6 +68,35 @@ int check_plane(const kvq_plane* p, const char* what, kvq::PlaneDev* out) {
     out->norms = static_cast<uint8_t*>(p->norms);
     out->params = static_cast<uint8_t*>(p->params);
     out->capacity = p->capacity;
+    out->H_kv = 0;  // set by the call
+    out->pages = nullptr;
+    out->page_tokens = 0;
+    out->max_pages = 0;
+    out->num_pages = 0;
+    return KVQ_OK;
+}
+
+// Validate a paged plane and fill the device descriptor.
+int check_paged_plane(const kvq_paged_plane* p, const char* what, kvq::PlaneDev* out) {
+    if (!p) return fail(KVQ_EINVAL, "%s: paged plane is NULL", what);
+    if (!p->angles || !p->norms || !p->params || !p->pages)
+        return fail(KVQ_EINVAL, "%s: NULL pool or page table", what);
+    if (!aligned16(p->angles) || !aligned16(p->norms) || !aligned16(p->params))
+        return fail(KVQ_EINVAL, "%s: pools must be 16-byte aligned", what);
+    if (p->page_tokens <= 0 || p->page_tokens % 128 != 0)
+        return fail(KVQ_EINVAL, "%s: page_tokens %d must be a positive multiple of 128", what,
+                    p->page_tokens);
+    if (p->max_pages <= 0 || p->num_pages <= 0)
+        return fail(KVQ_EINVAL, "%s: max_pages and num_pages must be positive", what);
+    out->angles = static_cast<uint8_t*>(p->angles);
+    out->norms = static_cast<uint8_t*>(p->norms);
+    out->params = static_cast<uint8_t*>(p->params);
+    out->capacity = (int64_t)p->max_pages * p->page_tokens;
+    out->H_kv = 0;
+    out->pages = p->pages;
+    out->page_tokens = p->page_tokens;
+    out->max_pages = p->max_pages;
+    out->num_pages = p->num_pages;
     return KVQ_OK;
 }
 
@@ -123,11 +152,13 @@ namespace {
 // to encode.
 int prep_encode(const kvq_codec* codec, const int8_t* signs, const void* x, int32_t B,
                 int32_t H_kv, int32_t T, int64_t pos0, const kvq_plane* out, const char* what,
-                const char* xname, kvq::EncodeJob* job) {
+                const char* xname, kvq::EncodeJob* job, const kvq_paged_plane* paged = nullptr) {
     int rc = check_codec(codec, what, &job->c);
     if (rc) return rc;
-    rc = check_plane(out, what, &job->out);
+    rc = paged ? check_paged_plane(paged, what, &job->out) : check_plane(out, what, &job->out);
     if (rc) return rc;
+    job->out.H_kv = H_kv;
+    job->err_word = nullptr;
     if (B < 0 || H_kv < 0 || T < 0) return fail(KVQ_EINVAL, "%s: negative size", what);
     if (pos0 < 0 || pos0 + (int64_t)T > job->out.capacity)
         return fail(KVQ_EINVAL, "%s: tokens [%lld, %lld) exceed capacity %lld", what,
@@ -173,6 +204,27 @@ int kvq_encode_kv(const kvq_codec* kc, const int8_t* signs_k, const void* k, con
     return cuda_status(kvq::launch_encode_jobs(j, 2, sm_count_current(),
                                                static_cast<cudaStream_t>(stream)),
                        "kvq_encode_kv");
+}
+
+int kvq_encode_kv_paged(const kvq_codec* kc, const int8_t* signs_k, const void* k,
+                        const kvq_paged_plane* K, const kvq_codec* vc, const int8_t* signs_v,
+                        const void* v, const kvq_paged_plane* V, int32_t B, int32_t H_kv,
+                        int32_t T, int64_t pos0, int32_t* err_word, void* stream) {
+    kvq::EncodeJob j[2];
+    int rc = prep_encode(kc, signs_k, k, B, H_kv, T, pos0, nullptr, "kvq_encode_kv_paged", "k",
+                         &j[0], K);
+    if (rc) return rc;
+    rc = prep_encode(vc, signs_v, v, B, H_kv, T, pos0, nullptr, "kvq_encode_kv_paged", "v", &j[1],
+                     V);
+    if (rc) return rc;
+    if (j[0].c.d != j[1].c.d)
+        return fail(KVQ_EINVAL, "kvq_encode_kv_paged: K head_dim %d differs from V head_dim %d",
+                    j[0].c.d, j[1].c.d);
+    if (j[0].n_vec == 0) return ok();
+    j[0].err_word = j[1].err_word = err_word;
+    return cuda_status(kvq::launch_encode_jobs(j, 2, sm_count_current(),
+                                               static_cast<cudaStream_t>(stream)),
+                       "kvq_encode_kv_paged");
 }
 
 int kvq_dequant(const kvq_codec* codec, const int8_t* signs, const kvq_plane* in, int32_t B,
@@ -240,7 +292,8 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
                 const int8_t* signs_v, const kvq_plane* K, const kvq_plane* V,
                 const int32_t* ctx_len, int32_t B, int32_t H_q, int32_t H_kv, int64_t max_ctx,
                 float softmax_scale, int32_t num_splits, void* workspace, int64_t ws_bytes,
-                int32_t* err_word, void* out, int32_t out_dtype, void* stream) {
+                int32_t* err_word, void* out, int32_t out_dtype, void* stream,
+                const kvq_paged_plane* PK = nullptr, const kvq_paged_plane* PV = nullptr) {
     char wk[64], wv[64];
     snprintf(wk, sizeof(wk), "%s (K)", what);
     snprintf(wv, sizeof(wv), "%s (V)", what);
@@ -249,10 +302,12 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
     if (rc) return rc;
     rc = check_codec(vc, wv, &a.vc);
     if (rc) return rc;
-    rc = check_plane(K, wk, &a.K);
+    const bool paged = PK != nullptr;
+    rc = paged ? check_paged_plane(PK, wk, &a.K) : check_plane(K, wk, &a.K);
     if (rc) return rc;
-    rc = check_plane(V, wv, &a.V);
+    rc = paged ? check_paged_plane(PV, wv, &a.V) : check_plane(V, wv, &a.V);
     if (rc) return rc;
+    a.K.H_kv = a.V.H_kv = H_kv;
     if (a.kc.d != a.vc.d) return fail(KVQ_EINVAL, "%s: K and V head_dim differ", what);
     if (a.K.capacity != a.V.capacity)
         return fail(KVQ_EINVAL, "%s: K and V capacity differ", what);
@@ -293,8 +348,10 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
     a.num_splits = num_splits;
     int64_t sl = (max_ctx + num_splits - 1) / num_splits;
-    sl = (sl + 15) / 16 * 16;
-    a.split_len = sl < 16 ? 16 : sl;
+    // paged: splits start on whole 128-token tiles, so no staged tile crosses a page
+    const int64_t gran = paged ? 128 : 16;
+    sl = (sl + gran - 1) / gran * gran;
+    a.split_len = sl < gran ? gran : sl;
     a.ws = static_cast<float*>(workspace);
     a.err_word = err_word;
     a.out = out;
@@ -334,6 +391,34 @@ int kvq_decode_step(const void* q, const void* k_new, const void* v_new, const k
     return decode_impl("kvq_decode_step", q, k_new, v_new, kc, vc, signs_k, signs_v, K, V,
                        ctx_len, B, H_q, H_kv, max_ctx, softmax_scale, num_splits, workspace,
                        ws_bytes, err_word, out, out_dtype, stream);
+}
+
+int kvq_decode_attn_paged(const void* q, const kvq_codec* kc, const kvq_codec* vc,
+                          const int8_t* signs_k, const int8_t* signs_v, const kvq_paged_plane* K,
+                          const kvq_paged_plane* V, const int32_t* ctx_len, int32_t B,
+                          int32_t H_q, int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                          int32_t num_splits, void* workspace, int64_t ws_bytes,
+                          int32_t* err_word, void* out, int32_t out_dtype, void* stream) {
+    if (!K || !V) return fail(KVQ_EINVAL, "kvq_decode_attn_paged: paged plane is NULL");
+    return decode_impl("kvq_decode_attn_paged", q, nullptr, nullptr, kc, vc, signs_k, signs_v,
+                       nullptr, nullptr, ctx_len, B, H_q, H_kv, max_ctx, softmax_scale,
+                       num_splits, workspace, ws_bytes, err_word, out, out_dtype, stream, K, V);
+}
+
+int kvq_decode_step_paged(const void* q, const void* k_new, const void* v_new,
+                          const kvq_codec* kc, const kvq_codec* vc, const int8_t* signs_k,
+                          const int8_t* signs_v, const kvq_paged_plane* K,
+                          const kvq_paged_plane* V, const int32_t* ctx_len, int32_t B,
+                          int32_t H_q, int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                          int32_t num_splits, void* workspace, int64_t ws_bytes,
+                          int32_t* err_word, void* out, int32_t out_dtype, void* stream) {
+    if (!K || !V) return fail(KVQ_EINVAL, "kvq_decode_step_paged: paged plane is NULL");
+    if (!k_new || !v_new) return fail(KVQ_EINVAL, "kvq_decode_step_paged: NULL k_new or v_new");
+    if (!aligned16(k_new) || !aligned16(v_new))
+        return fail(KVQ_EINVAL, "kvq_decode_step_paged: k_new and v_new must be 16-byte aligned");
+    return decode_impl("kvq_decode_step_paged", q, k_new, v_new, kc, vc, signs_k, signs_v,
+                       nullptr, nullptr, ctx_len, B, H_q, H_kv, max_ctx, softmax_scale,
+                       num_splits, workspace, ws_bytes, err_word, out, out_dtype, stream, K, V);
 }
 
 }  // extern "C"

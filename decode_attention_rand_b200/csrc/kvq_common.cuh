@@ -35,8 +35,26 @@ struct PlaneDev {
     uint8_t* angles;
     uint8_t* norms;
     uint8_t* params;
-    int64_t capacity;
+    int64_t capacity;      // tokens per sequence (max_pages * page_tokens when paged)
+    int H_kv;              // KV heads of the call
+    const int32_t* pages;  // NULL: contiguous [B][H_kv][capacity]; else [B][max_pages]
+    int page_tokens;
+    int max_pages;
+    int64_t num_pages;
 };
+
+// Row of token t of sequence (b, h) in each array of a plane.  A page-table
+// entry outside the pool is replaced by page 0 and flagged in *bad.
+__device__ __forceinline__ int64_t plane_row(const PlaneDev& p, int64_t b, int h, int64_t t,
+                                             bool* bad) {
+    if (!p.pages) return (b * p.H_kv + h) * p.capacity + t;
+    int64_t pg = p.pages[b * p.max_pages + t / p.page_tokens];
+    if (pg < 0 || pg >= p.num_pages) {
+        *bad = true;
+        pg = 0;
+    }
+    return (pg * p.H_kv + h) * p.page_tokens + t % p.page_tokens;
+}
 
 // --------------------------------------------------------------- warps --
 

@@ -348,18 +348,23 @@ decode_kernel(DecodeArgs A) {
     __syncthreads();
 
     // ---- producer lane: the first NST tiles go out before the prologue ------
-    const int64_t row0 = ((int64_t)b * A.H_kv + kvh) * A.K.capacity;
     int issued = 0;  // tiles issued (producer lane 0)
     auto issue_tile = [&](int tile) {
         const int rbK = A.kc.angle_words * 4, rbV = A.vc.angle_words * 4;
-        const uint8_t* srcs[6] = {A.K.angles + row0 * rbK, A.K.norms + row0 * A.kc.norm_bytes,
-                                  A.K.params + row0 * A.kc.param_bytes, A.V.angles + row0 * rbV,
-                                  A.V.norms + row0 * A.vc.norm_bytes,
-                                  A.V.params + row0 * A.vc.param_bytes};
-        const int rbs[6] = {rbK, A.kc.norm_bytes, A.kc.param_bytes, rbV, A.vc.norm_bytes,
-                            A.vc.param_bytes};
         const int s = tile % NST;
         const int64_t tt0 = t0 + (int64_t)tile * kTT;
+        // a tile never crosses a page: pages hold whole 128-token tiles and
+        // paged splits start on a multiple of 128
+        bool bad = false;
+        const int64_t rowK = plane_row(A.K, b, kvh, tt0, &bad);
+        const int64_t rowV = plane_row(A.V, b, kvh, tt0, &bad);
+        if (bad) report(A.err_word, KVQ_DEVERR_PAGE_RANGE);
+        const uint8_t* srcs[6] = {A.K.angles + rowK * rbK, A.K.norms + rowK * A.kc.norm_bytes,
+                                  A.K.params + rowK * A.kc.param_bytes, A.V.angles + rowV * rbV,
+                                  A.V.norms + rowV * A.vc.norm_bytes,
+                                  A.V.params + rowV * A.vc.param_bytes};
+        const int rbs[6] = {rbK, A.kc.norm_bytes, A.kc.param_bytes, rbV, A.vc.norm_bytes,
+                            A.vc.param_bytes};
         const int64_t left = t1m - tt0;
         const int n16 = (int)(((left < kTT ? left : kTT) + 15) / 16 * 16);
         uint32_t bytes = 0;
@@ -370,7 +375,7 @@ decode_kernel(DecodeArgs A) {
         unsigned char* dst = stages + (size_t)s * A.stage_bytes;
 #pragma unroll
         for (int k = 0; k < 6; k++)
-            bulk_g2s(dst + A.lay[k], srcs[k] + tt0 * rbs[k], (uint32_t)(n16 * rbs[k]), &full[s]);
+            bulk_g2s(dst + A.lay[k], srcs[k], (uint32_t)(n16 * rbs[k]), &full[s]);
     };
     // tile t + NST - 1 is issued once tile t - 1 is released, so NST - 1 tiles
     // are in flight ahead of the one being consumed
@@ -403,16 +408,14 @@ decode_kernel(DecodeArgs A) {
             // the same encode_tile as kvq_encode, one vector per warp
             using ECfg = EncCfg<D>;
             EncArgs E = warp == 0 ? A.enc_k : A.enc_v;
-            const PlaneDev& pl = warp == 0 ? A.K : A.V;
             const int64_t bh = (int64_t)b * A.H_kv + kvh;
             E.x = (warp == 0 ? A.k_new : A.v_new) + bh * D;
             E.n_vec = 1;
             E.T = 1;
             E.pos0 = ctx_in - 1;
-            E.out.angles = pl.angles + bh * pl.capacity * (int64_t)E.c.angle_words * 4;
-            E.out.norms = pl.norms + bh * pl.capacity * (int64_t)E.c.norm_bytes;
-            E.out.params = pl.params + bh * pl.capacity * (int64_t)E.c.param_bytes;
-            E.out.capacity = pl.capacity;
+            E.bh0 = bh;
+            E.out = warp == 0 ? A.K : A.V;
+            E.err_word = A.err_word;
             uint32_t* est = encst + warp * kEncStageWords;
             for (int i = lane; i < kEncStageWords; i += 32) est[i] = 0u;
             __syncwarp();

@@ -64,6 +64,7 @@ static EncArgs make_args(const EncodeJob& j) {
     a.T = j.T;
     a.pos0 = j.pos0;
     a.out = j.out;
+    a.err_word = j.err_word;
     return a;
 }
 
@@ -89,7 +90,7 @@ cudaError_t launch_encode_jobs(const EncodeJob* jobs, int n_jobs, int sm_count,
 cudaError_t launch_encode(const CodecDev& c, const int8_t* signs, const __half* x, int64_t n_vec,
                           int64_t T, int64_t pos0, const PlaneDev& out, int sm_count,
                           cudaStream_t stream) {
-    const EncodeJob j{c, signs, x, n_vec, T, pos0, out};
+    const EncodeJob j{c, signs, x, n_vec, T, pos0, out, nullptr};
     return launch_encode_jobs(&j, 1, sm_count, stream);
 }
 

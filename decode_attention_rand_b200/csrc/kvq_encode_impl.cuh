@@ -595,8 +595,12 @@ __device__ __forceinline__ bool encode_tile(const EncArgs& A, int64_t wt,
     // ---- pack and store ------------------------------------------------
     int64_t row = 0;
     if (valid) {
-        const int64_t bh = v / A.T;
-        row = bh * A.out.capacity + A.pos0 + (v - bh * A.T);
+        const int64_t vt = v / A.T;
+        const int64_t bh = A.bh0 + vt;
+        bool bad = false;
+        row = plane_row(A.out, bh / A.out.H_kv, (int)(bh % A.out.H_kv), A.pos0 + (v - vt * A.T),
+                        &bad);
+        if (bad && lg == 0) report(A.err_word, KVQ_DEVERR_PAGE_RANGE);
     }
     // angle bit stream: this lane's PPL codes occupy bits [cb, cb + PPL*bits)
     {

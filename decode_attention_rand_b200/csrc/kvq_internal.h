@@ -19,6 +19,7 @@ struct EncodeJob {
     int64_t T;
     int64_t pos0;
     PlaneDev out;
+    int32_t* err_word;  // device error bits, or NULL
 };
 
 // One launch for one or two jobs of the same head_dim (K and V appended
@@ -41,6 +42,8 @@ struct EncArgs {
     PlaneDev out;
     float inv_sqrt_d;
     float bins_per_rad;  // L / (2 pi)
+    int64_t bh0;         // (b * H_kv + h) of vector 0; vector v is sequence bh0 + v / T
+    int32_t* err_word;   // device error bits (page-table range), or NULL
 };
 
 // Codec-wide part of an encode job (x, n_vec, T, pos0 and out left empty).

@@ -23,7 +23,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "kvq.h")
 
 KVQ_OK, KVQ_EINVAL, KVQ_EUNSUPPORTED, KVQ_ECUDA, KVQ_ETIMEOUT = 0, -1, -2, -3, -4
 KVQ_NORM_LIN8, KVQ_NORM_LOG4 = 0, 1
-KVQ_DEVERR_CTX_RANGE, KVQ_DEVERR_TIMEOUT = 0x1, 0x2
+KVQ_DEVERR_CTX_RANGE, KVQ_DEVERR_TIMEOUT, KVQ_DEVERR_PAGE_RANGE = 0x1, 0x2, 0x4
 OUT_FP16, OUT_FP32 = 0, 1
 
 
@@ -40,6 +40,12 @@ class kvq_codec(C.Structure):
 class kvq_plane(C.Structure):
     _fields_ = [("angles", C.c_void_p), ("norms", C.c_void_p), ("params", C.c_void_p),
                 ("capacity", C.c_int64)]
+
+
+class kvq_paged_plane(C.Structure):
+    _fields_ = [("angles", C.c_void_p), ("norms", C.c_void_p), ("params", C.c_void_p),
+                ("pages", C.c_void_p), ("page_tokens", C.c_int32), ("max_pages", C.c_int32),
+                ("num_pages", C.c_int64)]
 
 
 _lock = threading.Lock()
@@ -70,6 +76,23 @@ _SIGNATURES = {
                                   C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_float, C.c_int32,
                                   C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int32,
                                   C.c_void_p]),
+    "kvq_encode_kv_paged": (C.c_int, [C.POINTER(kvq_codec), C.c_void_p, C.c_void_p,
+                                      C.POINTER(kvq_paged_plane), C.POINTER(kvq_codec),
+                                      C.c_void_p, C.c_void_p, C.POINTER(kvq_paged_plane),
+                                      C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_void_p,
+                                      C.c_void_p]),
+    "kvq_decode_attn_paged": (C.c_int, [C.c_void_p, C.POINTER(kvq_codec), C.POINTER(kvq_codec),
+                                        C.c_void_p, C.c_void_p, C.POINTER(kvq_paged_plane),
+                                        C.POINTER(kvq_paged_plane), C.c_void_p, C.c_int32,
+                                        C.c_int32, C.c_int32, C.c_int64, C.c_float, C.c_int32,
+                                        C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int32,
+                                        C.c_void_p]),
+    "kvq_decode_step_paged": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.POINTER(kvq_codec),
+                                        C.POINTER(kvq_codec), C.c_void_p, C.c_void_p,
+                                        C.POINTER(kvq_paged_plane), C.POINTER(kvq_paged_plane),
+                                        C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int64,
+                                        C.c_float, C.c_int32, C.c_void_p, C.c_int64, C.c_void_p,
+                                        C.c_void_p, C.c_int32, C.c_void_p]),
     "kvq_decode_attn": (C.c_int, [C.c_void_p, C.POINTER(kvq_codec), C.POINTER(kvq_codec),
                                   C.c_void_p, C.c_void_p, C.POINTER(kvq_plane),
                                   C.POINTER(kvq_plane), C.c_void_p, C.c_int32, C.c_int32,
@@ -179,6 +202,36 @@ def kvq_decode_step(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, sign
                                  _ptr(ctx_len), B, H_q, H_kv, max_ctx, softmax_scale, num_splits,
                                  _ptr(workspace), ws_bytes, _ptr(err_word), _ptr(out), out_dtype,
                                  _stream(stream)))
+
+
+def kvq_encode_kv_paged(kc: kvq_codec, signs_k, k, K: kvq_paged_plane, vc: kvq_codec, signs_v,
+                        v, V: kvq_paged_plane, B: int, H_kv: int, T: int, pos0: int,
+                        err_word=None, stream=None):
+    _check(lib().kvq_encode_kv_paged(C.byref(kc), _ptr(signs_k), _ptr(k), C.byref(K),
+                                     C.byref(vc), _ptr(signs_v), _ptr(v), C.byref(V), B, H_kv, T,
+                                     pos0, _ptr(err_word), _stream(stream)))
+
+
+def kvq_decode_attn_paged(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: kvq_paged_plane,
+                          V: kvq_paged_plane, ctx_len, B: int, H_q: int, H_kv: int, max_ctx: int,
+                          softmax_scale: float, num_splits: int, workspace, ws_bytes: int,
+                          err_word, out, out_dtype: int, stream=None):
+    _check(lib().kvq_decode_attn_paged(_ptr(q), C.byref(kc), C.byref(vc), _ptr(signs_k),
+                                       _ptr(signs_v), C.byref(K), C.byref(V), _ptr(ctx_len), B,
+                                       H_q, H_kv, max_ctx, softmax_scale, num_splits,
+                                       _ptr(workspace), ws_bytes, _ptr(err_word), _ptr(out),
+                                       out_dtype, _stream(stream)))
+
+
+def kvq_decode_step_paged(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v,
+                          K: kvq_paged_plane, V: kvq_paged_plane, ctx_len, B: int, H_q: int,
+                          H_kv: int, max_ctx: int, softmax_scale: float, num_splits: int,
+                          workspace, ws_bytes: int, err_word, out, out_dtype: int, stream=None):
+    _check(lib().kvq_decode_step_paged(_ptr(q), _ptr(k_new), _ptr(v_new), C.byref(kc),
+                                       C.byref(vc), _ptr(signs_k), _ptr(signs_v), C.byref(K),
+                                       C.byref(V), _ptr(ctx_len), B, H_q, H_kv, max_ctx,
+                                       softmax_scale, num_splits, _ptr(workspace), ws_bytes,
+                                       _ptr(err_word), _ptr(out), out_dtype, _stream(stream)))
 
 
 def kvq_decode_attn(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: kvq_plane,
@@ -321,3 +374,42 @@ def decode_step(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v,
                     K.H_kv, max_ctx, softmax_scale, num_splits, workspace.buf, workspace.nbytes,
                     err_word, out, out_dtype, stream)
     return out
+
+
+@dataclass
+class PagedPlane:
+    """Caller-owned pools [num_pages][H_kv][page_tokens][row] of one paged plane
+    and its page table [B][max_pages] (int32, device)."""
+    codec: kvq_codec
+    H_kv: int
+    page_tokens: int
+    num_pages: int
+    pages: object
+    angles: object
+    norms: object
+    params: object
+
+    @property
+    def max_pages(self) -> int:
+        return self.pages.shape[1]
+
+    def c(self) -> kvq_paged_plane:
+        return kvq_paged_plane(self.angles.data_ptr(), self.norms.data_ptr(),
+                               self.params.data_ptr(), self.pages.data_ptr(), self.page_tokens,
+                               self.max_pages, self.num_pages)
+
+    def rows(self, which: int):
+        """uint8 view [num_pages, H_kv, page_tokens, row_bytes] of one pool."""
+        t = (self.angles, self.norms, self.params)[which]
+        return t.view(self.num_pages, self.H_kv, self.page_tokens, -1)
+
+
+def alloc_paged_plane(c: kvq_codec, H_kv: int, page_tokens: int, num_pages: int, pages,
+                      device="cuda") -> PagedPlane:
+    """Zeroed pools for `num_pages` pages; `pages` is the [B][max_pages] table."""
+    import torch
+    n = num_pages * H_kv * page_tokens
+    arrs = [torch.zeros(max(1, n * kvq_row_bytes(c, w)), dtype=torch.uint8, device=device)
+            for w in range(3)]
+    pages = torch.as_tensor(pages, dtype=torch.int32, device=device).contiguous()
+    return PagedPlane(c, H_kv, page_tokens, num_pages, pages, *arrs)

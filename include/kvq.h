@@ -110,6 +110,8 @@ typedef enum { KVQ_NORM_LIN8 = 0, KVQ_NORM_LOG4 = 1 } kvq_norm_mode;
 /* Device error bits OR-ed into *err_word. */
 #define KVQ_DEVERR_CTX_RANGE 0x1  /* ctx_len[b] < 0 or > capacity: clipped   */
 #define KVQ_DEVERR_TIMEOUT 0x2    /* an mbarrier wait hit its iteration cap  */
+#define KVQ_DEVERR_PAGE_RANGE 0x4 /* a page-table entry outside [0, num_pages):
+                                     page 0 was read or written instead       */
 
 /* One codec: per layer and separately for K and V ("per-layer early-boost").
  * head_dim: power of two, 4..256 for encode/dequant; 64 or 128 for decode.
@@ -128,6 +130,32 @@ typedef struct {
     void* params;
     int64_t capacity;
 } kvq_plane;
+
+/* A paged plane: the rows of all sequences live in fixed-size pages of one
+ * shared pool, found through a page table (a serving cache that grows each
+ * sequence page by page; the TurboAngle page stores no cache layout of its
+ * own, this one keeps its row format and only moves rows between pages).
+ *   angles, norms, params  device pools laid out [num_pages][H_kv][page_tokens][row]
+ *                          (rows as in "Packed layout"), 16-byte aligned
+ *   pages        device int32 [B][max_pages]: pages[b][i] holds tokens
+ *                i*page_tokens .. (i+1)*page_tokens - 1 of sequence b, all KV heads
+ *   page_tokens  tokens per page: a positive multiple of 128 (one page holds
+ *                whole staged tiles of the decode kernel)
+ *   max_pages    entries per sequence in `pages`; the capacity of every
+ *                sequence is max_pages * page_tokens
+ *   num_pages    pages in the pool; an entry outside [0, num_pages) that a
+ *                call reaches is replaced by page 0 and sets KVQ_DEVERR_PAGE_RANGE
+ * Token t of sequence (b, h) is row (pages[b][t / page_tokens]*H_kv + h)
+ * * page_tokens + t % page_tokens of each pool.  K and V may share a table. */
+typedef struct {
+    void* angles;
+    void* norms;
+    void* params;
+    const int32_t* pages;
+    int32_t page_tokens;
+    int32_t max_pages;
+    int64_t num_pages;
+} kvq_paged_plane;
 
 /* Bytes per token of one plane array: which = 0 angles, 1 norms, 2 params.
  * Returns a negative kvq_status for an invalid codec or `which`.  Host only. */
@@ -246,6 +274,33 @@ int kvq_decode_step(const void* q, const void* k_new, const void* v_new,
                     int32_t num_splits, void* workspace, int64_t ws_bytes,
                     int32_t* err_word, void* out, int32_t out_dtype,
                     void* stream);
+
+/* The paged forms: kvq_encode_kv, kvq_decode_attn and kvq_decode_step with
+ * K and V in paged planes (see kvq_paged_plane).  Results are identical to
+ * the contiguous forms on the same rows; arguments and errors as there
+ * (tokens pos0 .. pos0+T-1 of every sequence must lie below its capacity). */
+int kvq_encode_kv_paged(const kvq_codec* kc, const int8_t* signs_k, const void* k,
+                        const kvq_paged_plane* K, const kvq_codec* vc,
+                        const int8_t* signs_v, const void* v, const kvq_paged_plane* V,
+                        int32_t B, int32_t H_kv, int32_t T, int64_t pos0,
+                        int32_t* err_word, void* stream);
+int kvq_decode_attn_paged(const void* q, const kvq_codec* kc, const kvq_codec* vc,
+                          const int8_t* signs_k, const int8_t* signs_v,
+                          const kvq_paged_plane* K, const kvq_paged_plane* V,
+                          const int32_t* ctx_len, int32_t B, int32_t H_q,
+                          int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                          int32_t num_splits, void* workspace, int64_t ws_bytes,
+                          int32_t* err_word, void* out, int32_t out_dtype,
+                          void* stream);
+int kvq_decode_step_paged(const void* q, const void* k_new, const void* v_new,
+                          const kvq_codec* kc, const kvq_codec* vc,
+                          const int8_t* signs_k, const int8_t* signs_v,
+                          const kvq_paged_plane* K, const kvq_paged_plane* V,
+                          const int32_t* ctx_len, int32_t B, int32_t H_q,
+                          int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                          int32_t num_splits, void* workspace, int64_t ws_bytes,
+                          int32_t* err_word, void* out, int32_t out_dtype,
+                          void* stream);
 
 /* Size of the scratch array built into the library for
  * kvq_decode_attn_noalloc (4 MiB of device memory per GPU that loads it). */

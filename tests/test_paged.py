@@ -1,0 +1,206 @@
+"""Paged K/V planes: kvq_encode_kv_paged, kvq_decode_attn_paged and
+kvq_decode_step_paged against the contiguous forms on the same rows.
+
+The pages hold whole 128-token tiles; the rows of each sequence are spread
+over a shuffled page table (with pages of other sequences and unused pages in
+between), so any mix-up of pages, heads or offsets changes the result."""
+import ctypes as C
+import math
+
+import numpy as np
+import pytest
+
+from decode_attention_rand_b200 import kvq
+
+FAKE = 1 << 20
+
+
+def _codecs(d=128):
+    return kvq.codec(d, 128, kvq.KVQ_NORM_LIN8), kvq.codec(d, 64, kvq.KVQ_NORM_LOG4)
+
+
+def _paged(page_tokens=128, max_pages=4, num_pages=16, pages=FAKE):
+    return kvq.kvq_paged_plane(FAKE, FAKE, FAKE, pages, page_tokens, max_pages, num_pages)
+
+
+@pytest.mark.parametrize("kw,msg", [
+    (dict(page_tokens=100), "multiple of 128"),
+    (dict(page_tokens=0), "multiple of 128"),
+    (dict(pages=None), "NULL pool or page table"),
+    (dict(max_pages=0), "must be positive"),
+])
+def test_paged_plane_checks(kw, msg):
+    kc, vc = _codecs()
+    K, V = _paged(**kw), _paged()
+    ws = kvq.kvq_decode_workspace_bytes(1, 8, 128, 2)
+    rc = kvq.lib().kvq_decode_attn_paged(FAKE, C.byref(kc), C.byref(vc), FAKE, FAKE, C.byref(K),
+                                         C.byref(V), FAKE, 1, 8, 2, 256, 0.1, 2, FAKE, ws, None,
+                                         FAKE, 0, None)
+    assert rc == kvq.KVQ_EINVAL
+    assert msg in kvq.kvq_last_error()
+
+
+def test_paged_encode_checks_capacity():
+    kc, vc = _codecs()
+    K, V = _paged(max_pages=2), _paged(max_pages=2)  # capacity 256
+    rc = kvq.lib().kvq_encode_kv_paged(C.byref(kc), FAKE, FAKE, C.byref(K), C.byref(vc), FAKE,
+                                       FAKE, C.byref(V), 1, 2, 10, 250, None, None)
+    assert rc == kvq.KVQ_EINVAL
+    assert "exceed capacity" in kvq.kvq_last_error()
+
+
+# ------------------------------------------------------------------- GPU --
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from decode_attention_rand_b200 import build as kbuild
+    kbuild.build()
+    kvq.lib()
+    return torch.device("cuda:0")
+
+
+def _signs(seed, d):
+    rng = np.random.default_rng(seed)
+    return torch.from_numpy(np.where(rng.integers(0, 2, d) == 0, 1, -1).astype(np.int8)).cuda()
+
+
+def _setup(B, H_kv, d, max_pages, page_tokens=128, spare=3, seed=0):
+    """Contiguous planes filled with encoded random K/V, and paged planes holding
+    the same rows under a shuffled page table."""
+    kc, vc = _codecs(d)
+    cap = max_pages * page_tokens
+    rng = np.random.default_rng(seed)
+    k = torch.from_numpy(rng.standard_normal((B, H_kv, cap, d)).astype(np.float16)).cuda()
+    v = torch.from_numpy(rng.standard_normal((B, H_kv, cap, d)).astype(np.float16)).cuda()
+    k[..., 3] *= 20
+    sk, sv = _signs(seed + 1, d), _signs(seed + 2, d)
+    Kc, Vc = kvq.alloc_plane(kc, B, H_kv, cap), kvq.alloc_plane(vc, B, H_kv, cap)
+    kvq.encode(kc, sk, k, Kc, 0)
+    kvq.encode(vc, sv, v, Vc, 0)
+    num_pages = B * max_pages + spare
+    table = rng.permutation(num_pages)[:B * max_pages].reshape(B, max_pages)
+    Kp = kvq.alloc_paged_plane(kc, H_kv, page_tokens, num_pages, table)
+    Vp = kvq.alloc_paged_plane(vc, H_kv, page_tokens, num_pages, table)
+    for P, Cn in ((Kp, Kc), (Vp, Vc)):
+        for w in range(3):
+            for b in range(B):
+                for i in range(max_pages):
+                    P.rows(w)[int(table[b, i])] = Cn.rows(w)[b, :, i * page_tokens:(i + 1) * page_tokens]
+    return kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table
+
+
+def _same_rows(P, Cn, table, page_tokens=128):
+    B, max_pages = table.shape
+    for w in range(3):
+        for b in range(B):
+            for i in range(max_pages):
+                got = P.rows(w)[int(table[b, i])]
+                want = Cn.rows(w)[b, :, i * page_tokens:(i + 1) * page_tokens]
+                if not torch.equal(got, want):
+                    return False
+    return True
+
+
+def _ws(B, H_q, d, S):
+    return kvq.DecodeWorkspace(B, H_q, d, S, "cuda")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("S", [1, 2, 3, 6])
+def test_paged_decode_equals_contiguous(dev, S):
+    B, H_kv, G, d, max_pages = 3, 2, 4, 128, 6
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=S)
+    H_q = G * H_kv
+    q = torch.randn((B, H_q, d), dtype=torch.float16, device="cuda")
+    ctx = torch.tensor([300, 129, 768], dtype=torch.int32, device="cuda")
+    maxc, tau = 768, 1 / math.sqrt(d)  # 768 / S is a whole number of tiles for these S
+    out_c = kvq.decode_attn(q, kc, vc, sk, sv, Kc, Vc, ctx, maxc, tau, num_splits=S)
+    ws = _ws(B, H_q, d, S)
+    out_p = torch.empty_like(out_c)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.kvq_decode_attn_paged(q, kc, vc, sk, sv, Kp.c(), Vp.c(), ctx, B, H_q, H_kv, maxc, tau, S,
+                              ws.buf, ws.nbytes, err, out_p, kvq.OUT_FP32)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(out_p, out_c)
+
+
+@pytest.mark.gpu
+def test_paged_decode_unaligned_split_count(dev):
+    # 5 splits of 768 tokens: the paged form starts its splits on whole tiles,
+    # the contiguous one on 16-token rows: the same attention up to rounding
+    B, H_kv, G, d, max_pages = 2, 2, 4, 128, 6
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=9)
+    H_q = G * H_kv
+    q = torch.randn((B, H_q, d), dtype=torch.float16, device="cuda")
+    ctx = torch.tensor([700, 401], dtype=torch.int32, device="cuda")
+    out_c = kvq.decode_attn(q, kc, vc, sk, sv, Kc, Vc, ctx, 768, None, num_splits=5)
+    ws = _ws(B, H_q, d, 5)
+    out_p = torch.empty_like(out_c)
+    kvq.kvq_decode_attn_paged(q, kc, vc, sk, sv, Kp.c(), Vp.c(), ctx, B, H_q, H_kv, 768,
+                              1 / math.sqrt(d), 5, ws.buf, ws.nbytes, None, out_p, kvq.OUT_FP32)
+    torch.cuda.synchronize()
+    rel = ((out_p - out_c).double().norm(dim=-1) / out_c.double().norm(dim=-1)).max().item()
+    assert rel < 1e-5
+
+
+@pytest.mark.gpu
+def test_paged_encode_kv_equals_contiguous(dev):
+    B, H_kv, d, max_pages = 2, 3, 128, 4
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=5)
+    # overwrite tokens 50 .. 349 (three pages) of both layouts with new vectors
+    rng = np.random.default_rng(6)
+    kn = torch.from_numpy(rng.standard_normal((B, H_kv, 300, d)).astype(np.float16)).cuda()
+    vn = torch.from_numpy(rng.standard_normal((B, H_kv, 300, d)).astype(np.float16)).cuda()
+    kvq.encode_kv(kc, sk, kn, Kc, vc, sv, vn, Vc, 50)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.kvq_encode_kv_paged(kc, sk, kn, Kp.c(), vc, sv, vn, Vp.c(), B, H_kv, 300, 50, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert _same_rows(Kp, Kc, table) and _same_rows(Vp, Vc, table)
+
+
+@pytest.mark.gpu
+def test_paged_decode_step_equals_contiguous(dev):
+    B, H_kv, G, d, max_pages = 3, 2, 4, 128, 4
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=7)
+    H_q = G * H_kv
+    q = torch.randn((B, H_q, d), dtype=torch.float16, device="cuda")
+    k_new = torch.randn((B, H_kv, d), dtype=torch.float16, device="cuda")
+    v_new = torch.randn((B, H_kv, d), dtype=torch.float16, device="cuda")
+    ctx = torch.tensor([129, 256, 384], dtype=torch.int32, device="cuda")  # page edges
+    S = 2
+    out_c = kvq.decode_step(q, k_new, v_new, kc, vc, sk, sv, Kc, Vc, ctx, 512, num_splits=S)
+    ws = _ws(B, H_q, d, S)
+    out_p = torch.empty_like(out_c)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.kvq_decode_step_paged(q, k_new, v_new, kc, vc, sk, sv, Kp.c(), Vp.c(), ctx, B, H_q, H_kv,
+                              512, 1 / math.sqrt(d), S, ws.buf, ws.nbytes, err, out_p,
+                              kvq.OUT_FP32)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert _same_rows(Kp, Kc, table) and _same_rows(Vp, Vc, table)
+    assert torch.equal(out_p, out_c)
+
+
+@pytest.mark.gpu
+def test_paged_bad_page_entry_is_reported(dev):
+    B, H_kv, G, d, max_pages = 1, 2, 4, 128, 2
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=8)
+    Kp.pages[0, 1] = 10_000  # beyond the pool
+    H_q = G * H_kv
+    q = torch.randn((B, H_q, d), dtype=torch.float16, device="cuda")
+    ctx = torch.tensor([256], dtype=torch.int32, device="cuda")
+    ws = _ws(B, H_q, d, 1)
+    out = torch.empty((B, H_q, d), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.kvq_decode_attn_paged(q, kc, vc, sk, sv, Kp.c(), Vp.c(), ctx, B, H_q, H_kv, 256,
+                              1 / math.sqrt(d), 1, ws.buf, ws.nbytes, err, out, kvq.OUT_FP32)
+    torch.cuda.synchronize()
+    assert int(err.item()) & kvq.KVQ_DEVERR_PAGE_RANGE
+    assert torch.isfinite(out).all()
