@@ -158,8 +158,11 @@ int prep_encode(const kvq_codec* codec, const int8_t* signs, const void* x, int3
     rc = paged ? check_paged_plane(paged, what, &job->out) : check_plane(out, what, &job->out);
     if (rc) return rc;
     job->out.H_kv = H_kv;
+    job->out.hdiv = kvq::make_fast_div(H_kv > 0 ? (uint32_t)H_kv : 1u);
     job->err_word = nullptr;
     if (B < 0 || H_kv < 0 || T < 0) return fail(KVQ_EINVAL, "%s: negative size", what);
+    if (paged && (int64_t)B * H_kv >= (1ll << 31))
+        return fail(KVQ_EINVAL, "%s: B * H_kv must be below 2^31 for a paged plane", what);
     if (pos0 < 0 || pos0 + (int64_t)T > job->out.capacity)
         return fail(KVQ_EINVAL, "%s: tokens [%lld, %lld) exceed capacity %lld", what,
                     (long long)pos0, (long long)(pos0 + T), (long long)job->out.capacity);
@@ -308,6 +311,7 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
     rc = paged ? check_paged_plane(PV, wv, &a.V) : check_plane(V, wv, &a.V);
     if (rc) return rc;
     a.K.H_kv = a.V.H_kv = H_kv;
+    a.K.hdiv = a.V.hdiv = kvq::make_fast_div(H_kv > 0 ? (uint32_t)H_kv : 1u);
     if (a.kc.d != a.vc.d) return fail(KVQ_EINVAL, "%s: K and V head_dim differ", what);
     if (a.K.capacity != a.V.capacity)
         return fail(KVQ_EINVAL, "%s: K and V capacity differ", what);

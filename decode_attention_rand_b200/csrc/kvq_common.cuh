@@ -31,6 +31,32 @@ struct CodecDev {
     int param_bytes;  // 2 (LIN8) or 4 (LOG4)
 };
 
+// Division of a 32-bit unsigned dividend by a divisor fixed per launch:
+// multiply-high and shifts (Granlund and Montgomery, "Division by Invariant
+// Integers using Multiplication", PLDI 1994, section 4), exact for every
+// dividend below 2^32 and divisor 1 <= d < 2^32.
+struct FastDiv {
+    uint32_t m;   // 2^32 (2^l - d) / d + 1, l = ceil(log2 d)
+    uint32_t s1;  // min(l, 1)
+    uint32_t s2;  // max(l - 1, 0)
+};
+
+inline FastDiv make_fast_div(uint32_t d) {
+    if (d == 0) d = 1;
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < (unsigned long long)d) l++;
+    FastDiv f;
+    f.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
+    f.s1 = l < 1 ? l : 1;
+    f.s2 = l > 1 ? l - 1 : 0;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+    const uint32_t t = __umulhi(f.m, n);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
 struct PlaneDev {
     uint8_t* angles;
     uint8_t* norms;
@@ -41,6 +67,7 @@ struct PlaneDev {
     int page_tokens;
     int max_pages;
     int64_t num_pages;
+    FastDiv hdiv;          // division by H_kv (paged row lookup by sequence index)
 };
 
 // Row of token t of sequence (b, h) in each array of a plane.  A page-table
@@ -54,6 +81,14 @@ __device__ __forceinline__ int64_t plane_row(const PlaneDev& p, int64_t b, int h
         pg = 0;
     }
     return (pg * p.H_kv + h) * p.page_tokens + t % p.page_tokens;
+}
+
+// Row of token t of sequence bh = b * H_kv + h (B * H_kv < 2^32 when paged).
+__device__ __forceinline__ int64_t plane_row_bh(const PlaneDev& p, int64_t bh, int64_t t,
+                                                bool* bad) {
+    if (!p.pages) return bh * p.capacity + t;
+    const uint32_t b = fast_div((uint32_t)bh, p.hdiv);
+    return plane_row(p, b, (int)((uint32_t)bh - b * (uint32_t)p.H_kv), t, bad);
 }
 
 // --------------------------------------------------------------- warps --

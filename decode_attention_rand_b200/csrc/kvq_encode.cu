@@ -1,6 +1,7 @@
-// kvq_encode.cu - the encode/append kernel and its launcher (the per-tile
-// encoding itself lives in kvq_encode_impl.cuh).
-#include "kvq_encode_impl.cuh"
+// kvq_encode.cu - the encode/append kernels and their launcher: the streaming
+// kernel of kvq_encode_fast.cuh where it applies, else the general one (the
+// per-tile encoding of kvq_encode_impl.cuh, shared with the fused append).
+#include "kvq_encode_fast.cuh"
 
 namespace kvq {
 
@@ -48,12 +49,44 @@ static cudaError_t launch_encode_d(const EncPair& pa, int n_args, int sm_count,
     return cudaGetLastError();
 }
 
+// The streaming and fixup kernels of kvq_encode_fast.cuh cover d = 64, 128,
+// 256 and L % 8 == 0 with 16 <= L <= 256, for fewer than 2^32 vectors.
+static bool fast_ok(const EncodeJob& j) {
+    const int d = j.c.d, L = j.c.L;
+    return (d == 64 || d == 128 || d == 256) && L % 8 == 0 && L >= 16 && L <= 256 &&
+           j.n_vec <= (1ll << 32) - 64 && j.T >= 1;
+}
+
+template <int D>
+static cudaError_t launch_encode_fast_d(const EncPair& pa, int n_args, int sm_count,
+                                        cudaStream_t stream) {
+    constexpr int VPW = FastCfg<D>::VPW;
+    int64_t n_max = pa.a[0].n_vec;
+    if (n_args > 1 && pa.a[1].n_vec > n_max) n_max = pa.a[1].n_vec;
+    const int64_t tiles = (n_max + VPW - 1) / VPW;
+    int64_t blocks = (tiles + kFastWarps - 1) / kFastWarps;
+    const int64_t cap = (int64_t)sm_count * kFastBlocksPerSM * 4 / n_args;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    encode_fast_kernel<D>
+        <<<dim3((unsigned)blocks, (unsigned)n_args), kFastWarps * 32, 0, stream>>>(pa);
+    // the fixup pass: one warp per 32 vectors
+    int64_t fblocks = ((n_max + 31) / 32 + kFastWarps - 1) / kFastWarps;
+    if (fblocks > cap) fblocks = cap;
+    if (fblocks < 1) fblocks = 1;
+    encode_fixup_kernel<D>
+        <<<dim3((unsigned)fblocks, (unsigned)n_args), kFastWarps * 32, 0, stream>>>(pa);
+    return cudaGetLastError();
+}
+
 EncArgs encode_args(const CodecDev& c, const int8_t* signs) {
     EncArgs a = {};
     a.signs = signs;
     a.c = c;
     a.inv_sqrt_d = (float)(1.0 / sqrt((double)c.d));
     a.bins_per_rad = (float)((double)c.L / (2.0 * kPi));
+    a.tdiv = make_fast_div(1);
+    a.small = 1;
     return a;
 }
 
@@ -65,6 +98,8 @@ static EncArgs make_args(const EncodeJob& j) {
     a.pos0 = j.pos0;
     a.out = j.out;
     a.err_word = j.err_word;
+    a.small = j.n_vec < (1ll << 32) && j.T >= 1 && j.T < (1ll << 32);
+    a.tdiv = make_fast_div(a.small ? (uint32_t)j.T : 1u);
     return a;
 }
 
@@ -75,6 +110,14 @@ cudaError_t launch_encode_jobs(const EncodeJob* jobs, int n_jobs, int sm_count,
     EncPair pa;
     pa.a[0] = make_args(jobs[0]);
     pa.a[1] = n_jobs == 2 ? make_args(jobs[1]) : pa.a[0];
+    if (fast_ok(jobs[0]) && (n_jobs == 1 || fast_ok(jobs[1]))) {
+        switch (jobs[0].c.d) {
+            case 64: return launch_encode_fast_d<64>(pa, n_jobs, sm_count, stream);
+            case 128: return launch_encode_fast_d<128>(pa, n_jobs, sm_count, stream);
+            case 256: return launch_encode_fast_d<256>(pa, n_jobs, sm_count, stream);
+            default: break;
+        }
+    }
     switch (jobs[0].c.d) {
         case 4: return launch_encode_d<4>(pa, n_jobs, sm_count, stream);
         case 8: return launch_encode_d<8>(pa, n_jobs, sm_count, stream);

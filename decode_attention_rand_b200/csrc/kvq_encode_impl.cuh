@@ -132,12 +132,13 @@ __device__ __forceinline__ int log4_code_exact(double l, double LO, double HI) {
 template <int EPL, int NL>
 __device__ __forceinline__ void exact_pair_z(const uint32_t (&raw)[EPL / 2], int p, int lg,
                                              double& z0, double& z1) {
-    constexpr int LOGE = EPL == 2 ? 1 : EPL == 4 ? 2 : EPL == 8 ? 3 : 4;
-    static_assert(EPL <= 16, "word signs below assume at most 8 words per lane");
+    constexpr int LOGE = EPL == 2 ? 1 : EPL == 4 ? 2 : EPL == 8 ? 3 : EPL == 16 ? 4 : 5;
+    static_assert(EPL <= 32, "word signs below assume at most 16 words per lane");
     const unsigned j0 = 2u * (unsigned)p;
     const unsigned m = (j0 & (unsigned)(EPL - 1)) >> 1;
     // bit w of `row` = parity(m & w): the Sylvester row m over the lane's words
-    const unsigned row = ((m & 1u) ? 0xAAu : 0u) ^ ((m & 2u) ? 0xCCu : 0u) ^ ((m & 4u) ? 0xF0u : 0u);
+    const unsigned row = ((m & 1u) ? 0xAAAAu : 0u) ^ ((m & 2u) ? 0xCCCCu : 0u) ^
+                         ((m & 4u) ? 0xF0F0u : 0u) ^ ((m & 8u) ? 0xFF00u : 0u);
     double E = 0.0, O = 0.0;
 #pragma unroll
     for (int w = 0; w < EPL / 2; w++) {
@@ -215,10 +216,9 @@ struct ExactOut {
 // The transform recomputed in fp64 (exact for fp16 inputs) and the flagged
 // decisions re-taken with the definition's own formulas.  Called by every
 // lane of the warp (it shuffles across the group).
-template <int D>
-__device__ __noinline__ ExactOut<EncCfg<D>::PPL> exact_fixup(ExactIn<EncCfg<D>::PPL> in, int lg,
-                                                            int L, int mode) {
-    using Cfg = EncCfg<D>;
+template <int D, class Cfg = EncCfg<D>>
+__device__ __noinline__ ExactOut<Cfg::PPL> exact_fixup(ExactIn<Cfg::PPL> in, int lg, int L,
+                                                      int mode) {
     constexpr int EPL = Cfg::EPL, NL = Cfg::NL, PPL = Cfg::PPL;
     ExactOut<PPL> o;
 #pragma unroll
@@ -306,11 +306,10 @@ __device__ __noinline__ ExactOut<EncCfg<D>::PPL> exact_fixup(ExactIn<EncCfg<D>::
 // every code of the group changes, and exact_fixup redoes the whole vector.
 // Out of line, so none of this costs the streaming pass registers; called by
 // every lane of the warp.
-template <int D>
-__device__ __noinline__ ExactOut<EncCfg<D>::PPL> exact_path(ExactIn<EncCfg<D>::PPL> in, int lg,
-                                                           int grp, int L, int mode,
-                                                           float bins_per_rad) {
-    using Cfg = EncCfg<D>;
+// Cfg gives the lane layout (EPL elements per lane, NL lanes per vector).
+template <int D, class Cfg = EncCfg<D>>
+__device__ __noinline__ ExactOut<Cfg::PPL> exact_path(ExactIn<Cfg::PPL> in, int lg, int grp,
+                                                     int L, int mode, float bins_per_rad) {
     constexpr int EPL = Cfg::EPL, NL = Cfg::NL, PPL = Cfg::PPL;
     ExactOut<PPL> o;
 #pragma unroll
@@ -370,7 +369,7 @@ __device__ __noinline__ ExactOut<EncCfg<D>::PPL> exact_path(ExactIn<EncCfg<D>::P
             redo = in.unsure || o.prm != in.prm;
         }
     }
-    if (__any_sync(KVQ_FULL_MASK, redo)) return exact_fixup<D>(in, lg, L, mode);
+    if (__any_sync(KVQ_FULL_MASK, redo)) return exact_fixup<D, Cfg>(in, lg, L, mode);
     return o;
 }
 
@@ -595,11 +594,9 @@ __device__ __forceinline__ bool encode_tile(const EncArgs& A, int64_t wt,
     // ---- pack and store ------------------------------------------------
     int64_t row = 0;
     if (valid) {
-        const int64_t vt = v / A.T;
-        const int64_t bh = A.bh0 + vt;
+        const int64_t vt = A.small ? (int64_t)fast_div((uint32_t)v, A.tdiv) : v / A.T;
         bool bad = false;
-        row = plane_row(A.out, bh / A.out.H_kv, (int)(bh % A.out.H_kv), A.pos0 + (v - vt * A.T),
-                        &bad);
+        row = plane_row_bh(A.out, A.bh0 + vt, A.pos0 + (v - vt * A.T), &bad);
         if (bad && lg == 0) report(A.err_word, KVQ_DEVERR_PAGE_RANGE);
     }
     // angle bit stream: this lane's PPL codes occupy bits [cb, cb + PPL*bits)

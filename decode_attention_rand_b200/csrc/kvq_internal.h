@@ -44,6 +44,8 @@ struct EncArgs {
     float bins_per_rad;  // L / (2 pi)
     int64_t bh0;         // (b * H_kv + h) of vector 0; vector v is sequence bh0 + v / T
     int32_t* err_word;   // device error bits (page-table range), or NULL
+    FastDiv tdiv;        // division by T
+    int small;           // n_vec and T below 2^32: v / T through tdiv
 };
 
 // Codec-wide part of an encode job (x, n_vec, T, pos0 and out left empty).

@@ -104,7 +104,7 @@ def test_encode_hand_examples(dev):
 
 
 @pytest.mark.parametrize("d", [4, 8, 16, 32, 64, 128, 256])
-@pytest.mark.parametrize("L", [2, 3, 5, 8, 64, 128, 256, 1000, 65536])
+@pytest.mark.parametrize("L", [2, 3, 5, 8, 16, 24, 40, 64, 128, 200, 256, 1000, 65536])
 def test_encode_sweep(dev, d, L):
     s = _signs(d * 7 + L, d)
     x = _rand_x(2, 3, 37, d, seed=d * 1000 + L)
@@ -162,8 +162,8 @@ def test_encode_kv_rejects_mismatched_head_dims(dev):
     assert "head_dim" in str(e.value)
 
 
-def test_encode_edge_cases(dev):
-    d = 128
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_encode_edge_cases(dev, d):
     s = _signs(3, d)
     xs = []
     xs.append(np.zeros((1, d)))                          # all-zero vector
@@ -182,7 +182,7 @@ def test_encode_edge_cases(dev):
     sparse[:, [0, 1]] = [[3.0, 1.0], [1.0, 3.0], [-2.0, 2.0], [0.5, -0.25]]
     xs.append(sparse)
     x = np.concatenate(xs).astype(np.float16)[None, None]
-    for L in (4, 8, 16, 128, 256, 3, 65536):
+    for L in (4, 8, 16, 24, 40, 128, 200, 256, 3, 65536):
         for mode in (O.MODE_LIN8, O.MODE_LOG4):
             check_encode(x, s, L, mode)
 
