@@ -143,193 +143,76 @@ __device__ __forceinline__ void split_fwht(const uint32_t (&raw)[16], int lg, f3
     fwht_pairs<NL>(LO, lg);
 }
 
-// r (LIN8) or log2 max(r, 2^-24) (LOG4) of an exact rotated pair, in fp64
-// (the formulas of exact_path); inv_d = 1/d.
-static __device__ __noinline__ double exact_norm_value(double z0, double z1, bool lin8,
-                                                       double inv_d) {
-    const double r2 = fma(z0, z0, z1 * z1) * inv_d;
-    return lin8 ? sqrt(r2) : 0.5 * exact_log2_sq(r2);
-}
-
-// Per-lane state handed to exact_fast through shared memory: word i of lane
-// l at st[i * 32 + l] (the lane's column; no bank conflicts).
-constexpr int kFsNv = 0;      // 16 words: LIN8 |w pair|, LOG4 fp32 log2 r
-constexpr int kFsQ4 = 16;     // 4 words: angle codes, four per word
-constexpr int kFsNc = 20;     // 4 words: norm codes (bytes or nibbles)
-constexpr int kFsNeedA = 24, kFsNeedN = 25, kFsPrm = 26, kFsPmin = 27, kFsPmax = 28,
-              kFsPband = 29, kFsFlags = 30;
-constexpr uint32_t kFsValid = 1u, kFsNeedP = 2u, kFsUnsure = 4u, kFsInexact = 8u;
-constexpr int kFsWords = 32;
-
 // Parameter of a vector left for the fixup pass: an fp16 NaN (LIN8 M) or two
 // (LOG4 LO, HI), values the codec never stores (its parameters saturate to
 // finite fp16).
 constexpr uint32_t kFixupMark16 = 0xFFFFu;
 constexpr uint32_t kFixupMark32 = 0xFFFFFFFFu;
 
-// The decisions in doubt of one warp tile.  From the split transform, the
-// exact pair (w0, w1) is hi_w + lo_w in fp64, and z = (w0 + w1, w0 - w1) is
-// exact as well; each lane re-takes its own flagged decisions with the
-// definition's formulas (encode_tile's exact_path rules: a parameter in doubt
-// is settled by the pairs that can hold the extreme, and if it moves every
-// norm code of the vector is re-decided).  A warp holding a vector outside
-// the exact range of the split takes the general fp64 path (exact_fixup).
-// Out of line, fed through shared memory, so the streaming loop keeps its
-// registers; called by every lane of the warp.
+// Pack and store one vector's codes: this lane's 16 angle codes (q4, four
+// per word, b bits each) at bit 16 b lg of the angle row, its norm codes (nc:
+// 4 bytes a word for LIN8, 8 nibbles for LOG4) and, from lane 0 of the
+// group, the parameter.  Called by every lane (odd b exchanges half words).
 template <int D>
-__device__ __noinline__ void exact_fast(const __half* x, const uint32_t* smask, uint32_t v, int lg,
-                                        uint32_t* st, int L, int mode, int bits, float bpr) {
-    using Cfg = FastCfg<D>;
-    constexpr int NL = Cfg::NL;
-    const float sc = (float)(Cfg::S == 6 ? 0.17677669529663687
-                                         : Cfg::S == 7 ? 0.125 : 0.08838834764831845);
-    uint32_t raw[16];
-    {
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)v * D + lg * 32);
-        const uint4* msk = reinterpret_cast<const uint4*>(smask);
+__device__ __forceinline__ void store_codes(const EncArgs& A, uint32_t v, bool valid, int lg,
+                                            const uint32_t (&q4)[4], const uint32_t (&nc)[4],
+                                            uint32_t prm) {
+    const uint32_t bits = (uint32_t)A.c.bits;
+    const uint32_t s4 = 4u * bits;  // 16 .. 32
+    const uint32_t a0 = q4[0] | shl_c(q4[1], s4), a1 = shr_c(q4[1], 32u - s4);
+    const uint32_t b0 = q4[2] | shl_c(q4[3], s4), b1 = shr_c(q4[3], 32u - s4);
+    const uint32_t r8 = 8u * bits - 32u;  // 0 .. 32: offset of codes 8..15 past word 1
+    uint32_t o[4];
+    o[0] = a0;
+    o[1] = a1 | shl_c(b0, r8);
+    o[2] = shr_c(b0, 32u - r8) | shl_c(b1, r8);
+    o[3] = shr_c(b1, 32u - r8);
+    if (bits & 1u) {
+        // odd b: odd lanes start half way into a word; they hand their first
+        // 16 bits to the lane below, which completes its last word with them
+        const uint32_t up = __shfl_down_sync(KVQ_FULL_MASK, o[0], 1);
+        const uint32_t last = (bits - 1u) >> 1;  // half-filled word of an even lane
+        if (lg & 1) {
+            o[0] = __funnelshift_r(o[0], o[1], 16);
+            o[1] = __funnelshift_r(o[1], o[2], 16);
+            o[2] = __funnelshift_r(o[2], o[3], 16);
+            o[3] >>= 16;
+        } else {
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-            const uint4 t = src[q];
-            const uint4 m = msk[q];
-            raw[4 * q + 0] = t.x ^ m.x;
-            raw[4 * q + 1] = t.y ^ m.y;
-            raw[4 * q + 2] = t.z ^ m.z;
-            raw[4 * q + 3] = t.w ^ m.w;
+            for (int j = 0; j < 4; j++)
+                if ((uint32_t)j == last) o[j] |= up << 16;
         }
     }
-    const bool lin8 = mode == KVQ_NORM_LIN8;
-    const uint32_t am = (1u << bits) - 1u;
-    int acode[16], ncode[16];
+    if (!valid) return;
+    const uint32_t vt = fast_div(v, A.tdiv);
+    bool bad = false;
+    const int64_t row =
+        plane_row_bh(A.out, A.bh0 + vt, A.pos0 + (int64_t)(v - vt * (uint32_t)A.T), &bad);
+    if (bad && lg == 0) report(A.err_word, KVQ_DEVERR_PAGE_RANGE);
+    // this lane's words: [ceil(lg b / 2), ceil((lg + 1) b / 2))
+    const uint32_t w0 = ((uint32_t)lg * bits + 1u) >> 1;
+    const uint32_t nw = (((uint32_t)lg + 1u) * bits + 1u) / 2u - w0;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(A.out.angles) + row * A.c.angle_words + w0;
 #pragma unroll
-    for (int k = 0; k < 16; k++) {
-        acode[k] = (int)((st[(kFsQ4 + (k >> 2)) * 32] >> ((uint32_t)bits * (uint32_t)(k & 3))) & am);
-        ncode[k] = lin8 ? (int)((st[(kFsNc + (k >> 2)) * 32] >> (8 * (k & 3))) & 255u)
-                        : (int)((st[(kFsNc + (k >> 3)) * 32] >> (4 * (k & 7))) & 15u);
-    }
-    const uint32_t need_a = st[kFsNeedA * 32], need_n = st[kFsNeedN * 32];
-    uint32_t prm = st[kFsPrm * 32];
-    const float pmin = __uint_as_float(st[kFsPmin * 32]), pmax = __uint_as_float(st[kFsPmax * 32]),
-                pband = __uint_as_float(st[kFsPband * 32]);
-    const uint32_t fl = st[kFsFlags * 32];
-    const bool valid = fl & kFsValid, need_p = fl & kFsNeedP, unsure = fl & kFsUnsure;
-    // fp32 value of pair k the parameter decision was based on
-    auto v32 = [&](int k) -> float {
-        const float nv = __uint_as_float(st[(kFsNv + k) * 32]);
-        return lin8 ? nv * sc : nv;
-    };
-    if (__any_sync(KVQ_FULL_MASK, (fl & kFsInexact) != 0u)) {
-        ExactIn<16> in;
-#pragma unroll
-        for (int k = 0; k < 16; k++) {
-            in.raw[k] = raw[k];
-            in.rr[k] = lin8 ? v32(k) : 0.f;
-            in.ll[k] = lin8 ? 0.f : v32(k);
-            in.acode[k] = acode[k];
-            in.ncode[k] = ncode[k];
-        }
-        in.need_a = need_a;
-        in.need_n = need_n;
-        in.prm = prm;
-        in.pmin = pmin;
-        in.pmax = pmax;
-        in.pband = pband;
-        in.valid = valid;
-        in.need_p = need_p;
-        in.unsure = unsure;
-        const ExactOut<16> o = exact_fixup<D, Cfg>(in, lg, L, mode);
-#pragma unroll
-        for (int k = 0; k < 16; k++) {
-            acode[k] = o.acode[k];
-            ncode[k] = o.ncode[k];
-        }
-        prm = o.prm;
+    for (int j = 0; j < 4; j++)
+        if ((uint32_t)j < nw) dst[j] = o[j];
+    if (A.c.mode == KVQ_NORM_LIN8) {
+        *reinterpret_cast<uint4*>(A.out.norms + row * (D / 2) + lg * 16) =
+            make_uint4(nc[0], nc[1], nc[2], nc[3]);
+        if (lg == 0) reinterpret_cast<uint16_t*>(A.out.params)[row] = (uint16_t)prm;
     } else {
-        // the exact rotated pairs (rolled loops below index them at run time,
-        // from local memory: this path is rare, its code is kept small)
-        double z0[16], z1[16];
-        {
-            f32x2 HI[16], LO[16];
-            int E;
-            bool zero;
-            split_fwht<D>(raw, lg, HI, LO, E, zero);
-            (void)E;
-            (void)zero;
-#pragma unroll
-            for (int k = 0; k < 16; k++) {
-                const double w0 = (double)lo2(HI[k]) + (double)lo2(LO[k]);
-                const double w1 = (double)hi2(HI[k]) + (double)hi2(LO[k]);
-                z0[k] = w0 + w1;
-                z1[k] = w0 - w1;
-            }
-        }
-#pragma unroll 1
-        for (uint32_t t = valid ? need_a : 0u; t; t &= t - 1u) {
-            const int k = __ffs(t) - 1;
-            acode[k] = angle_code_from_exact(z0[k], z1[k], L, bpr);
-        }
-        const bool gp = valid && need_p;  // uniform within the group
-        bool redo = false;
-        if (__any_sync(KVQ_FULL_MASK, gp)) {
-            double ext_hi = lin8 ? 0.0 : -1e300, ext_lo = 1e300;
-            uint32_t ch = 0, cl = 0;  // candidates for the largest / smallest value
-            if (gp) {
-#pragma unroll
-                for (int k = 0; k < 16; k++) {
-                    const float f = v32(k);
-                    if (unsure || f >= pmax - pband) ch |= 1u << k;
-                    if (!lin8 && (unsure || f <= pmin + pband)) cl |= 1u << k;
-                }
-            }
-#pragma unroll 1
-            for (uint32_t t = ch | cl; t; t &= t - 1u) {
-                const int k = __ffs(t) - 1;
-                const double xk = exact_norm_value(z0[k], z1[k], lin8, 1.0 / D);
-                if ((ch >> k) & 1u) ext_hi = fmax(ext_hi, xk);
-                if ((cl >> k) & 1u) ext_lo = fmin(ext_lo, xk);
-            }
-            ext_hi = group_max_d<NL>(ext_hi);
-            ext_lo = group_min_d<NL>(ext_lo);
-            if (gp) {
-                const uint32_t px = lin8 ? (uint32_t)f64_to_f16_sat(ext_hi)
-                                         : ((uint32_t)f64_to_f16_sat(ext_lo) |
-                                            ((uint32_t)f64_to_f16_sat(ext_hi) << 16));
-                redo = unsure || px != prm;
-                prm = px;
-            }
-        }
-        const double M = (double)half_bits_to_float((uint16_t)(prm & 0xFFFF));
-        const double HIp = (double)half_bits_to_float((uint16_t)(prm >> 16));
-#pragma unroll 1
-        for (uint32_t t = redo ? 0xFFFFu : (valid ? need_n : 0u); t; t &= t - 1u) {
-            const int k = __ffs(t) - 1;
-            const double xk = exact_norm_value(z0[k], z1[k], lin8, 1.0 / D);
-            ncode[k] = lin8 ? lin8_code_exact(xk, M) : log4_code_exact(xk, M, HIp);
-        }
+        *reinterpret_cast<uint2*>(A.out.norms + row * (D / 4) + lg * 8) = make_uint2(nc[0], nc[1]);
+        if (lg == 0) reinterpret_cast<uint32_t*>(A.out.params)[row] = prm;
     }
-    uint32_t q4[4] = {0u, 0u, 0u, 0u}, nc[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int k = 0; k < 16; k++) {
-        q4[k >> 2] |= (uint32_t)acode[k] << ((uint32_t)bits * (uint32_t)(k & 3));
-        if (lin8)
-            nc[k >> 2] |= (uint32_t)ncode[k] << (8 * (k & 3));
-        else
-            nc[k >> 3] |= (uint32_t)ncode[k] << (4 * (k & 7));
-    }
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-        st[(kFsQ4 + j) * 32] = q4[j];
-        st[(kFsNc + j) * 32] = nc[j];
-    }
-    st[kFsPrm * 32] = prm;
 }
 
 // One warp tile: vector v per group of NL lanes (lanes past n_vec compute on
 // vector 0 and store nothing).  pwk = {1, 2^b, 2^2b, 2^3b} places four b-bit
-// angle codes in one word; st is this lane's column of the warp's state.
-template <int D, bool EXACT>
+// angle codes in one word.
+template <int D>
 __device__ __forceinline__ void encode_tile_fast(const EncArgs& A, uint32_t v,
                                                  const uint32_t* smask, int lg,
-                                                 const uint32_t (&pwk)[4], uint32_t* st) {
+                                                 const uint32_t (&pwk)[4]) {
     using Cfg = FastCfg<D>;
     constexpr int NL = Cfg::NL, S = Cfg::S;
     const bool valid = (int64_t)v < A.n_vec;
@@ -455,87 +338,11 @@ __device__ __forceinline__ void encode_tile_fast(const EncArgs& A, uint32_t v,
         need_p = unsure = true;
     }
 
-    // ---- decisions in doubt ----------------------------------------------------
-    // streaming pass: the vector keeps its fp32 codes and gets the marker
-    // parameter (fixup pass); fixup pass: exact_fast re-takes them
-    const uint32_t bits = (uint32_t)A.c.bits;
+    // ---- decisions in doubt: the vector keeps its fp32 codes and gets the
+    // marker parameter; encode_fixup_kernel re-encodes it exactly -----------
     const bool lane_need = valid && ((need_a | need_n) != 0u || need_p);
-    if constexpr (!EXACT) {
-        if (group_any<NL>(lane_need)) prm = lin8 ? kFixupMark16 : kFixupMark32;
-    } else if (__any_sync(KVQ_FULL_MASK, lane_need)) {
-#pragma unroll
-        for (int k = 0; k < 16; k++) st[(kFsNv + k) * 32] = __float_as_uint(nv[k]);
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            st[(kFsQ4 + j) * 32] = q4[j];
-            st[(kFsNc + j) * 32] = nc[j];
-        }
-        st[kFsNeedA * 32] = need_a;
-        st[kFsNeedN * 32] = need_n;
-        st[kFsPrm * 32] = prm;
-        st[kFsPmin * 32] = __float_as_uint(pmin);
-        st[kFsPmax * 32] = __float_as_uint(pmax);
-        st[kFsPband * 32] = __float_as_uint(pband);
-        st[kFsFlags * 32] = (valid ? kFsValid : 0u) | (need_p ? kFsNeedP : 0u) |
-                            (unsure ? kFsUnsure : 0u) | (inexact ? kFsInexact : 0u);
-        exact_fast<D>(A.x, smask, valid ? v : 0u, lg, st, L, A.c.mode, (int)bits, bpr);
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            q4[j] = st[(kFsQ4 + j) * 32];
-            nc[j] = st[(kFsNc + j) * 32];
-        }
-        prm = st[kFsPrm * 32];
-    }
-
-    // ---- pack and store ------------------------------------------------------
-    // angle stream of this lane: 16 codes of b bits at bit 16 b lg of the row
-    const uint32_t s4 = 4u * bits;  // 16 .. 32
-    const uint32_t a0 = q4[0] | shl_c(q4[1], s4), a1 = shr_c(q4[1], 32u - s4);
-    const uint32_t b0 = q4[2] | shl_c(q4[3], s4), b1 = shr_c(q4[3], 32u - s4);
-    const uint32_t r8 = 8u * bits - 32u;  // 0 .. 32: offset of codes 8..15 past word 1
-    uint32_t o[4];
-    o[0] = a0;
-    o[1] = a1 | shl_c(b0, r8);
-    o[2] = shr_c(b0, 32u - r8) | shl_c(b1, r8);
-    o[3] = shr_c(b1, 32u - r8);
-    if (bits & 1u) {
-        // odd b: odd lanes start half way into a word; they hand their first
-        // 16 bits to the lane below, which completes its last word with them
-        const uint32_t up = __shfl_down_sync(KVQ_FULL_MASK, o[0], 1);
-        const uint32_t last = (bits - 1u) >> 1;  // half-filled word of an even lane
-        if (lg & 1) {
-            o[0] = __funnelshift_r(o[0], o[1], 16);
-            o[1] = __funnelshift_r(o[1], o[2], 16);
-            o[2] = __funnelshift_r(o[2], o[3], 16);
-            o[3] >>= 16;
-        } else {
-#pragma unroll
-            for (int j = 0; j < 4; j++)
-                if ((uint32_t)j == last) o[j] |= up << 16;
-        }
-    }
-    if (valid) {
-        const uint32_t vt = fast_div(v, A.tdiv);
-        bool bad = false;
-        const int64_t row =
-            plane_row_bh(A.out, A.bh0 + vt, A.pos0 + (int64_t)(v - vt * (uint32_t)A.T), &bad);
-        if (bad && lg == 0) report(A.err_word, KVQ_DEVERR_PAGE_RANGE);
-        // this lane's words: [ceil(lg b / 2), ceil((lg + 1) b / 2))
-        const uint32_t w0 = ((uint32_t)lg * bits + 1u) >> 1;
-        const uint32_t nw = (((uint32_t)lg + 1u) * bits + 1u) / 2u - w0;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(A.out.angles) + row * A.c.angle_words + w0;
-#pragma unroll
-        for (int j = 0; j < 4; j++)
-            if ((uint32_t)j < nw) dst[j] = o[j];
-        if (lin8) {
-            *reinterpret_cast<uint4*>(A.out.norms + row * (D / 2) + lg * 16) =
-                make_uint4(nc[0], nc[1], nc[2], nc[3]);
-            if (lg == 0) reinterpret_cast<uint16_t*>(A.out.params)[row] = (uint16_t)prm;
-        } else {
-            *reinterpret_cast<uint2*>(A.out.norms + row * (D / 4) + lg * 8) = make_uint2(nc[0], nc[1]);
-            if (lg == 0) reinterpret_cast<uint32_t*>(A.out.params)[row] = prm;
-        }
-    }
+    if (group_any<NL>(lane_need)) prm = lin8 ? kFixupMark16 : kFixupMark32;
+    store_codes<D>(A, v, valid, lg, q4, nc, prm);
 }
 
 // Streaming pass: grid-stride over warp tiles; blockIdx.y selects the tensor
@@ -559,20 +366,85 @@ encode_fast_kernel(EncPair PA) {
     const uint32_t n_tiles = (uint32_t)((A.n_vec + Cfg::VPW - 1) / Cfg::VPW);
     const uint32_t stride = gridDim.x * kFastWarps;
     for (uint32_t wt = blockIdx.x * kFastWarps + warp; wt < n_tiles; wt += stride)
-        encode_tile_fast<D, false>(A, wt * Cfg::VPW + grp, masks[lg], lg, pwk, nullptr);
+        encode_tile_fast<D>(A, wt * Cfg::VPW + grp, masks[lg], lg, pwk);
+}
+
+// Exact re-encode of one vector per group (fixup pass).  The transform runs
+// in fp64, where it is exact for fp16 inputs (partial sums over at most 256
+// multiples of 2^-24 below 2^16 fit in 53 bits); then every decision follows
+// the definition:
+//   - angle: the fp32 polynomial on the exact pair, and where that lies
+//     within its slack of an edge, atan2 and the bin formula in fp64
+//     (angle_code_from_exact);
+//   - norms and parameters: the fp64 formulas of exact_path.
+template <int D>
+__device__ __forceinline__ void fixup_tile(const EncArgs& A, uint32_t v, const uint32_t* smask,
+                                           int lg, const uint32_t (&pwk)[4]) {
+    using Cfg = FastCfg<D>;
+    constexpr int NL = Cfg::NL;
+    const bool valid = (int64_t)v < A.n_vec;
+    const int L = A.c.L;
+    const bool lin8 = A.c.mode == KVQ_NORM_LIN8;
+    double z[32];  // H D x (unscaled) at this lane's 32 indices
+    {
+        uint32_t raw[16];
+        fast_load<D>(A, valid ? v : 0u, lg, smask, raw);
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&raw[k]));
+            z[2 * k] = (double)f.x;
+            z[2 * k + 1] = (double)f.y;
+        }
+    }
+    fwht_local<32>(z);
+    fwht_cross<32, NL>(z, lg);
+
+    const float bpr = A.bins_per_rad;
+    uint32_t q4[4] = {0u, 0u, 0u, 0u};
+    double x[16];  // r (LIN8) or log2 max(r, 2^-24) (LOG4) of each pair
+    double ext_hi = lin8 ? 0.0 : -1e300, ext_lo = 1e300;
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        const double z0 = z[2 * i], z1 = z[2 * i + 1];
+        const int a = angle_code_from_exact(z0, z1, L, bpr);
+        q4[i >> 2] += (uint32_t)a * pwk[i & 3];
+        const double r2 = fma(z0, z0, z1 * z1) * (1.0 / D);
+        x[i] = lin8 ? sqrt(r2) : 0.5 * exact_log2_sq(r2);
+        ext_hi = fmax(ext_hi, x[i]);
+        ext_lo = fmin(ext_lo, x[i]);
+    }
+    ext_hi = group_max_d<NL>(ext_hi);
+    ext_lo = group_min_d<NL>(ext_lo);
+    uint32_t nc[4] = {0u, 0u, 0u, 0u};
+    uint32_t prm;
+    if (lin8) {
+        prm = f64_to_f16_sat(ext_hi);
+        const double M = (double)half_bits_to_float((uint16_t)prm);
+#pragma unroll
+        for (int i = 0; i < 16; i++)
+            nc[i >> 2] |= (uint32_t)lin8_code_exact(x[i], M) << (8 * (i & 3));
+    } else {
+        const uint16_t LOh = f64_to_f16_sat(ext_lo), HIh = f64_to_f16_sat(ext_hi);
+        prm = (uint32_t)LOh | ((uint32_t)HIh << 16);
+        const double LO = (double)half_bits_to_float(LOh), HI = (double)half_bits_to_float(HIh);
+#pragma unroll
+        for (int i = 0; i < 16; i++)
+            nc[i >> 3] |= (uint32_t)log4_code_exact(x[i], LO, HI) << (4 * (i & 7));
+    }
+    store_codes<D>(A, v, valid, lg, q4, nc, prm);
 }
 
 // Fixup pass: every lane reads the parameter of one vector; the marked ones
-// are gathered, VPW at a time (one per group), and encoded again with their
-// decisions in doubt re-taken exactly.
+// queue per warp and are re-encoded VPW at a time (one per group).
 template <int D>
-__global__ void __launch_bounds__(kFastWarps * 32, kFastBlocksPerSM)
+__global__ void __launch_bounds__(kFastWarps * 32, 1)
 encode_fixup_kernel(EncPair PA) {
     asm volatile("griddepcontrol.launch_dependents;");
     const EncArgs A = blockIdx.y ? PA.a[1] : PA.a[0];
     using Cfg = FastCfg<D>;
+    constexpr uint32_t VPW = Cfg::VPW;
     __shared__ __align__(16) uint32_t masks[Cfg::NL][16];
-    __shared__ uint32_t state[kFastWarps][kFsWords * 32];
+    __shared__ uint32_t queue[kFastWarps][64];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int grp = lane / Cfg::NL, lg = lane % Cfg::NL;
     if (threadIdx.x < Cfg::NL) fast_sign_masks(A.signs, threadIdx.x, masks[threadIdx.x]);
@@ -583,6 +455,8 @@ encode_fixup_kernel(EncPair PA) {
     const uint32_t n = (uint32_t)A.n_vec;
     const uint32_t n_chunks = (n + 31u) / 32u;
     const uint32_t stride = gridDim.x * kFastWarps;
+    uint32_t* q = queue[warp];
+    uint32_t head = 0, tail = 0;  // ring of 64: fewer than VPW + 32 entries at any time
     for (uint32_t ch = blockIdx.x * kFastWarps + warp; ch < n_chunks; ch += stride) {
         const uint32_t v = ch * 32u + (uint32_t)lane;
         bool marked = false;
@@ -594,14 +468,20 @@ encode_fixup_kernel(EncPair PA) {
             marked = lin8 ? reinterpret_cast<const uint16_t*>(A.out.params)[row] == kFixupMark16
                           : reinterpret_cast<const uint32_t*>(A.out.params)[row] == kFixupMark32;
         }
-        uint32_t bal = __ballot_sync(KVQ_FULL_MASK, marked);
-        while (bal) {
-            // group g takes the (g+1)-th marked vector, if there is one
-            const uint32_t pos = __fns(bal, 0, grp + 1);
-            const uint32_t vg = pos < 32u ? ch * 32u + pos : n;  // n: no vector
-            encode_tile_fast<D, true>(A, vg, masks[lg], lg, pwk, state[warp] + lane);
-            for (int g = 0; g < Cfg::VPW && bal; g++) bal &= bal - 1u;
+        const uint32_t bal = __ballot_sync(KVQ_FULL_MASK, marked);
+        if (marked) q[(tail + __popc(bal & ((1u << lane) - 1u))) & 63u] = v;
+        tail += __popc(bal);
+        __syncwarp();
+        while (tail - head >= VPW) {
+            const uint32_t vg = q[(head + grp) & 63u];
+            __syncwarp();
+            fixup_tile<D>(A, vg, masks[lg], lg, pwk);
+            head += VPW;
         }
+    }
+    if (tail != head) {
+        const uint32_t vg = (uint32_t)grp < tail - head ? q[(head + grp) & 63u] : n;  // n: none
+        fixup_tile<D>(A, vg, masks[lg], lg, pwk);
     }
 }
 
