@@ -50,11 +50,11 @@ static cudaError_t launch_encode_d(const EncPair& pa, int n_args, int sm_count,
 }
 
 // The streaming and fixup kernels of kvq_encode_fast.cuh cover d = 64, 128,
-// 256 and L % 8 == 0 with 16 <= L <= 256, for fewer than 2^32 vectors.
+// 256 and L % 8 == 0 with 16 <= L <= 256, for at most 2^31 vectors.
 static bool fast_ok(const EncodeJob& j) {
     const int d = j.c.d, L = j.c.L;
     return (d == 64 || d == 128 || d == 256) && L % 8 == 0 && L >= 16 && L <= 256 &&
-           j.n_vec <= (1ll << 32) - 64 && j.T >= 1;
+           j.n_vec <= (1ll << 31) && j.T >= 1;
 }
 
 template <int D>
@@ -70,8 +70,8 @@ static cudaError_t launch_encode_fast_d(const EncPair& pa, int n_args, int sm_co
     if (blocks < 1) blocks = 1;
     encode_fast_kernel<D>
         <<<dim3((unsigned)blocks, (unsigned)n_args), kFastWarps * 32, 0, stream>>>(pa);
-    // the fixup pass: one warp per 32 vectors, one block per SM at most
-    int64_t fblocks = ((n_max + 31) / 32 + kFastWarps - 1) / kFastWarps;
+    // the fixup pass: one warp per 128 vectors, one block per SM at most
+    int64_t fblocks = ((n_max + 127) / 128 + kFastWarps - 1) / kFastWarps;
     if (fblocks > sm_count / n_args) fblocks = sm_count / n_args;
     if (fblocks < 1) fblocks = 1;
     encode_fixup_kernel<D>

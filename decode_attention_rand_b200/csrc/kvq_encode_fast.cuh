@@ -236,35 +236,42 @@ __device__ __forceinline__ void encode_tile_fast(const EncArgs& A, uint32_t v,
     const float sc = (float)(S == 6 ? 0.17677669529663687 : S == 7 ? 0.125 : 0.08838834764831845);
 
     // ---- angles ------------------------------------------------------------
+    // Rounding uses the 2^23 trick: for 0 <= y < 2^22, y + (2^23 - 1/2) rounds
+    // to 2^23 + floor(y) (a tie, y an integer, lands on a decision edge and is
+    // in doubt anyway), so the float's low bits are floor(y); the decision's
+    // distance to its edges comes from |y - (floor(y) + 1/2)|, kept as a
+    // running maximum: the streaming pass only needs to know whether any
+    // decision of the vector is in doubt.
     const float bpr = A.bins_per_rad;
     const float u0 = 0.625f * (float)L;  // 5L/8
     const float du = angle_margin(A);
+    constexpr float kMagicFloor = 8388607.5f;  // 2^23 - 1/2
+    constexpr float kMagicRound = 8388608.f;   // 2^23
+    constexpr int kMagicBits = 0x4B000000;     // bits of 2^23
     uint32_t q4[4] = {0u, 0u, 0u, 0u};  // angle codes, four per word
-    uint32_t need_a = 0;
+    float amax = 0.f;                   // max |u - (floor(u) + 1/2)|
     float rw2[16];
 #pragma unroll
     for (int k = 0; k < 16; k++) {
         const float a = lo2(P[k]), b = hi2(P[k]);
         rw2[k] = fmaf(a, a, b * b);
-        const float th = atan2_poly(b, a);
-        const float u = fmaf(th, -bpr, u0);
-        const float fl = floorf(u);
-        const float fr = u - fl;
-        int c = (int)fl;
+        const float u = fmaf(atan2_poly(b, a), -bpr, u0);  // in [L/8, 9L/8]
+        const float tm = u + kMagicFloor;
+        int c = __float_as_int(tm) - kMagicBits;
         c = c >= L ? c - L : c;
-        // an exactly zero pair has code 0 (its fr is NaN: never flagged)
+        // an exactly zero pair has code 0 (its u is NaN, which fmaxf drops)
         c = rw2[k] > 0.f ? c : 0;
         q4[k >> 2] += (uint32_t)c * pwk[k & 3];
-        need_a |= (0.5f - fabsf(fr - 0.5f) < du) ? (1u << k) : 0u;
+        amax = fmaxf(amax, fabsf(u - (tm - kMagicFloor)));
     }
+    bool doubt = amax > 0.5f - du;
 
     // ---- norms and parameters (the formulas and slacks of encode_tile) ----
     uint32_t nc[4] = {0u, 0u, 0u, 0u};  // norm codes: 4 bytes (LIN8) / 8 nibbles (LOG4) a word
-    float nv[16];  // LIN8: |w pair|; LOG4: fp32 log2 r
-    uint32_t prm = 0, need_n = 0;
-    bool need_p = false, unsure = false;
-    float pmax = 0.f, pmin = 0.f, pband = 0.f;
+    uint32_t prm = 0;
+    float nmax = 0.f;  // max over the codes of (distance to the nearest integer + slack)
     if (lin8) {
+        float nv[16];  // |w pair|
         float m = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; k++) {
@@ -272,32 +279,29 @@ __device__ __forceinline__ void encode_tile_fast(const EncArgs& A, uint32_t v,
             m = fmaxf(m, nv[k]);
         }
         m = group_max<NL>(m) * sc;  // max r
-        const float eM = m * 1e-6f;
-        need_p = near_f16_midpoint(m, eM);
-        pmax = m;
-        pband = 2.f * eM;
+        doubt |= near_f16_midpoint(m, m * 1e-6f);
         const uint16_t Mh = f32_to_f16_sat(m);
         const float Mf = half_bits_to_float(Mh);
         prm = Mh;
-        const float inv = Mf > 0.f ? 255.f * rcp_approx(Mf) : 0.f;
-        const float invw = inv * sc;
+        const float invw = Mf > 0.f ? 255.f * rcp_approx(Mf) * sc : 0.f;
 #pragma unroll
         for (int k = 0; k < 16; k++) {
+            // c = floor(vq + 1/2), in doubt within vq 1.2e-6 + 2e-6 of the edge
             const float vq = nv[k] * invw;
-            const float t = vq + 0.5f;
-            const float fl = floorf(t);
-            const float fr = t - fl;
-            const float dv = fmaf(vq, 1.2e-6f, 2e-6f);
-            if (Mf > 0.f && (fr < dv || fr > 1.f - dv)) need_n |= 1u << k;
-            const uint32_t c = Mf > 0.f ? (uint32_t)min(255, (int)fl) : 0u;
+            const float tq = vq + kMagicRound;
+            const uint32_t c = (uint32_t)min(255, __float_as_int(tq) - kMagicBits);
             nc[k >> 2] |= c << (8 * (k & 3));
+            nmax = fmaxf(nmax, fmaf(vq, 1.2e-6f, fabsf(vq - (tq - kMagicRound))));
         }
+        doubt |= nmax > 0.5f - 2e-6f;
     } else {
         // l = log2 max(r, 2^-24) with r^2 = (2/d) rw2:
         // l = (log2 max(rw2, 2^(S-49)) + 1 - S) / 2
         const float lfloor = __uint_as_float((uint32_t)(S - 49 + 127) << 23);
         const float tiny = __uint_as_float((uint32_t)(S - 45 + 127) << 23);  // r < 2^-22
+        float nv[16];  // fp32 log2 r
         float lmin = 1e30f, lmax = -1e30f;
+        bool unsure = false;
 #pragma unroll
         for (int k = 0; k < 16; k++) {
             nv[k] = fmaf(0.5f, lg2_approx(fmaxf(rw2[k], lfloor)), 0.5f * (float)(1 - S));
@@ -308,40 +312,31 @@ __device__ __forceinline__ void encode_tile_fast(const EncArgs& A, uint32_t v,
         unsure &= !zero;  // a zero vector is exact: every l is -24
         lmin = group_min<NL>(lmin);
         lmax = group_max<NL>(lmax);
-        unsure = group_any<NL>(unsure);
         // log2 error of a pair norm (relative 1e-6 of r, lg2 approximation),
         // as in encode_tile, plus 2^-23 of |l|
-        const float elmax = fmaf(fmaxf(fabsf(lmin), fabsf(lmax)), 1.2e-7f, 2.6717e-6f);
-        need_p = unsure || near_f16_midpoint(lmin, elmax) || near_f16_midpoint(lmax, elmax);
-        pmin = lmin;
-        pmax = lmax;
-        pband = 2.f * elmax;
+        const float lab = fmaxf(fabsf(lmin), fabsf(lmax));
+        const float elmax = fmaf(lab, 1.2e-7f, 2.6717e-6f);
+        doubt |= unsure || near_f16_midpoint(lmin, elmax) || near_f16_midpoint(lmax, elmax);
         const uint16_t LOh = f32_to_f16_sat(lmin), HIh = f32_to_f16_sat(lmax);
         const float LOf = half_bits_to_float(LOh), HIf = half_bits_to_float(HIh);
         prm = (uint32_t)LOh | ((uint32_t)HIh << 16);
         const float inv = HIf != LOf ? 15.f * rcp_approx(HIf - LOf) : 0.f;
+        // encode_tile's per-code slack with |l| bounded by the vector's largest
+        const float dvc = (2.6717e-6f + (lab + fabsf(LOf)) * 1.2e-7f) * inv * 1.02f + 2e-6f;
 #pragma unroll
         for (int k = 0; k < 16; k++) {
-            const float vq = (nv[k] - LOf) * inv;
-            const float t = vq + 0.5f;
-            const float fl = floorf(t);
-            const float fr = t - fl;
-            const float dv = (2.6717e-6f + (fabsf(nv[k]) + fabsf(LOf)) * 1.2e-7f) * inv * 1.02f +
-                             fabsf(vq) * 1e-6f + 2e-6f;
-            if (HIf != LOf && (fr < dv || fr > 1.f - dv)) need_n |= 1u << k;
-            const uint32_t c = HIf != LOf ? (uint32_t)min(15, max(0, (int)fl)) : 0u;
-            nc[k >> 3] |= c << (4 * (k & 7));
+            const float vq = fminf(fmaxf((nv[k] - LOf) * inv, 0.f), 15.f);
+            const float tq = vq + kMagicRound;
+            nc[k >> 3] |= (uint32_t)(__float_as_int(tq) - kMagicBits) << (4 * (k & 7));
+            nmax = fmaxf(nmax, fmaf(vq, 1e-6f, fabsf(vq - (tq - kMagicRound))));
         }
+        doubt |= nmax > 0.5f - dvc;
     }
-    if (inexact) {
-        need_a = need_n = 0xFFFFu;
-        need_p = unsure = true;
-    }
+    doubt |= inexact;
 
     // ---- decisions in doubt: the vector keeps its fp32 codes and gets the
     // marker parameter; encode_fixup_kernel re-encodes it exactly -----------
-    const bool lane_need = valid && ((need_a | need_n) != 0u || need_p);
-    if (group_any<NL>(lane_need)) prm = lin8 ? kFixupMark16 : kFixupMark32;
+    if (group_any<NL>(valid && doubt)) prm = lin8 ? kFixupMark16 : kFixupMark32;
     store_codes<D>(A, v, valid, lg, q4, nc, prm);
 }
 
@@ -457,31 +452,46 @@ encode_fixup_kernel(EncPair PA) {
     const uint32_t stride = gridDim.x * kFastWarps;
     uint32_t* q = queue[warp];
     uint32_t head = 0, tail = 0;  // ring of 64: fewer than VPW + 32 entries at any time
-    for (uint32_t ch = blockIdx.x * kFastWarps + warp; ch < n_chunks; ch += stride) {
-        const uint32_t v = ch * 32u + (uint32_t)lane;
-        bool marked = false;
-        if (v < n) {
-            const uint32_t vt = fast_div(v, A.tdiv);
-            bool bad = false;
-            const int64_t row =
-                plane_row_bh(A.out, A.bh0 + vt, A.pos0 + (int64_t)(v - vt * (uint32_t)A.T), &bad);
-            marked = lin8 ? reinterpret_cast<const uint16_t*>(A.out.params)[row] == kFixupMark16
-                          : reinterpret_cast<const uint32_t*>(A.out.params)[row] == kFixupMark32;
+    // four chunks of 32 vectors per step, their parameter loads in flight
+    // together; after the last step the queue is drained.  The (large) fixup
+    // tile has a single call site.
+    for (uint32_t c0 = (blockIdx.x * kFastWarps + warp) * 4u;; c0 += stride * 4u) {
+        const bool more = c0 < n_chunks;
+        uint32_t marked = 0;  // bit j: vector (c0 + j) * 32 + lane is marked
+        if (more) {
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t v = (c0 + (uint32_t)j) * 32u + (uint32_t)lane;
+                if (v < n) {
+                    const uint32_t vt = fast_div(v, A.tdiv);
+                    bool bad = false;
+                    const int64_t row = plane_row_bh(
+                        A.out, A.bh0 + vt, A.pos0 + (int64_t)(v - vt * (uint32_t)A.T), &bad);
+                    const bool mk = lin8
+                        ? reinterpret_cast<const uint16_t*>(A.out.params)[row] == kFixupMark16
+                        : reinterpret_cast<const uint32_t*>(A.out.params)[row] == kFixupMark32;
+                    marked |= mk ? 1u << j : 0u;
+                }
+            }
         }
-        const uint32_t bal = __ballot_sync(KVQ_FULL_MASK, marked);
-        if (marked) q[(tail + __popc(bal & ((1u << lane) - 1u))) & 63u] = v;
-        tail += __popc(bal);
-        __syncwarp();
-        while (tail - head >= VPW) {
-            const uint32_t vg = q[(head + grp) & 63u];
+#pragma unroll 1
+        for (int j = 0; j < 4; j++) {
+            const bool mk = (marked >> j) & 1u;
+            const uint32_t bal = __ballot_sync(KVQ_FULL_MASK, mk);
+            if (mk)
+                q[(tail + __popc(bal & ((1u << lane) - 1u))) & 63u] =
+                    (c0 + (uint32_t)j) * 32u + (uint32_t)lane;
+            tail += __popc(bal);
             __syncwarp();
-            fixup_tile<D>(A, vg, masks[lg], lg, pwk);
-            head += VPW;
+            while (tail - head >= VPW || (!more && tail != head)) {
+                const uint32_t cnt = min(tail - head, VPW);
+                const uint32_t vg = (uint32_t)grp < cnt ? q[(head + grp) & 63u] : n;  // n: none
+                __syncwarp();
+                fixup_tile<D>(A, vg, masks[lg], lg, pwk);
+                head += cnt;
+            }
         }
-    }
-    if (tail != head) {
-        const uint32_t vg = (uint32_t)grp < tail - head ? q[(head + grp) & 63u] : n;  // n: none
-        fixup_tile<D>(A, vg, masks[lg], lg, pwk);
+        if (!more) break;
     }
 }
 
