@@ -2,7 +2,9 @@
 // codebooks with L % 8 == 0, 16 <= L <= 256 (angle codes of 4 to 8 bits);
 // codec of "TurboAngle: Near-Lossless KV Cache Compression via Uniform Angle
 // Quantization", Abstract.  Produces the same codes as encode_tile, byte for
-// byte, with a third of its instructions.
+// byte, with about half of its instructions, in two passes: a streaming pass
+// that decides everything in fp32 and marks the vectors with a decision
+// within its error margin, and a fixup pass that re-encodes those exactly.
 //
 // Layout: 32 elements per lane, NL = d / 32 lanes per vector, 32 / NL vectors
 // per warp tile; 128-bit streaming loads.
@@ -21,9 +23,9 @@
 // transform of hi is exact in fp32.  lo is a multiple of 2^-24 (as every fp16
 // value is) below 2^(E+S-25), and its transform is exact too when
 // E <= 26 - 2S.  Then w = hi_w + lo_w exactly, the decisions see w rounded
-// once to fp32 (the slacks of encode_tile cover that), and a decision in doubt
-// is re-taken from the exact pair, formed in fp64, by exact_fast.  Vectors
-// with a larger E (|x| >= 2^(27-2S)) go through the general fp64 path.
+// once to fp32 (the slacks of encode_tile cover that).  Vectors with a larger
+// E (|x| >= 2^(27-2S)) are marked for the fixup pass, whose transform runs in
+// fp64.
 #pragma once
 
 #include "kvq_encode_impl.cuh"
