@@ -241,6 +241,36 @@ __device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
     return d;
 }
 
+// Walsh-Hadamard butterflies over every index bit but bit 0, for 32 elements
+// per lane held as 16 packed pairs (w[2k], w[2k+1]) in P[k]: local stages on
+// pair strides 1, 2, 4, 8, then the NL lanes of the group.
+template <int NL>
+__device__ __forceinline__ void fwht_pairs(f32x2 (&P)[16], int lg) {
+#pragma unroll
+    for (int s = 1; s < 16; s <<= 1) {
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            if ((k & s) == 0) {
+                const f32x2 a = P[k], b = P[k + s];
+                P[k] = add2(a, b);
+                P[k + s] = sub2(a, b);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 1; m < NL; m <<= 1) {
+        // lower lane: own + other; upper lane: other - own
+        const float sg = (lg & m) ? -1.f : 1.f;
+        const f32x2 sg2 = pack2(sg, sg);
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            const uint32_t lo = __shfl_xor_sync(KVQ_FULL_MASK, (uint32_t)P[k], m);
+            const uint32_t hi = __shfl_xor_sync(KVQ_FULL_MASK, (uint32_t)(P[k] >> 32), m);
+            P[k] = fma2(sg2, P[k], ((f32x2)hi << 32) | lo);
+        }
+    }
+}
+
 // ------------------------------------------------------ device errors ----
 
 __device__ __forceinline__ void report(int32_t* err_word, int bits) {

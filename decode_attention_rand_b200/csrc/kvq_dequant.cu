@@ -33,6 +33,7 @@ struct DqArgs {
     CodecDev c;
     __half* y;
     float inv_sqrt_d;
+    FastDiv tdiv;  // division by T (fast kernel: n_vec <= 2^31)
 };
 
 // Bits [0, 128) of a lane's code chunk that starts at bit `cb` of a row of
@@ -170,6 +171,141 @@ dequant_kernel(DqArgs A) {
     }
 }
 
+// ------------------------------------------------------------ fast path --
+// d = 64, 128, 256 and L <= 256 (codes of B <= 8 bits, B a template
+// parameter): 32 elements per lane, d/32 lanes per vector.  The butterfly
+// inside each element pair is applied to the table instead of the data:
+// (z[2i], z[2i+1]) = r (cos, sin) becomes r (cos + sin, cos - sin), the
+// remaining index bits go through the packed fp32 transform, 1/sqrt(d) rides
+// on r and the signs of D on the fp16 sign bits.
+
+template <int D>
+struct DqFastCfg {
+    static constexpr int NL = D / 32;    // lanes per vector
+    static constexpr int VPW = 32 / NL;  // vectors per warp tile
+    static constexpr int S = D == 64 ? 6 : D == 128 ? 7 : 8;
+};
+
+template <int D, int B>
+__global__ void __launch_bounds__(kDqWarps * 32)
+dequant_fast_kernel(DqArgs A) {
+    using Cfg = DqFastCfg<D>;
+    constexpr int NL = Cfg::NL, VPW = Cfg::VPW, S = Cfg::S;
+    __shared__ float2 tab[256];                        // r-free (cos + sin, cos - sin)
+    __shared__ __align__(16) uint32_t masks[NL][16];  // fp16 sign bits of D
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int grp = lane / NL, lg = lane % NL;
+    const int L = A.c.L;
+    for (int j = threadIdx.x; j < L; j += blockDim.x) {
+        float sn, cs;
+        sincospif((float)(2 * j + 1) / (float)L - 1.f, &sn, &cs);
+        tab[j] = make_float2(cs + sn, cs - sn);
+    }
+    if (threadIdx.x < NL) {
+#pragma unroll
+        for (int w = 0; w < 16; w++) {
+            const int e = threadIdx.x * 32 + 2 * w;
+            masks[threadIdx.x][w] =
+                (A.signs[e] < 0 ? 0x8000u : 0u) | (A.signs[e + 1] < 0 ? 0x80000000u : 0u);
+        }
+    }
+    __syncthreads();
+    const int AW = A.c.angle_words;
+    const bool lin8 = A.c.mode == KVQ_NORM_LIN8;
+    const float isd = A.inv_sqrt_d;
+    // this lane's 16 codes start at bit 16 B lg of the row
+    const int wbase = (lg * 16 * B) >> 5, sh = (lg * 16 * B) & 31;
+    const uint32_t n_tiles = (uint32_t)((A.n_vec + VPW - 1) / VPW);
+    const uint32_t stride = gridDim.x * kDqWarps;
+    for (uint32_t wt = blockIdx.x * kDqWarps + warp; wt < n_tiles; wt += stride) {
+        const uint32_t v = wt * VPW + grp;
+        const bool valid = (int64_t)v < A.n_vec;
+        const uint32_t vv = valid ? v : 0u;
+        const uint32_t vt = fast_div(vv, A.tdiv);
+        const int64_t row =
+            (int64_t)vt * A.in.capacity + A.pos0 + (int64_t)(vv - vt * (uint32_t)A.T);
+        // angle codes: up to five words, aligned to the lane's first bit
+        uint32_t W[4];
+        {
+            const uint32_t* ar = reinterpret_cast<const uint32_t*>(A.in.angles) + row * AW;
+            uint32_t w[5];
+#pragma unroll
+            for (int j = 0; j < 5; j++) w[j] = wbase + j < AW ? ar[wbase + j] : 0u;
+#pragma unroll
+            for (int j = 0; j < 4; j++) W[j] = __funnelshift_r(w[j], w[j + 1], sh);
+        }
+        // norms: r / sqrt(d) of each pair
+        float r[16];
+        if (lin8) {
+            const uint4 nq = *reinterpret_cast<const uint4*>(A.in.norms + row * (D / 2) + lg * 16);
+            const uint32_t nw[4] = {nq.x, nq.y, nq.z, nq.w};
+            const float sc = half_bits_to_float(reinterpret_cast<const uint16_t*>(A.in.params)[row]) *
+                             (1.f / 255.f) * isd;
+#pragma unroll
+            for (int k = 0; k < 16; k++)
+                r[k] = (float)((nw[k >> 2] >> (8 * (k & 3))) & 0xFFu) * sc;
+        } else {
+            const uint2 nq = *reinterpret_cast<const uint2*>(A.in.norms + row * (D / 4) + lg * 8);
+            const uint32_t pr = reinterpret_cast<const uint32_t*>(A.in.params)[row];
+            const float LO = half_bits_to_float((uint16_t)(pr & 0xFFFF));
+            const float step = (half_bits_to_float((uint16_t)(pr >> 16)) - LO) * (1.f / 15.f);
+            // 2^(LO + c step) / sqrt(d) = 2^(LO - S/2 + c step)
+            const float base = LO - 0.5f * (float)S;
+#pragma unroll
+            for (int k = 0; k < 16; k++) {
+                const uint32_t c = ((k < 8 ? nq.x : nq.y) >> (4 * (k & 7))) & 0xFu;
+                r[k] = exp2f(fmaf((float)c, step, base));
+            }
+        }
+        f32x2 P[16];
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            constexpr uint32_t mask = (1u << B) - 1u;
+            const int pos = k * B, wi = pos >> 5, bi = pos & 31;
+            const uint32_t a = (bi + B <= 32 ? (W[wi] >> bi) : __funnelshift_r(W[wi], W[wi + 1], bi)) & mask;
+            const float2 t = tab[a];
+            P[k] = pack2(r[k] * t.x, r[k] * t.y);
+        }
+        fwht_pairs<NL>(P, lg);
+        if (valid) {
+            const uint32_t* m = masks[lg];
+            uint32_t o[16];
+#pragma unroll
+            for (int k = 0; k < 16; k++) {
+                const __half2 h = __floats2half2_rn(lo2(P[k]), hi2(P[k]));
+                o[k] = *reinterpret_cast<const uint32_t*>(&h) ^ m[k];
+            }
+            uint4* dst = reinterpret_cast<uint4*>(A.y + (size_t)v * D + lg * 32);
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+                dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        }
+    }
+}
+
+template <int D>
+static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStream_t stream) {
+    constexpr int VPW = DqFastCfg<D>::VPW;
+    const int64_t tiles = (a.n_vec + VPW - 1) / VPW;
+    int64_t blocks = (tiles + kDqWarps - 1) / kDqWarps;
+    const int64_t cap = (int64_t)sm_count * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    const dim3 g((unsigned)blocks), b(kDqWarps * 32);
+    switch (a.c.bits) {
+        case 1: dequant_fast_kernel<D, 1><<<g, b, 0, stream>>>(a); break;
+        case 2: dequant_fast_kernel<D, 2><<<g, b, 0, stream>>>(a); break;
+        case 3: dequant_fast_kernel<D, 3><<<g, b, 0, stream>>>(a); break;
+        case 4: dequant_fast_kernel<D, 4><<<g, b, 0, stream>>>(a); break;
+        case 5: dequant_fast_kernel<D, 5><<<g, b, 0, stream>>>(a); break;
+        case 6: dequant_fast_kernel<D, 6><<<g, b, 0, stream>>>(a); break;
+        case 7: dequant_fast_kernel<D, 7><<<g, b, 0, stream>>>(a); break;
+        case 8: dequant_fast_kernel<D, 8><<<g, b, 0, stream>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 template <int D>
 static cudaError_t launch_dequant_d(const DqArgs& a, int sm_count, cudaStream_t stream) {
     constexpr int VPW = DqCfg<D>::VPW;
@@ -194,6 +330,14 @@ cudaError_t launch_dequant(const CodecDev& c, const int8_t* signs, const PlaneDe
     a.c = c;
     a.y = y;
     a.inv_sqrt_d = (float)(1.0 / sqrt((double)c.d));
+    a.tdiv = make_fast_div(n_vec <= (1ll << 31) && T >= 1 ? (uint32_t)T : 1u);
+    if ((c.d == 64 || c.d == 128 || c.d == 256) && c.L <= 256 && n_vec <= (1ll << 31) && T >= 1) {
+        switch (c.d) {
+            case 64: return launch_dequant_fast_d<64>(a, sm_count, stream);
+            case 128: return launch_dequant_fast_d<128>(a, sm_count, stream);
+            default: return launch_dequant_fast_d<256>(a, sm_count, stream);
+        }
+    }
     switch (c.d) {
         case 4: return launch_dequant_d<4>(a, sm_count, stream);
         case 8: return launch_dequant_d<8>(a, sm_count, stream);

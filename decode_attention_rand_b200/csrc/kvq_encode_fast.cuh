@@ -82,35 +82,6 @@ __device__ __forceinline__ void fast_load(const EncArgs& A, uint32_t v, int lg,
 }
 
 
-// Transform over index bits 1 .. S-1 of 16 packed pairs: local butterflies on
-// pair strides 1, 2, 4, 8, then the lanes of the group.
-template <int NL>
-__device__ __forceinline__ void fwht_pairs(f32x2 (&P)[16], int lg) {
-#pragma unroll
-    for (int s = 1; s < 16; s <<= 1) {
-#pragma unroll
-        for (int k = 0; k < 16; k++) {
-            if ((k & s) == 0) {
-                const f32x2 a = P[k], b = P[k + s];
-                P[k] = add2(a, b);
-                P[k + s] = sub2(a, b);
-            }
-        }
-    }
-#pragma unroll
-    for (int m = 1; m < NL; m <<= 1) {
-        // lower lane: own + other; upper lane: other - own
-        const float sg = (lg & m) ? -1.f : 1.f;
-        const f32x2 sg2 = pack2(sg, sg);
-#pragma unroll
-        for (int k = 0; k < 16; k++) {
-            const uint32_t lo = __shfl_xor_sync(KVQ_FULL_MASK, (uint32_t)P[k], m);
-            const uint32_t hi = __shfl_xor_sync(KVQ_FULL_MASK, (uint32_t)(P[k] >> 32), m);
-            P[k] = fma2(sg2, P[k], ((f32x2)hi << 32) | lo);
-        }
-    }
-}
-
 // The split transform of the header: HI and LO hold the transforms of hi and
 // lo (pairs (w[2k], w[2k+1]) of this lane); E as defined there and whether
 // the vector is all zero (both uniform over the group).
