@@ -75,13 +75,14 @@ def parse():
                    help="wall time of the bounded oracle sample (cpu_baseline)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-encode", action="store_true")
-    p.add_argument("--case", default=None, choices=["decode_layer", "encode_layer"],
+    p.add_argument("--case", default=None, choices=["decode_layer", "encode_layer", "dequant_layer"],
                    help="run one kernel case only (for profiler captures): the decode of "
-                        "--layer of --workload, or the prefill encode of 8 batch entries of "
-                        "one layer; --steps launches after 3 warm-up launches")
+                        "--layer of --workload, or the prefill encode (or dequant) of 8 batch "
+                        "entries of one layer; --steps launches after 3 warm-up launches")
     p.add_argument("--layer", type=int, default=0)
     p.add_argument("--tensor", default="k", choices=["k", "v"],
-                   help="encode_layer case: encode the layer's K (8-bit linear norms) or V (4-bit log)")
+                   help="encode_layer / dequant_layer case: the layer's K (8-bit linear norms) "
+                        "or V (4-bit log)")
     return p.parse_args()
 
 
@@ -510,9 +511,17 @@ def run_case(args):
         x = synth.kv(w, 0, synth.KIND_K if isk else synth.KIND_V, device=device, b_range=(0, nb))
         skd = torch.from_numpy(sk if isk else sv).to(device)
 
-        def run():
+        if args.case == "encode_layer":
+            def run():
+                kvq.encode(c, skd, x, p, 0)
+            what = f"encode {w.name} layer 0 {'K' if isk else 'V'}, batch entries 0..{nb - 1}"
+        else:
             kvq.encode(c, skd, x, p, 0)
-        what = f"encode {w.name} layer 0 {'K' if isk else 'V'}, batch entries 0..{nb - 1}"
+            y = torch.empty_like(x)
+
+            def run():
+                kvq.dequant(c, skd, p, w.ctx, 0, out=y)
+            what = f"dequant {w.name} layer 0 {'K' if isk else 'V'}, batch entries 0..{nb - 1}"
     for _ in range(3):
         run()
     torch.cuda.synchronize()

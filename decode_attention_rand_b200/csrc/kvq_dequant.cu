@@ -187,29 +187,33 @@ struct DqFastCfg {
 };
 
 template <int D, int B>
-__global__ void __launch_bounds__(kDqWarps * 32)
+__global__ void __launch_bounds__(kDqWarps * 32, 4)
 dequant_fast_kernel(DqArgs A) {
     using Cfg = DqFastCfg<D>;
     constexpr int NL = Cfg::NL, VPW = Cfg::VPW, S = Cfg::S;
-    __shared__ float2 tab[256];                        // r-free (cos + sin, cos - sin)
-    __shared__ __align__(16) uint32_t masks[NL][16];  // fp16 sign bits of D
+    // r-free (cos + sin, cos - sin) of each bin centre, 16 copies side by side
+    // ([code][16]): lane l of a half warp reads copy l, so a lookup never
+    // shares a bank within the half warp
+    extern __shared__ float2 tab[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int grp = lane / NL, lg = lane % NL;
     const int L = A.c.L;
     for (int j = threadIdx.x; j < L; j += blockDim.x) {
         float sn, cs;
         sincospif((float)(2 * j + 1) / (float)L - 1.f, &sn, &cs);
-        tab[j] = make_float2(cs + sn, cs - sn);
-    }
-    if (threadIdx.x < NL) {
-#pragma unroll
-        for (int w = 0; w < 16; w++) {
-            const int e = threadIdx.x * 32 + 2 * w;
-            masks[threadIdx.x][w] =
-                (A.signs[e] < 0 ? 0x8000u : 0u) | (A.signs[e + 1] < 0 ? 0x80000000u : 0u);
-        }
+        tab[j * 16] = make_float2(cs + sn, cs - sn);
     }
     __syncthreads();
+    for (int i = threadIdx.x; i < L * 16; i += blockDim.x)
+        if (i & 15) tab[i] = tab[i & ~15];
+    uint32_t m[16];  // fp16 sign bits of D for this lane's element pairs
+#pragma unroll
+    for (int w = 0; w < 16; w++) {
+        const int e = lg * 32 + 2 * w;
+        m[w] = (A.signs[e] < 0 ? 0x8000u : 0u) | (A.signs[e + 1] < 0 ? 0x80000000u : 0u);
+    }
+    __syncthreads();
+    const float2* tl = tab + (lane & 15);
     const int AW = A.c.angle_words;
     const bool lin8 = A.c.mode == KVQ_NORM_LIN8;
     const float isd = A.inv_sqrt_d;
@@ -263,12 +267,11 @@ dequant_fast_kernel(DqArgs A) {
             constexpr uint32_t mask = (1u << B) - 1u;
             const int pos = k * B, wi = pos >> 5, bi = pos & 31;
             const uint32_t a = (bi + B <= 32 ? (W[wi] >> bi) : __funnelshift_r(W[wi], W[wi + 1], bi)) & mask;
-            const float2 t = tab[a];
+            const float2 t = tl[a * 16];
             P[k] = pack2(r[k] * t.x, r[k] * t.y);
         }
         fwht_pairs<NL>(P, lg);
         if (valid) {
-            const uint32_t* m = masks[lg];
             uint32_t o[16];
 #pragma unroll
             for (int k = 0; k < 16; k++) {
@@ -292,15 +295,16 @@ static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStre
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     const dim3 g((unsigned)blocks), b(kDqWarps * 32);
+    const size_t smem = (size_t)a.c.L * 16 * sizeof(float2);  // at most 32 KB
     switch (a.c.bits) {
-        case 1: dequant_fast_kernel<D, 1><<<g, b, 0, stream>>>(a); break;
-        case 2: dequant_fast_kernel<D, 2><<<g, b, 0, stream>>>(a); break;
-        case 3: dequant_fast_kernel<D, 3><<<g, b, 0, stream>>>(a); break;
-        case 4: dequant_fast_kernel<D, 4><<<g, b, 0, stream>>>(a); break;
-        case 5: dequant_fast_kernel<D, 5><<<g, b, 0, stream>>>(a); break;
-        case 6: dequant_fast_kernel<D, 6><<<g, b, 0, stream>>>(a); break;
-        case 7: dequant_fast_kernel<D, 7><<<g, b, 0, stream>>>(a); break;
-        case 8: dequant_fast_kernel<D, 8><<<g, b, 0, stream>>>(a); break;
+        case 1: dequant_fast_kernel<D, 1><<<g, b, smem, stream>>>(a); break;
+        case 2: dequant_fast_kernel<D, 2><<<g, b, smem, stream>>>(a); break;
+        case 3: dequant_fast_kernel<D, 3><<<g, b, smem, stream>>>(a); break;
+        case 4: dequant_fast_kernel<D, 4><<<g, b, smem, stream>>>(a); break;
+        case 5: dequant_fast_kernel<D, 5><<<g, b, smem, stream>>>(a); break;
+        case 6: dequant_fast_kernel<D, 6><<<g, b, smem, stream>>>(a); break;
+        case 7: dequant_fast_kernel<D, 7><<<g, b, smem, stream>>>(a); break;
+        case 8: dequant_fast_kernel<D, 8><<<g, b, smem, stream>>>(a); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
