@@ -70,9 +70,9 @@ static cudaError_t launch_encode_fast_d(const EncPair& pa, int n_args, int sm_co
     if (blocks < 1) blocks = 1;
     encode_fast_kernel<D>
         <<<dim3((unsigned)blocks, (unsigned)n_args), kFastWarps * 32, 0, stream>>>(pa);
-    // the fixup pass: one warp per 128 vectors, one block per SM at most
+    // the fixup pass: one warp per 128 vectors, two blocks per SM at most
     int64_t fblocks = ((n_max + 127) / 128 + kFastWarps - 1) / kFastWarps;
-    if (fblocks > sm_count / n_args) fblocks = sm_count / n_args;
+    if (fblocks > 2 * sm_count / n_args) fblocks = 2 * sm_count / n_args;
     if (fblocks < 1) fblocks = 1;
     encode_fixup_kernel<D>
         <<<dim3((unsigned)fblocks, (unsigned)n_args), kFastWarps * 32, 0, stream>>>(pa);

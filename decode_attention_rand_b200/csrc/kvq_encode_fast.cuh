@@ -405,7 +405,7 @@ __device__ __forceinline__ void fixup_tile(const EncArgs& A, uint32_t v, const u
 // Fixup pass: every lane reads the parameter of one vector; the marked ones
 // queue per warp and are re-encoded VPW at a time (one per group).
 template <int D>
-__global__ void __launch_bounds__(kFastWarps * 32, 1)
+__global__ void __launch_bounds__(kFastWarps * 32, 2)
 encode_fixup_kernel(EncPair PA) {
     asm volatile("griddepcontrol.launch_dependents;");
     const EncArgs A = blockIdx.y ? PA.a[1] : PA.a[0];
