@@ -238,13 +238,29 @@ class DecodeStep:
             for _ in range(1, self.nbuf):
                 planes.append(tuple(kvq.Plane(p.codec, p.B, p.H_kv, p.capacity, p.angles.clone(),
                                               p.norms.clone(), p.params.clone()) for p in bufs))
-            q = synth.queries(w, layer, device=device)
-            knew = synth.kv(w, layer, synth.KIND_K, device=device, T=1, salt=7)
-            vnew = synth.kv(w, layer, synth.KIND_V, device=device, T=1, salt=7)
+            q0 = synth.queries(w, layer, device=device)
+            k0 = synth.kv(w, layer, synth.KIND_K, device=device, T=1, salt=7)
+            v0 = synth.kv(w, layer, synth.KIND_V, device=device, T=1, salt=7)
+            # the step's inputs (q, new K, new V) in one buffer: one copy per
+            # layer and token when they come from the host
+            nq, nk = q0.numel(), k0.numel()
+            io = torch.empty(nq + 2 * nk, dtype=torch.float16, device=device)
+            q, knew, vnew = (io[:nq].view_as(q0), io[nq:nq + nk].view_as(k0),
+                             io[nq + nk:].view_as(v0))
+            q.copy_(q0)
+            knew.copy_(k0)
+            vnew.copy_(v0)
             out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float16, device=device)
-            self.layers.append(dict(kc=kc, vc=vc, skd=skd, svd=svd, planes=planes, q=q,
-                                    knew=knew, vnew=vnew, out=out,
-                                    cK=[p[0].c() for p in planes], cV=[p[1].c() for p in planes]))
+            L = dict(kc=kc, vc=vc, skd=skd, svd=svd, planes=planes, io=io, q=q, knew=knew,
+                     vnew=vnew, out=out, cK=[p[0].c() for p in planes],
+                     cV=[p[1].c() for p in planes])
+            # one kernel: append the new K and V at position ctx - 1, then attend
+            L["calls"] = [kvq.DecodeStepCall(q, knew, vnew, kc, vc, skd, svd, L["cK"][b],
+                                             L["cV"][b], self.ctx, w.B, w.H_q, w.H_kv, w.ctx,
+                                             self.tau, self.S, self.ws.buf, self.ws.nbytes,
+                                             self.err, out, kvq.OUT_FP16)
+                          for b in range(self.nbuf)]
+            self.layers.append(L)
         torch.cuda.synchronize(device)
         self.kernels_per_step = w.layers  # one fused append + decode launch per layer
 
@@ -255,11 +271,7 @@ class DecodeStep:
         for li, L in enumerate(self.layers):
             if ev is not None:
                 ev[li][0].record()
-            # one kernel: append the new K and V at position ctx - 1, then attend
-            kvq.kvq_decode_step(L["q"], L["knew"], L["vnew"], L["kc"], L["vc"], L["skd"],
-                                L["svd"], L["cK"][b], L["cV"][b], self.ctx, w.B, w.H_q, w.H_kv,
-                                w.ctx, self.tau, self.S, self.ws.buf, self.ws.nbytes, self.err,
-                                L["out"], kvq.OUT_FP16, st)
+            L["calls"][b](st)  # kvq_decode_step, arguments marshalled at setup
             if ev is not None:
                 ev[li][1].record()
 
@@ -329,22 +341,19 @@ def time_graph(state, K, W, dist_ctx):
 
 def time_e2e(state, K, dist_ctx):
     """Eager C-ABI calls with host buffers: per step copy q and the new K/V
-    from pinned memory, run the step, copy the attention output back."""
+    (one pinned buffer per layer) to the device, run the step, copy the
+    attention output back."""
     import torch
     w = state.w
-    hq = [L["q"].cpu().pin_memory() for L in state.layers]
-    hk = [L["knew"].cpu().pin_memory() for L in state.layers]
-    hv = [L["vnew"].cpu().pin_memory() for L in state.layers]
+    hin = [L["io"].cpu().pin_memory() for L in state.layers]  # q | new K | new V
     ho = [torch.empty_like(L["out"], device="cpu").pin_memory() for L in state.layers]
-    h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv)
+    h2d = sum(t.numel() * t.element_size() for t in hin)
     d2h = sum(t.numel() * t.element_size() for t in ho)
     cur = torch.cuda.current_stream()
 
     def one(i):
         for li, L in enumerate(state.layers):
-            L["q"].copy_(hq[li], non_blocking=True)
-            L["knew"].copy_(hk[li], non_blocking=True)
-            L["vnew"].copy_(hv[li], non_blocking=True)
+            L["io"].copy_(hin[li], non_blocking=True)
         state.step(i)
         for li, L in enumerate(state.layers):
             ho[li].copy_(L["out"], non_blocking=True)

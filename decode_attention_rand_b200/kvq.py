@@ -204,6 +204,28 @@ def kvq_decode_step(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, sign
                                  _stream(stream)))
 
 
+class DecodeStepCall:
+    """kvq_decode_step with its arguments marshalled once, for a serving loop
+    that calls it every token on the same buffers: the pointers, sizes and
+    codec structs are converted to ctypes values here, and each call passes
+    them unchanged (only the stream may vary).  The buffers must stay alive
+    and in place while the object is used."""
+
+    def __init__(self, q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v,
+                 K: kvq_plane, V: kvq_plane, ctx_len, B: int, H_q: int, H_kv: int,
+                 max_ctx: int, softmax_scale: float, num_splits: int, workspace, ws_bytes: int,
+                 err_word, out, out_dtype: int):
+        self._kc, self._vc, self._K, self._V = kc, vc, K, V  # keep the structs alive
+        self._fn = lib().kvq_decode_step
+        self._args = (_ptr(q), _ptr(k_new), _ptr(v_new), C.byref(kc), C.byref(vc),
+                      _ptr(signs_k), _ptr(signs_v), C.byref(K), C.byref(V), _ptr(ctx_len),
+                      B, H_q, H_kv, max_ctx, C.c_float(softmax_scale), num_splits,
+                      _ptr(workspace), ws_bytes, _ptr(err_word), _ptr(out), out_dtype)
+
+    def __call__(self, stream=None):
+        _check(self._fn(*self._args, _stream(stream)))
+
+
 def kvq_encode_kv_paged(kc: kvq_codec, signs_k, k, K: kvq_paged_plane, vc: kvq_codec, signs_v,
                         v, V: kvq_paged_plane, B: int, H_kv: int, T: int, pos0: int,
                         err_word=None, stream=None):

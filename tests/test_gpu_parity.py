@@ -343,6 +343,43 @@ def test_decode_step_equals_append_then_decode(dev, ctx_lens, splits, H_kv, G):
     compare_codes(plane_rows(Vs, t_range=(0, cap)), O.encode(v, sv, 64, O.MODE_LOG4))
 
 
+def test_decode_step_prepared_call_equals_call(dev):
+    """DecodeStepCall (arguments marshalled once) runs the same C entry point:
+    on twin caches it writes the same codes and returns the same output as
+    kvq_decode_step, and repeated calls keep doing so."""
+    d, B, H_kv, G = 128, 2, 2, 4
+    H_q, cap = G * H_kv, 512
+    kc, vc = kvq.codec(d, 128, O.MODE_LIN8), kvq.codec(d, 64, O.MODE_LOG4)
+    skd, svd = _dev_signs(_signs(41, d)), _dev_signs(_signs(42, d))
+    kd = torch.from_numpy(_rand_x(B, H_kv, cap, d, seed=43)).cuda()
+    vd = torch.from_numpy(_rand_x(B, H_kv, cap, d, seed=44, outliers=False)).cuda()
+    planes = []
+    for _ in range(2):
+        K, V = kvq.alloc_plane(kc, B, H_kv, cap), kvq.alloc_plane(vc, B, H_kv, cap)
+        kvq.encode(kc, skd, kd, K, 0)
+        kvq.encode(vc, svd, vd, V, 0)
+        planes.append((K, V))
+    q = torch.randn((B, H_q, d), dtype=torch.float16, device="cuda")
+    k_new = torch.randn((B, H_kv, d), dtype=torch.float16, device="cuda")
+    v_new = torch.randn((B, H_kv, d), dtype=torch.float16, device="cuda")
+    ctx = torch.tensor([400, 129], dtype=torch.int32, device="cuda")
+    S, tau = 3, 1 / math.sqrt(d)
+    ws = [kvq.DecodeWorkspace(B, H_q, d, S) for _ in range(2)]
+    outs = [torch.empty((B, H_q, d), dtype=torch.float32, device="cuda") for _ in range(2)]
+    (K0, V0), (K1, V1) = planes
+    Kc0, Vc0, Kc1, Vc1 = K0.c(), V0.c(), K1.c(), V1.c()
+    call = kvq.DecodeStepCall(q, k_new, v_new, kc, vc, skd, svd, Kc1, Vc1, ctx, B, H_q, H_kv,
+                              cap, tau, S, ws[1].buf, ws[1].nbytes, None, outs[1], kvq.OUT_FP32)
+    for _ in range(2):
+        kvq.kvq_decode_step(q, k_new, v_new, kc, vc, skd, svd, Kc0, Vc0, ctx, B, H_q, H_kv, cap,
+                            tau, S, ws[0].buf, ws[0].nbytes, None, outs[0], kvq.OUT_FP32)
+        call()
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0], outs[1])
+        for w in range(3):
+            assert torch.equal(K0.rows(w), K1.rows(w)) and torch.equal(V0.rows(w), V1.rows(w))
+
+
 def test_decode_step_clipped_context_appends_nothing(dev):
     d, B, H_kv, cap = 128, 1, 2, 64
     kc, vc = kvq.codec(d, 128, O.MODE_LIN8), kvq.codec(d, 64, O.MODE_LOG4)
