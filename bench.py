@@ -12,9 +12,10 @@ kvq_decode_step launch per layer.
          (packed K/V codes + fp16 params read, q read, output written, the
          appended token's fp16 read and codes written) / device time,
          summed over ranks (weak scaling: every rank runs its own replica)
-  e2e    the same through the C-ABI calls with the step's per-step inputs
-         (q, new K/V) copied from pinned host memory and the output copied
-         back inside the timed region
+  e2e    the same through kvq_decode_step_host, the C-ABI call with host
+         buffers: per layer and step q and the new K/V come from pinned host
+         memory and the output goes back there (read and written by the
+         kernel itself), all inside the timed region
   encode prefill encode throughput on one layer of the prefill workload
          (tokens/s) and dequant GB/s, reported alongside
 
@@ -22,8 +23,8 @@ Default workload: the Llama-7B-shaped single-layer decode (B 1, 32 query /
 8 KV heads, d 128, 4096 cached tokens, L_K 128, L_V 64).  Its caches are
 rotated over enough copies to exceed twice the L2 size between reuses.
 
---impl reference times the fp64 CPU oracle (the reference arm of this
-build) on the host cores on a bounded sample of the same workload.
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload.
 """
 from __future__ import annotations
 
@@ -340,23 +341,30 @@ def time_graph(state, K, W, dist_ctx):
 
 
 def time_e2e(state, K, dist_ctx):
-    """Eager C-ABI calls with host buffers: per step copy q and the new K/V
-    (one pinned buffer per layer) to the device, run the step, copy the
-    attention output back."""
+    """The step through the C-ABI call with host buffers: per layer and step,
+    kvq_decode_step_host moves q and the new K/V from pinned memory (one
+    buffer per layer) to the GPU and the attention output back, the
+    transfers made by the kernel's own loads and stores."""
     import torch
-    w = state.w
+    kvq, w = state.kvq, state.w
     hin = [L["io"].cpu().pin_memory() for L in state.layers]  # q | new K | new V
     ho = [torch.empty_like(L["out"], device="cpu").pin_memory() for L in state.layers]
     h2d = sum(t.numel() * t.element_size() for t in hin)
     d2h = sum(t.numel() * t.element_size() for t in ho)
     cur = torch.cuda.current_stream()
+    # no device staging buffers: the kernel reads the inputs from, and writes
+    # the output to, the page-locked host buffers (transfers inside the launch)
+    calls = [[kvq.DecodeStepHostCall(hin[li], None, ho[li], None, L["kc"], L["vc"],
+                                     L["skd"], L["svd"], L["cK"][b], L["cV"][b], state.ctx, w.B,
+                                     w.H_q, w.H_kv, w.ctx, state.tau, state.S, state.ws.buf,
+                                     state.ws.nbytes, state.err, kvq.OUT_FP16)
+              for b in range(state.nbuf)] for li, L in enumerate(state.layers)]
+    st = cur.cuda_stream
 
     def one(i):
-        for li, L in enumerate(state.layers):
-            L["io"].copy_(hin[li], non_blocking=True)
-        state.step(i)
-        for li, L in enumerate(state.layers):
-            ho[li].copy_(L["out"], non_blocking=True)
+        b = i % state.nbuf
+        for per_layer in calls:
+            per_layer[b](st)
 
     for i in range(3):
         one(i)

@@ -290,13 +290,23 @@ namespace {
 
 // Argument checks and launch of a decode, with (kvq_decode_step) or without
 // (kvq_decode_attn) the fused append of the new token.
+// Host buffers of kvq_decode_step_host: copied in after the argument checks
+// and before the launch, copied out after it.
+struct HostIO {
+    const void* in_host;
+    int64_t in_bytes;
+    void* out_host;
+    int64_t out_bytes;
+};
+
 int decode_impl(const char* what, const void* q, const void* k_new, const void* v_new,
                 const kvq_codec* kc, const kvq_codec* vc, const int8_t* signs_k,
                 const int8_t* signs_v, const kvq_plane* K, const kvq_plane* V,
                 const int32_t* ctx_len, int32_t B, int32_t H_q, int32_t H_kv, int64_t max_ctx,
                 float softmax_scale, int32_t num_splits, void* workspace, int64_t ws_bytes,
                 int32_t* err_word, void* out, int32_t out_dtype, void* stream,
-                const kvq_paged_plane* PK = nullptr, const kvq_paged_plane* PV = nullptr) {
+                const kvq_paged_plane* PK = nullptr, const kvq_paged_plane* PV = nullptr,
+                const HostIO* hio = nullptr) {
     char wk[64], wv[64];
     snprintf(wk, sizeof(wk), "%s (K)", what);
     snprintf(wv, sizeof(wv), "%s (V)", what);
@@ -366,7 +376,18 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
         a.enc_k = kvq::encode_args(a.kc, signs_k);
         a.enc_v = kvq::encode_args(a.vc, signs_v);
     }
-    return cuda_status(kvq::launch_decode(a, static_cast<cudaStream_t>(stream)), what);
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc2;
+    if (hio && hio->in_bytes > 0) {
+        rc2 = cuda_status(cudaMemcpyAsync(const_cast<void*>(q), hio->in_host, (size_t)hio->in_bytes,
+                                          cudaMemcpyHostToDevice, st), what);
+        if (rc2) return rc2;
+    }
+    rc2 = cuda_status(kvq::launch_decode(a, st), what);
+    if (rc2 || !hio || hio->out_bytes <= 0) return rc2;
+    return cuda_status(
+        cudaMemcpyAsync(hio->out_host, out, (size_t)hio->out_bytes, cudaMemcpyDeviceToHost, st),
+        what);
 }
 
 }  // namespace
@@ -395,6 +416,55 @@ int kvq_decode_step(const void* q, const void* k_new, const void* v_new, const k
     return decode_impl("kvq_decode_step", q, k_new, v_new, kc, vc, signs_k, signs_v, K, V,
                        ctx_len, B, H_q, H_kv, max_ctx, softmax_scale, num_splits, workspace,
                        ws_bytes, err_word, out, out_dtype, stream);
+}
+
+int kvq_decode_step_host(const void* in_host, void* in_dev, void* out_host, void* out_dev,
+                         const kvq_codec* kc, const kvq_codec* vc, const int8_t* signs_k,
+                         const int8_t* signs_v, const kvq_plane* K, const kvq_plane* V,
+                         const int32_t* ctx_len, int32_t B, int32_t H_q, int32_t H_kv,
+                         int64_t max_ctx, float softmax_scale, int32_t num_splits,
+                         void* workspace, int64_t ws_bytes, int32_t* err_word, int32_t out_dtype,
+                         void* stream) {
+    const char* what = "kvq_decode_step_host";
+    if (!in_host || !out_host) return fail(KVQ_EINVAL, "%s: NULL host buffer", what);
+    const bool mapped = !in_dev && !out_dev;
+    if (!mapped && (!in_dev || !out_dev))
+        return fail(KVQ_EINVAL, "%s: give both device buffers or neither", what);
+    if (!kc) return fail(KVQ_EINVAL, "%s (K): codec is NULL", what);
+    if (B < 0 || H_q < 0 || H_kv < 0) return fail(KVQ_EINVAL, "%s: negative size", what);
+    const int64_t d = kc->head_dim;
+    const int64_t nq = (int64_t)B * H_q * d, nkv = (int64_t)B * H_kv * d;
+    if ((nq * 2) % 16 != 0 || (nkv * 2) % 16 != 0)
+        return fail(KVQ_EINVAL, "%s: q and k_new sizes must be multiples of 16 bytes", what);
+    if (mapped) {
+        // the kernel reads the inputs from, and writes the output to, host
+        // memory that the device can address: page-locked memory only
+        void* dev_ptr[2] = {nullptr, nullptr};
+        const void* host[2] = {in_host, out_host};
+        for (int i = 0; i < 2; i++) {
+            cudaPointerAttributes at;
+            if (cudaPointerGetAttributes(&at, host[i]) != cudaSuccess ||
+                at.type != cudaMemoryTypeHost || !at.devicePointer) {
+                (void)cudaGetLastError();
+                return fail(KVQ_EINVAL, "%s: host buffers must be page-locked to pass no device "
+                            "buffers", what);
+            }
+            dev_ptr[i] = at.devicePointer;
+        }
+        if (!aligned16(dev_ptr[0]) || !aligned16(dev_ptr[1]))
+            return fail(KVQ_EINVAL, "%s: host buffers must be 16-byte aligned", what);
+        const uint16_t* dq = static_cast<const uint16_t*>(dev_ptr[0]);
+        return decode_impl(what, dq, dq + nq, dq + nq + nkv, kc, vc, signs_k, signs_v, K, V,
+                           ctx_len, B, H_q, H_kv, max_ctx, softmax_scale, num_splits, workspace,
+                           ws_bytes, err_word, dev_ptr[1], out_dtype, stream);
+    }
+    if (!aligned16(in_dev) || !aligned16(out_dev))
+        return fail(KVQ_EINVAL, "%s: device buffers must be 16-byte aligned", what);
+    const HostIO hio{in_host, (nq + 2 * nkv) * 2, out_host, nq * (out_dtype == 1 ? 4 : 2)};
+    const uint16_t* dq = static_cast<const uint16_t*>(in_dev);
+    return decode_impl(what, dq, dq + nq, dq + nq + nkv, kc, vc, signs_k, signs_v, K, V, ctx_len,
+                       B, H_q, H_kv, max_ctx, softmax_scale, num_splits, workspace, ws_bytes,
+                       err_word, out_dev, out_dtype, stream, nullptr, nullptr, &hio);
 }
 
 int kvq_decode_attn_paged(const void* q, const kvq_codec* kc, const kvq_codec* vc,

@@ -76,6 +76,12 @@ _SIGNATURES = {
                                   C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_float, C.c_int32,
                                   C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int32,
                                   C.c_void_p]),
+    "kvq_decode_step_host": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                       C.POINTER(kvq_codec), C.POINTER(kvq_codec), C.c_void_p,
+                                       C.c_void_p, C.POINTER(kvq_plane), C.POINTER(kvq_plane),
+                                       C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_int64,
+                                       C.c_float, C.c_int32, C.c_void_p, C.c_int64, C.c_void_p,
+                                       C.c_int32, C.c_void_p]),
     "kvq_encode_kv_paged": (C.c_int, [C.POINTER(kvq_codec), C.c_void_p, C.c_void_p,
                                       C.POINTER(kvq_paged_plane), C.POINTER(kvq_codec),
                                       C.c_void_p, C.c_void_p, C.POINTER(kvq_paged_plane),
@@ -202,6 +208,37 @@ def kvq_decode_step(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, sign
                                  _ptr(ctx_len), B, H_q, H_kv, max_ctx, softmax_scale, num_splits,
                                  _ptr(workspace), ws_bytes, _ptr(err_word), _ptr(out), out_dtype,
                                  _stream(stream)))
+
+
+def kvq_decode_step_host(in_host, in_dev, out_host, out_dev, kc: kvq_codec, vc: kvq_codec,
+                         signs_k, signs_v, K: kvq_plane, V: kvq_plane, ctx_len, B: int, H_q: int,
+                         H_kv: int, max_ctx: int, softmax_scale: float, num_splits: int, workspace,
+                         ws_bytes: int, err_word, out_dtype: int, stream=None):
+    _check(lib().kvq_decode_step_host(_ptr(in_host), _ptr(in_dev), _ptr(out_host), _ptr(out_dev),
+                                      C.byref(kc), C.byref(vc), _ptr(signs_k), _ptr(signs_v),
+                                      C.byref(K), C.byref(V), _ptr(ctx_len), B, H_q, H_kv,
+                                      max_ctx, softmax_scale, num_splits, _ptr(workspace),
+                                      ws_bytes, _ptr(err_word), out_dtype, _stream(stream)))
+
+
+class DecodeStepHostCall:
+    """kvq_decode_step_host with its arguments marshalled once (host and
+    device buffers fixed for the life of the object), for a serving loop that
+    feeds each token's inputs from host memory."""
+
+    def __init__(self, in_host, in_dev, out_host, out_dev, kc: kvq_codec, vc: kvq_codec,
+                 signs_k, signs_v, K: kvq_plane, V: kvq_plane, ctx_len, B: int, H_q: int,
+                 H_kv: int, max_ctx: int, softmax_scale: float, num_splits: int, workspace,
+                 ws_bytes: int, err_word, out_dtype: int):
+        self._kc, self._vc, self._K, self._V = kc, vc, K, V  # keep the structs alive
+        self._fn = lib().kvq_decode_step_host
+        self._args = (_ptr(in_host), _ptr(in_dev), _ptr(out_host), _ptr(out_dev), C.byref(kc),
+                      C.byref(vc), _ptr(signs_k), _ptr(signs_v), C.byref(K), C.byref(V),
+                      _ptr(ctx_len), B, H_q, H_kv, max_ctx, C.c_float(softmax_scale),
+                      num_splits, _ptr(workspace), ws_bytes, _ptr(err_word), out_dtype)
+
+    def __call__(self, stream=None):
+        _check(self._fn(*self._args, _stream(stream)))
 
 
 class DecodeStepCall:

@@ -275,6 +275,35 @@ int kvq_decode_step(const void* q, const void* k_new, const void* v_new,
                     int32_t* err_word, void* out, int32_t out_dtype,
                     void* stream);
 
+/* kvq_decode_step for a caller whose step inputs and output live in host
+ * memory: on `stream`, copies in_host to in_dev, runs kvq_decode_step on
+ * in_dev and out_dev, and copies out_dev to out_host.  With in_dev and
+ * out_dev both NULL, the kernel reads the inputs from in_host and writes the
+ * output to out_host directly (the transfers happen inside the launch, with
+ * no separate copies); both must then be page-locked host memory the device
+ * can address (cudaHostAlloc or cudaHostRegister), which is checked, and
+ * 16-byte aligned.
+ *   in_host   host [q | k_new | v_new], fp16: B*H_q*head_dim values of q,
+ *             then B*H_kv*head_dim of k_new and of v_new (the layouts of
+ *             kvq_decode_step), caller-owned; page-locked memory makes the
+ *             copies asynchronous, pageable memory makes them synchronous
+ *   in_dev    device buffer of the same size, 16-byte aligned, caller-owned
+ *   out_host  host buffer for the output (B*H_q*head_dim values of the
+ *             out_dtype of kvq_decode_step), caller-owned
+ *   out_dev   device buffer of the same size, 16-byte aligned
+ * The step's result is in out_host once the stream has passed the call.
+ * Errors as for kvq_decode_step, plus KVQ_EINVAL for a NULL host buffer,
+ * one device buffer without the other, or unmapped host memory without
+ * device buffers, and KVQ_ECUDA when a copy cannot be issued. */
+int kvq_decode_step_host(const void* in_host, void* in_dev, void* out_host, void* out_dev,
+                         const kvq_codec* kc, const kvq_codec* vc,
+                         const int8_t* signs_k, const int8_t* signs_v,
+                         const kvq_plane* K, const kvq_plane* V,
+                         const int32_t* ctx_len, int32_t B, int32_t H_q,
+                         int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                         int32_t num_splits, void* workspace, int64_t ws_bytes,
+                         int32_t* err_word, int32_t out_dtype, void* stream);
+
 /* The paged forms: kvq_encode_kv, kvq_decode_attn and kvq_decode_step with
  * K and V in paged planes (see kvq_paged_plane).  Results are identical to
  * the contiguous forms on the same rows; arguments and errors as there

@@ -191,6 +191,47 @@ def test_decode_step_shares_the_decode_checks():
     assert "kvq_decode_step: K and V head_dim differ" in kvq.kvq_last_error()
 
 
+@pytest.mark.parametrize("bufs,msg", [
+    ((None, FAKE, FAKE, FAKE), "NULL host buffer"),
+    ((FAKE, FAKE, None, FAKE), "NULL host buffer"),
+    ((FAKE, None, FAKE, FAKE), "both device buffers or neither"),
+    ((FAKE, FAKE + 8, FAKE, FAKE), "16-byte aligned"),
+    ((FAKE, FAKE, FAKE, FAKE + 4), "16-byte aligned"),
+])
+def test_decode_step_host_rejects_bad_buffers(bufs, msg):
+    kc, vc = kvq.codec(128, 128, 0), kvq.codec(128, 64, 1)
+    K, V = _plane(), _plane()
+    ws = kvq.kvq_decode_workspace_bytes(1, 8, 128, 2)
+    rc = kvq.lib().kvq_decode_step_host(*bufs, C.byref(kc), C.byref(vc), FAKE, FAKE, C.byref(K),
+                                        C.byref(V), FAKE, 1, 8, 2, 32, 0.1, 2, FAKE, ws, None, 0,
+                                        None)
+    assert rc == kvq.KVQ_EINVAL
+    assert msg in kvq.kvq_last_error()
+
+
+def test_decode_step_host_without_device_buffers_needs_mapped_memory():
+    # FAKE is no page-locked allocation: refused before any launch
+    kc, vc = kvq.codec(128, 128, 0), kvq.codec(128, 64, 1)
+    K, V = _plane(), _plane()
+    ws = kvq.kvq_decode_workspace_bytes(1, 8, 128, 2)
+    rc = kvq.lib().kvq_decode_step_host(FAKE, None, FAKE, None, C.byref(kc), C.byref(vc), FAKE,
+                                        FAKE, C.byref(K), C.byref(V), FAKE, 1, 8, 2, 32, 0.1, 2,
+                                        FAKE, ws, None, 0, None)
+    assert rc == kvq.KVQ_EINVAL
+    assert "page-locked" in kvq.kvq_last_error()
+
+
+def test_decode_step_host_checks_before_copying():
+    # an argument error is reported before any copy or launch (no GPU here)
+    kc, vc = kvq.codec(128, 128, 0), kvq.codec(64, 64, 1)
+    K, V = _plane(), _plane()
+    rc = kvq.lib().kvq_decode_step_host(FAKE, FAKE, FAKE, FAKE, C.byref(kc), C.byref(vc), FAKE,
+                                        FAKE, C.byref(K), C.byref(V), FAKE, 1, 8, 2, 32, 0.1, 2,
+                                        FAKE, 1 << 20, None, 0, None)
+    assert rc == kvq.KVQ_EINVAL
+    assert "kvq_decode_step_host: K and V head_dim differ" in kvq.kvq_last_error()
+
+
 def test_error_state_is_per_thread():
     import threading
     c = kvq.codec(128, 1, 0)

@@ -380,6 +380,57 @@ def test_decode_step_prepared_call_equals_call(dev):
             assert torch.equal(K0.rows(w), K1.rows(w)) and torch.equal(V0.rows(w), V1.rows(w))
 
 
+def test_decode_step_host_equals_device_step(dev):
+    """kvq_decode_step_host (inputs and output in pinned host memory, copies
+    on the stream, or read and written by the kernel itself) equals
+    kvq_decode_step on twin caches, through the prepared-call wrapper too."""
+    d, B, H_kv, G = 128, 2, 2, 4
+    H_q, cap = G * H_kv, 512
+    kc, vc = kvq.codec(d, 128, O.MODE_LIN8), kvq.codec(d, 64, O.MODE_LOG4)
+    skd, svd = _dev_signs(_signs(51, d)), _dev_signs(_signs(52, d))
+    kd = torch.from_numpy(_rand_x(B, H_kv, cap, d, seed=53)).cuda()
+    vd = torch.from_numpy(_rand_x(B, H_kv, cap, d, seed=54, outliers=False)).cuda()
+    planes = []
+    for _ in range(4):
+        K, V = kvq.alloc_plane(kc, B, H_kv, cap), kvq.alloc_plane(vc, B, H_kv, cap)
+        kvq.encode(kc, skd, kd, K, 0)
+        kvq.encode(vc, svd, vd, V, 0)
+        planes.append((K, V, K.c(), V.c()))
+    nq, nk = B * H_q * d, B * H_kv * d
+    hin = torch.randn(nq + 2 * nk, dtype=torch.float16).pin_memory()
+    din = torch.empty(nq + 2 * nk, dtype=torch.float16, device="cuda")
+    q, k_new, v_new = (hin[:nq].cuda().view(B, H_q, d), hin[nq:nq + nk].cuda().view(B, H_kv, d),
+                       hin[nq + nk:].cuda().view(B, H_kv, d))
+    ctx = torch.tensor([333, 129], dtype=torch.int32, device="cuda")
+    S, tau = 2, 1 / math.sqrt(d)
+    ws = [kvq.DecodeWorkspace(B, H_q, d, S) for _ in range(4)]
+    out_ref = torch.empty((B, H_q, d), dtype=torch.float16, device="cuda")
+    kvq.kvq_decode_step(q, k_new, v_new, kc, vc, skd, svd, planes[0][2], planes[0][3], ctx, B, H_q,
+                        H_kv, cap, tau, S, ws[0].buf, ws[0].nbytes, None, out_ref, kvq.OUT_FP16)
+    hout = [torch.empty((B, H_q, d), dtype=torch.float16).pin_memory() for _ in range(2)]
+    dout = [torch.empty((B, H_q, d), dtype=torch.float16, device="cuda") for _ in range(2)]
+    kvq.kvq_decode_step_host(hin, din, hout[0], dout[0], kc, vc, skd, svd, planes[1][2],
+                             planes[1][3], ctx, B, H_q, H_kv, cap, tau, S, ws[1].buf, ws[1].nbytes,
+                             None, kvq.OUT_FP16)
+    call = kvq.DecodeStepHostCall(hin, din, hout[1], dout[1], kc, vc, skd, svd, planes[2][2],
+                                  planes[2][3], ctx, B, H_q, H_kv, cap, tau, S, ws[2].buf,
+                                  ws[2].nbytes, None, kvq.OUT_FP16)
+    call()
+    # no device buffers: the kernel reads and writes the page-locked host memory
+    hout.append(torch.empty((B, H_q, d), dtype=torch.float16).pin_memory())
+    kvq.kvq_decode_step_host(hin, None, hout[2], None, kc, vc, skd, svd, planes[3][2],
+                             planes[3][3], ctx, B, H_q, H_kv, cap, tau, S, ws[3].buf,
+                             ws[3].nbytes, None, kvq.OUT_FP16)
+    torch.cuda.synchronize()
+    ref = out_ref.cpu()
+    for h in hout:
+        assert torch.equal(h, ref)
+    for w in range(3):
+        for P in planes[1:]:
+            assert torch.equal(P[0].rows(w), planes[0][0].rows(w))
+            assert torch.equal(P[1].rows(w), planes[0][1].rows(w))
+
+
 def test_decode_step_clipped_context_appends_nothing(dev):
     d, B, H_kv, cap = 128, 1, 2, 64
     kc, vc = kvq.codec(d, 128, O.MODE_LIN8), kvq.codec(d, 64, O.MODE_LOG4)
