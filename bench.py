@@ -340,7 +340,7 @@ def time_graph(state, K, W, dist_ctx):
     return ms, statistics.fmean(dec_ms), (t_wall0, t_wall1)
 
 
-def time_e2e(state, K, dist_ctx):
+def time_e2e(state, K, dist_ctx, staged=False):
     """The step through the C-ABI call with host buffers: per layer and step,
     kvq_decode_step_host moves q and the new K/V from pinned memory (one
     buffer per layer) to the GPU and the attention output back, the
@@ -352,9 +352,11 @@ def time_e2e(state, K, dist_ctx):
     h2d = sum(t.numel() * t.element_size() for t in hin)
     d2h = sum(t.numel() * t.element_size() for t in ho)
     cur = torch.cuda.current_stream()
-    # no device staging buffers: the kernel reads the inputs from, and writes
-    # the output to, the page-locked host buffers (transfers inside the launch)
-    calls = [[kvq.DecodeStepHostCall(hin[li], None, ho[li], None, L["kc"], L["vc"],
+    # default: no device staging buffers, the kernel reads the inputs from,
+    # and writes the output to, the page-locked host buffers (transfers inside
+    # the launch); staged: a copy in and a copy out on the stream per call
+    calls = [[kvq.DecodeStepHostCall(hin[li], L["io"] if staged else None, ho[li],
+                                     L["out"] if staged else None, L["kc"], L["vc"],
                                      L["skd"], L["svd"], L["cK"][b], L["cV"][b], state.ctx, w.B,
                                      w.H_q, w.H_kv, w.ctx, state.tau, state.S, state.ws.buf,
                                      state.ws.nbytes, state.err, kvq.OUT_FP16)
@@ -739,6 +741,8 @@ def main():
     ms = max_over_ranks(ctx, ms)
     e2e_ms, e2e_n, h2d, d2h = time_e2e(state, args.steps, ctx)
     e2e_ms = max_over_ranks(ctx, e2e_ms)
+    st_ms, st_n, _, _ = time_e2e(state, args.steps, ctx, staged=True)
+    st_ms = max_over_ranks(ctx, st_ms)
     enc = None if args.no_encode else time_encode(device, hbm_peak)
     big = None if args.no_encode else time_decode_layers(device, hbm_peak, SM_MAX_MHZ)
     t_end = time.time()
@@ -754,6 +758,7 @@ def main():
     world = ctx["world"]
     value = world * total_bytes * args.steps / (ms / 1e3) / 1e9
     e2e = world * total_bytes * e2e_n / (e2e_ms / 1e3) / 1e9
+    e2e_staged = world * total_bytes * st_n / (st_ms / 1e3) / 1e9
     # the step is one kvq_decode_step launch per layer, so the timed region's
     # device time over its launches is the kernel's average launch duration;
     # dec_ms (event nodes around each launch, which add their own dispatch
@@ -801,7 +806,11 @@ def main():
             "peak_kind": f"{peak_kind} copy bandwidth", "traffic": traffic,
         },
         "e2e": {"value": e2e, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_n},
+                "d2h_bytes_per_step": d2h, "steps": e2e_n,
+                "transfer": "kernel loads / stores of page-locked host memory"},
+        "e2e_staged": {"value": e2e_staged, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "steps": st_n,
+                       "transfer": "cudaMemcpyAsync in and out on the stream per call"},
         "gpu_launches": state.kernels_per_step * args.steps,
         "clocks": clocks,
     }
