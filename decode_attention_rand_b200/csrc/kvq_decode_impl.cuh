@@ -307,6 +307,12 @@ __device__ __forceinline__ float2 lds_f2(uint32_t smem_addr) {
 template <int D, int G, int BK, int BV>
 __global__ void __launch_bounds__(DecCfg<D, G>::THREADS, 1)
 decode_kernel(DecodeArgs A) {
+    // A kernel launched after this one as its programmatic dependent (the
+    // next layer's or step's decode) may start its setup once every CTA here
+    // has started: it touches no global memory before griddepcontrol.wait,
+    // which returns only when this grid has completed and its writes are
+    // visible, so it overlaps its barrier setup and tables with this tail.
+    asm volatile("griddepcontrol.launch_dependents;");
     using Cfg = DecCfg<D, G>;
     constexpr int P = Cfg::P, PP = Cfg::PP, NL = Cfg::NL, GPW = Cfg::GPW, NG = Cfg::NG;
     constexpr int WARPS = Cfg::WARPS, TW = Cfg::TW;
