@@ -649,6 +649,9 @@ def cpu_baseline(w, seconds):
 # ------------------------------------------------------------- ranks ----
 
 def init_dist(gpus):
+    """One process per GPU from the torchrun environment: NCCL over the
+    GPUs, or gloo on the host cores where there is no GPU (the CPU tests of
+    the multi-rank path)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -656,10 +659,12 @@ def init_dist(gpus):
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        return dict(world=world, rank=rank, local=local, dist=dist)
-    return dict(world=1, rank=0, local=0, dist=None)
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        return dict(world=world, rank=rank, local=local, dist=dist, backend=backend)
+    return dict(world=1, rank=0, local=0, dist=None, backend=None)
 
 
 def barrier(ctx):
@@ -671,7 +676,8 @@ def max_over_ranks(ctx, value):
     if ctx["dist"] is None:
         return value
     import torch
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64,
+                     device="cuda" if ctx["backend"] == "nccl" else "cpu")
     ctx["dist"].all_reduce(t, op=ctx["dist"].ReduceOp.MAX)
     return float(t.item())
 
@@ -712,8 +718,11 @@ def main():
     w = synth.WORKLOADS[args.workload]
     ctx = init_dist(args.gpus)
     if args.impl == "reference":
+        # rank 0 alone times the oracle; the other ranks leave without work
         if ctx["rank"] == 0:
             run_reference(args, w)
+        if ctx["dist"] is not None:
+            ctx["dist"].destroy_process_group()
         return 0
     import torch
     from decode_attention_rand_b200 import build as kbuild
