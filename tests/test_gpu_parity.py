@@ -187,6 +187,23 @@ def test_encode_edge_cases(dev, d):
             check_encode(x, s, L, mode)
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_encode_every_vector_in_doubt(dev, d):
+    """Every vector has pairs exactly on bin edges (one nonzero channel: its
+    rotated pairs lie on multiples of pi/4, edges when 8 | L), so the
+    streaming pass marks all of them and the fixup pass re-encodes them all:
+    its per-warp queue fills and wraps many times over."""
+    n = 3000
+    s = _signs(d + 5, d)
+    rng = np.random.default_rng(d)
+    x = np.zeros((n, d))
+    x[np.arange(n), rng.integers(0, d, n)] = rng.choice([-1, 1], n) * 2.0 ** rng.integers(-6, 6, n)
+    x = x.astype(np.float16)[None, None]
+    for L, mode in ((128, O.MODE_LIN8), (64, O.MODE_LOG4), (256, O.MODE_LIN8)):
+        stats, *_ = check_encode(x, s, L, mode)
+        assert stats["vectors"] == n
+
+
 def test_encode_distributions_llama_layer(dev):
     """Full Llama-7B-shaped layer (8 KV heads x 4096 tokens, d = 128), K with
     lognormal channel scales and outliers, V ~ N(0,1): every code checked."""
