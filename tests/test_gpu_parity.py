@@ -220,7 +220,7 @@ def test_encode_distributions_llama_layer(dev):
 # ----------------------------------------------------------------- dequant --
 
 @pytest.mark.parametrize("d", [4, 16, 64, 128, 256])
-@pytest.mark.parametrize("L", [3, 64, 128, 256, 5000, 65536])
+@pytest.mark.parametrize("L", [2, 3, 5, 16, 24, 64, 128, 256, 5000, 65536])
 def test_dequant_sweep(dev, d, L):
     s = _signs(d + L, d)
     x = _rand_x(2, 2, 21, d, seed=5 * d + L)
