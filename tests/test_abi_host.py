@@ -29,6 +29,22 @@ def test_exports_every_declared_function():
     assert kvq.kvq_version() >= 10000
 
 
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature of the binding has as many parameters as the
+    declaration in include/kvq.h (a missing or extra argument would shift
+    every later one)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", open(kvq.HEADER).read(), flags=re.S)
+    decls = {}
+    for m in re.finditer(r"\b(kvq_\w+)\s*\(([^;{]*?)\)\s*;", text):
+        params = m.group(2).strip()
+        decls[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    assert set(kvq._SIGNATURES) == set(decls)  # every entry point has its ctypes signature
+    for name, (_, argtypes) in kvq._SIGNATURES.items():
+        assert len(argtypes) == decls[name], name
+    assert set(decls) == set(kvq.header_functions())
+
+
 def test_angle_bits_and_row_bytes_match_layout():
     for L in [2, 3, 4, 5, 7, 8, 100, 128, 129, 255, 256, 4096, 65535, 65536]:
         assert kvq.kvq_angle_bits(L) == O.angle_bits(L)
