@@ -4,8 +4,10 @@ Argument marshalling only: every step of encode, dequant and decode attention
 runs in the CUDA kernels of libkvq.so.  PyTorch provides device memory and
 streams.  The functions named ``kvq_*`` mirror the C entry points one to one
 (they take the same arguments, as ctypes values or torch tensors, and raise
-KvqError on a non-OK status); the small helpers below them only allocate
-caller-owned buffers with torch and fill the C structs.
+KvqError on a non-OK status); DecodeStepCall and DecodeStepHostCall are
+kvq_decode_step / kvq_decode_step_host with their arguments marshalled once
+for per-token reuse; the small helpers below them only allocate caller-owned
+buffers with torch and fill the C structs.
 
 A missing or unloadable libkvq.so raises at first use: there is no fallback.
 """
