@@ -41,6 +41,37 @@ MUTANTS = {
                                 "sc += rh[i] * (qr[2 * i] * sin(th) + qr[2 * i + 1] * cos(th));"),
     "log4_floor_missing": ("l[i] = log2(fmax(r[i], ldexp(1.0, -24)));", "l[i] = log2(r[i]);"),
     "rotate_scale_sqrt2": ("z[j] = zt[j] / sqrt((double)d);", "z[j] = zt[j] / sqrt((double)(2 * d));"),
+    # the edge flags decide which GPU/oracle code differences the parity rule excuses
+    "lin8_norm_flag_never": (
+        "if (fabs((vq - floor(vq)) - 0.5) < EDGE_TOL * fmax(vq, 1.0)) fl[i] |= FLAG_NORM;",
+        "if (0) fl[i] |= FLAG_NORM;"),
+    "lin8_norm_flag_always": (
+        "if (fabs((vq - floor(vq)) - 0.5) < EDGE_TOL * fmax(vq, 1.0)) fl[i] |= FLAG_NORM;",
+        "fl[i] |= FLAG_NORM;"),
+    "lin8_norm_tol_x1e3": ("< EDGE_TOL * fmax(vq, 1.0))", "< 1e3 * EDGE_TOL * fmax(vq, 1.0))"),
+    "log4_norm_flag_never": (
+        "if (fabs((vq - floor(vq)) - 0.5) < EDGE_TOL * fmax(fabs(vq), 1.0)) fl[i] |= FLAG_NORM;",
+        "if (0) fl[i] |= FLAG_NORM;"),
+    "log4_norm_flag_always": (
+        "if (fabs((vq - floor(vq)) - 0.5) < EDGE_TOL * fmax(fabs(vq), 1.0)) fl[i] |= FLAG_NORM;",
+        "fl[i] |= FLAG_NORM;"),
+    "log4_norm_tol_x1e3": ("< EDGE_TOL * fmax(fabs(vq), 1.0))",
+                           "< 1e3 * EDGE_TOL * fmax(fabs(vq), 1.0))"),
+    "param_flag_never": ("int pflag = near_half_midpoint(mx, EDGE_TOL);", "int pflag = 0;"),
+    "param_flag_always": ("norm_row[i] = (uint8_t)c;\n            if (pflag) fl[i] |= FLAG_PARAM;",
+                          "norm_row[i] = (uint8_t)c;\n            fl[i] |= FLAG_PARAM;"),
+    "param_tol_x1e3": ("int pflag = near_half_midpoint(mx, EDGE_TOL);",
+                       "int pflag = near_half_midpoint(mx, 1e3 * EDGE_TOL);"),
+    "midpoint_wrong_upper_neighbour": ("double up = half_to_double((uint16_t)(h + 1));",
+                                       "double up = half_to_double((uint16_t)(h + 2));"),
+    "midpoint_wrong_lower_neighbour": ("double dn = half_to_double((uint16_t)(h - 1));",
+                                       "double dn = half_to_double((uint16_t)(h - 2));"),
+    "log4_param_hi_ignored": (
+        "near_half_midpoint(lmin, EDGE_TOL) || near_half_midpoint(lmax, EDGE_TOL)",
+        "near_half_midpoint(lmin, EDGE_TOL)"),
+    "log4_param_lo_ignored": (
+        "near_half_midpoint(lmin, EDGE_TOL) || near_half_midpoint(lmax, EDGE_TOL)",
+        "near_half_midpoint(lmax, EDGE_TOL)"),
 }
 
 

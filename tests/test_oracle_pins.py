@@ -122,6 +122,36 @@ def test_hand_examples(ex):
             assert c.params[0].tolist() == ex["log4"]["param_row"]
 
 
+FLAGS = json.load(open(os.path.join(HERE, "golden", "flag_examples.json")))
+
+
+@pytest.mark.parametrize("ex", FLAGS["examples"], ids=lambda e: e["name"])
+def test_norm_and_parameter_flags(ex):
+    """The oracle's norm-edge and fp16-midpoint flags on vectors built to sit
+    exactly on a rounding edge, just off it (a few 1e-4 .. 1e-2 away, outside
+    the 1e-6 band), or on / within 5e-7 of an fp16 rounding midpoint of the
+    parameter (tests/golden/make_flag_examples.py derives every expectation
+    in exact or 60-digit arithmetic).  Exact edges must be flagged, near
+    misses must not, a midpoint parameter flags every pair of its vector, and
+    codes away from every edge are the definition's."""
+    d = FLAGS["d"]
+    s = np.array(FLAGS["signs"], np.int8)
+    x = np.array(ex["x"], np.float16)
+    assert np.array_equal(x.astype(np.float64), np.array(ex["x"]))  # exact fp16 inputs
+    z = O.rotate(x.astype(np.float64), s)[0]
+    assert np.array_equal(z, np.array(ex["z_pairs"], np.float64).ravel())
+    c = O.encode(x[None], s, ex["L"], ex["mode"])
+    assert c.flags[0].tolist() == ex["flags"]
+    a, cc, _ = O.unpack(c)
+    assert a[0].tolist() == ex["angles"]
+    for got, want in zip(cc[0].tolist(), ex["codes"]):
+        if want is not None:
+            assert got == want
+    p = c.params[0]
+    bits = [int(p[2 * i]) | int(p[2 * i + 1]) << 8 for i in range(len(ex["params"]))]
+    assert bits == ex["params"]
+
+
 def test_packing_layout():
     g = GOLD["packing"]
     d, L = g["d"], g["L"]
@@ -300,9 +330,15 @@ def test_zero_and_tiny_vectors():
     tiny = np.zeros((1, d), np.float16)
     tiny[0, 5] = np.float16(2.0 ** -24)  # smallest subnormal
     c = O.encode(tiny, s, 64, O.MODE_LIN8)
-    assert (c.flags == 0).all() or True
+    # every rotated pair is +-(1, -1) 2^-24 / 4 (a single odd channel maps to the
+    # diagonals -pi/4, 3pi/4, which are bin edges at L = 64: t = 24 or 56, so
+    # every angle is flagged); r = 2^-24 sqrt(2) / 4 = 2.1e-8 is below half the
+    # smallest fp16 subnormal (2.98e-8): M rounds to +0, every norm code is 0,
+    # and 2.1e-8 lies 8.7e-9 from that midpoint, far outside 1e-6 relative
+    assert (c.flags == O.FLAG_ANGLE).all()
+    assert c.params.sum() == 0 and c.norms.sum() == 0
     xh = O.dequant(c, s)
-    assert np.all(np.isfinite(xh))
+    assert np.all(xh == 0)
 
 
 def test_uniform_angles_after_rotation():
