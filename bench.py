@@ -571,12 +571,13 @@ class OracleSteps:
     def __init__(self, w):
         import numpy as np
         import oracle as O
-        from decode_attention_rand_b200 import kvq
         self.w, self.O, self.np = w, O, np
         self.threads = O.default_threads()
         self.units = [(l, b, h) for l in range(w.layers) for b in range(w.B) for h in range(w.H_kv)]
-        self.rows = {l: (row_bytes_total(kvq, w.d, w.L_K[l], w.mode_K),
-                         row_bytes_total(kvq, w.d, w.L_V[l], w.mode_V)) for l in range(w.layers)}
+        # row sizes from the oracle's own layout: this arm loads nothing but oracle/
+        self.rows = {l: (sum(O.row_bytes(w.d, w.L_K[l], w.mode_K, k) for k in range(3)),
+                         sum(O.row_bytes(w.d, w.L_V[l], w.mode_V, k) for k in range(3)))
+                     for l in range(w.layers)}
         self.prepared = {}
         self.slice_len = w.ctx
 

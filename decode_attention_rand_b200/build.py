@@ -4,9 +4,15 @@ Each .cu file is compiled separately (in parallel) with nvcc for
 -gencode arch=compute_100a,code=sm_100a, then linked into a shared library
 next to this file.  No fast-math: the codec's decisions rely on IEEE sqrt and
 division and on the documented accuracy of atan2f/log2f.
+
+A library is reused only when the SHA-256 of every source, the public header,
+this script and the compiler flags equals the digest recorded beside it
+(libkvq.so.sha256) when it was built; anything else, including a library
+copied in from elsewhere without its record, is rebuilt.
 """
 from __future__ import annotations
 
+import hashlib
 import os
 import subprocess
 import sys
@@ -24,16 +30,36 @@ FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
 
-def _deps_mtime() -> float:
-    files = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if not f.endswith(".py")]
-    files.append(os.path.join(ROOT, "include", "kvq.h"))
-    files.append(os.path.abspath(__file__))
-    return max(os.path.getmtime(f) for f in files)
+STAMP = OUT + ".sha256"
+
+
+def source_digest(extra_flags=()) -> str:
+    """SHA-256 over the names and contents of every input of the build and
+    the flags it is compiled with."""
+    files = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if not f.endswith(".py"))
+    files += [os.path.join(ROOT, "include", "kvq.h"), os.path.abspath(__file__)]
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode() + b"\0")
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    h.update(" ".join([*FLAGS, *extra_flags]).encode())
+    return h.hexdigest()
+
+
+def is_current(extra_flags=()) -> bool:
+    """True when libkvq.so exists and was built from exactly these sources."""
+    try:
+        with open(STAMP) as f:
+            return os.path.exists(OUT) and f.read().strip() == source_digest(extra_flags)
+    except OSError:
+        return False
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and os.path.exists(OUT) and os.path.getmtime(OUT) >= _deps_mtime():
+    if not force and is_current(extra_flags):
         return OUT
+    digest = source_digest(extra_flags)
     os.makedirs(BUILD, exist_ok=True)
 
     def compile_one(src):
@@ -57,6 +83,9 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, OUT)
+    with open(STAMP + f".tmp{os.getpid()}", "w") as f:
+        f.write(digest + "\n")
+    os.replace(STAMP + f".tmp{os.getpid()}", STAMP)
     return OUT
 
 
