@@ -6,7 +6,12 @@ for every layer of the workload: append the new token's K and V (encode,
 T = 1, at the last cache slot) and run split-K decode attention over the
 whole compressed context (query rotation, scores from codes, online softmax,
 value accumulation in the rotated domain, combine, inverse rotation), in one
-kvq_decode_step launch per layer.
+kvq_decode_step launch per layer.  The layers of a step are one CUDA graph.
+
+Headline workload: the Mistral-7B-shaped 32-layer decode step (B 8, 32
+query / 8 KV heads, d 128, 32768 cached tokens, layers 0-3 at L 256/256, the
+rest at L_K 128 / L_V 64): 14.03 GB of packed codes per step, far larger than
+L2, so every step streams its cache from HBM.
 
   value  decode-attention effective HBM GB/s = algorithmic bytes of the step
          (packed K/V codes + fp16 params read, q read, output written, the
@@ -15,14 +20,17 @@ kvq_decode_step launch per layer.
   e2e    the same through kvq_decode_step_host, the C-ABI call with host
          buffers: per layer and step q and the new K/V are copied from pinned
          host memory and the output copied back, on the stream, inside the
-         timed region (e2e_zero_copy: the same call letting the kernel read
-         and write the pinned host memory itself, without copies)
-  encode prefill encode throughput on one layer of the prefill workload
-         (tokens/s) and dequant GB/s, reported alongside
-
-Default workload: the Llama-7B-shaped single-layer decode (B 1, 32 query /
-8 KV heads, d 128, 4096 cached tokens, L_K 128, L_V 64).  Its caches are
-rotated over enough copies to exceed twice the L2 size between reuses.
+         timed region
+  roofline / roofline_fp32
+         the decode kernel against the measured HBM copy bandwidth, and
+         against the FP32 pipe (2 d (G + 1) FMA-pipe operations per cached
+         token and KV head)
+  decode_tinyllama, decode_llama_layer
+         the TinyLlama-shaped 22-layer step (d 64, G 8, 65536 tokens) and the
+         Llama-7B-shaped single layer (the latency case), measured the same way
+  encode the prefill workload in full: K and V of 32 layers x 16 x 8192
+         tokens x 8 KV heads encoded (tokens/s, GB/s), then dequantized back
+         to fp16
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload.
@@ -43,7 +51,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "llama7b_layer_b1_hq32_hkv8_d128_ctx4096"
+DEFAULT_WORKLOAD = "mistral7b_32layers_b8_hq32_hkv8_d128_ctx32768"
+TINYLLAMA = "tinyllama_22layers_b4_hq32_hkv4_d64_ctx65536"
+LLAMA_LAYER = "llama7b_layer_b1_hq32_hkv8_d128_ctx4096"
+PREFILL = "prefill_32layers_b16_t8192_hkv8_d128"
 METRIC = "decode-attn effective HBM GB/s"
 FALLBACK_HBM_GBS = 6650.0
 SM_COUNT_B200 = 148
@@ -61,22 +72,22 @@ def decode_flops_per_token_head(d, G):
     flops with every pipe operation counted as an FMA (two flops): each pair
     is scaled by its norm once for K and once for V (2 d multiplies), then
     every one of the G query heads takes d FMAs for its score and d FMAs for
-    its value accumulation, 2 d (G + 1) operations in all.  A multiply fills
-    an FMA lane slot, so this is the work that meets the FMA-pipe peak."""
+    its value accumulation, 2 d (G + 1) operations in all."""
     return 2 * 2 * d * (G + 1)
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20000)
-    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="wall time of the bounded oracle sample (cpu_baseline)")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--no-encode", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="headline workload only (no TinyLlama / Llama-layer steps, no prefill)")
     p.add_argument("--case", default=None, choices=["decode_layer", "encode_layer", "dequant_layer"],
                    help="run one kernel case only (for profiler captures): the decode of "
                         "--layer of --workload, or the prefill encode (or dequant) of 8 batch "
@@ -145,38 +156,76 @@ def profile_traffic(kernel_tag):
 
 # ---------------------------------------------------------------- clocks --
 
+REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
 class ClockSampler:
-    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of this process's GPU, sampled
+    every 10 ms through NVML in a thread (nvidia-smi at 100 ms where NVML is
+    not importable)."""
 
     def __init__(self, bus_id: str | None):
         self.bus_id = (bus_id or "").lower()
-        self.samples = []
-        self.proc = None
+        self.samples = []  # (time, sm_mhz, sm_max_mhz, reasons tuple)
+        self.stop_ev = threading.Event()
         self.thread = None
+        self.proc = None
 
     def start(self):
         try:
+            import pynvml as N
+            N.nvmlInit()
+            h = N.nvmlDeviceGetHandleByPciBusId(self.bus_id.upper()) if self.bus_id \
+                else N.nvmlDeviceGetHandleByIndex(0)
+            self.thread = threading.Thread(target=self._nvml, args=(N, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
+        try:
+            fields = ("pci.bus_id,clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                      "clocks_event_reasons.hw_thermal_slowdown,"
+                      "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._smi, daemon=True)
+            self.thread.start()
         except Exception:
             self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
-        self.thread.start()
 
-    def _read(self):
+    def _nvml(self, N, h):
+        bits = {"hw_slowdown": N.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": N.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": N.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": N.nvmlClocksEventReasonSwPowerCap}
+        mx = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+        while not self.stop_ev.is_set():
+            try:
+                sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.time(), float(sm), float(mx),
+                                     tuple(n for n in REASONS if r & bits[n])))
+            except Exception:
+                pass
+            self.stop_ev.wait(0.01)
+
+    def _smi(self):
         for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 7:
                 continue
-            if self.bus_id and not parts[0].lower().endswith(self.bus_id[-12:]):
+            if self.bus_id and not p[0].lower().endswith(self.bus_id[-12:]):
                 continue
-            self.samples.append((time.time(), parts))
+            try:
+                self.samples.append((time.time(), float(p[1]), float(p[2]),
+                                     tuple(n for n, v in zip(REASONS, p[3:7])
+                                           if v.lower() == "active")))
+            except ValueError:
+                pass
 
     def stop(self):
+        self.stop_ev.set()
         if self.proc:
             self.proc.terminate()
             try:
@@ -185,27 +234,20 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self, t0, t1):
-        sel = [p for (t, p) in self.samples if t0 <= t <= t1] or [p for _, p in self.samples]
+        sel = [s for s in self.samples if t0 <= s[0] <= t1]
         if not sel:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(p[1]) for p in sel if num(p[1]) is not None]
-        mx = [num(p[2]) for p in sel if num(p[2]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for p in sel for n, v in zip(names, p[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(sel)}
+        return {"sm_mhz": statistics.median(s[1] for s in sel),
+                "sm_max_mhz": max(s[2] for s in sel),
+                "reasons": sorted({n for s in sel for n in s[3]}), "samples": len(sel)}
 
 
 # ------------------------------------------------------------ GPU state --
 
 class DecodeStep:
-    """Device-resident caches of a workload and the launch sequence of one step."""
+    """Device-resident caches of a workload and the launch sequence of one
+    step (one kvq_decode_step per layer).  Caches smaller than twice the L2
+    size are replicated and rotated so that every step reads from HBM."""
 
     def __init__(self, w, device, l2_bytes):
         import torch
@@ -265,9 +307,10 @@ class DecodeStep:
             self.layers.append(L)
         torch.cuda.synchronize(device)
         self.kernels_per_step = w.layers  # one fused append + decode launch per layer
+        self.bytes_per_step, self.bytes_per_launch = total, per_layer
+        self.cache_bytes = cache_bytes * self.nbuf
 
     def step(self, i, ev=None, stream=None):
-        kvq, w = self.kvq, self.w
         b = i % self.nbuf
         st = stream.cuda_stream if stream is not None else self.torch.cuda.current_stream().cuda_stream
         for li, L in enumerate(self.layers):
@@ -277,20 +320,27 @@ class DecodeStep:
             if ev is not None:
                 ev[li][1].record()
 
+    def release(self):
+        self.layers = []
+        self.ws = None
+        self.torch.cuda.synchronize(self.device)
+        self.torch.cuda.empty_cache()
+
 
 def time_graph(state, K, W, dist_ctx):
-    """Device time of exactly K steps replayed from CUDA graphs, plus the
-    average decode-launch duration from events captured in a separate graph.
+    """Device time of exactly K steps replayed from CUDA graphs, plus
+    per-launch durations from events captured in a separate graph.
 
-    The timed graphs hold the steps' kernels only: an event node between the
-    append and the decode would cut the programmatic dependency that lets the
-    decode's setup overlap the append."""
+    The timed graphs hold the steps' kernels only: an event node between two
+    launches would cut the programmatic dependency that lets each decode's
+    setup overlap the previous launch."""
     import torch
     stream = torch.cuda.Stream()
     for i in range(W):
         state.step(i)
     torch.cuda.synchronize()
-    unit = max(1, min(K, state.nbuf * max(1, math.ceil(64 / state.nbuf))))
+    per_graph = max(1, math.ceil(256 / max(1, state.kernels_per_step)))
+    unit = max(1, min(K, state.nbuf * max(1, math.ceil(per_graph / state.nbuf))))
     n_full, rem = divmod(K, unit)
     g_unit = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_unit, stream=stream):
@@ -304,7 +354,7 @@ def time_graph(state, K, W, dist_ctx):
                 state.step(n_full * unit + i, stream=torch.cuda.current_stream())
     # external events become event-record nodes of the graph, so each decode
     # launch is timed inside the replay
-    n_ev = min(unit, 16)
+    n_ev = max(1, min(unit, 4 if state.kernels_per_step > 1 else 16))
     evs = [[[torch.cuda.Event(enable_timing=True, external=True),
              torch.cuda.Event(enable_timing=True, external=True)]
             for _ in state.layers] for _ in range(n_ev)]
@@ -332,21 +382,22 @@ def time_graph(state, K, W, dist_ctx):
     t_wall1 = time.time()
     barrier(dist_ctx)
     ms = start.elapsed_time(end)
-    dec_ms = []
-    for _ in range(4):
+    per_layer = [[] for _ in state.layers]
+    for _ in range(2):
         g_ev.replay()
         torch.cuda.synchronize()
-        dec_ms += [evs[i][li][0].elapsed_time(evs[i][li][1]) for i in range(n_ev)
-                   for li in range(len(state.layers))]
-    return ms, statistics.fmean(dec_ms), (t_wall0, t_wall1)
+        for i in range(n_ev):
+            for li in range(len(state.layers)):
+                per_layer[li].append(evs[i][li][0].elapsed_time(evs[i][li][1]))
+    del g_unit, g_rem, g_ev
+    return ms, [statistics.fmean(x) for x in per_layer], (t_wall0, t_wall1)
 
 
-def time_e2e(state, K, dist_ctx, staged=False):
+def time_e2e(state, K, dist_ctx):
     """The step through the C-ABI call with host buffers: per layer and step,
-    kvq_decode_step_host moves q and the new K/V from pinned memory (one
-    buffer per layer) to the GPU and the attention output back: staged, by a
-    copy in and a copy out on the stream; otherwise by the kernel's own
-    loads and stores of the page-locked host memory."""
+    kvq_decode_step_host copies q and the new K/V from pinned host memory (one
+    buffer per layer) to the GPU and the attention output back, on the
+    stream, inside the timed region."""
     import torch
     kvq, w = state.kvq, state.w
     hin = [L["io"].cpu().pin_memory() for L in state.layers]  # q | new K | new V
@@ -354,11 +405,7 @@ def time_e2e(state, K, dist_ctx, staged=False):
     h2d = sum(t.numel() * t.element_size() for t in hin)
     d2h = sum(t.numel() * t.element_size() for t in ho)
     cur = torch.cuda.current_stream()
-    # staged: device staging buffers, a copy in and a copy out on the stream
-    # per call; otherwise the kernel reads the inputs from, and writes the
-    # output to, the page-locked host buffers (transfers inside the launch)
-    calls = [[kvq.DecodeStepHostCall(hin[li], L["io"] if staged else None, ho[li],
-                                     L["out"] if staged else None, L["kc"], L["vc"],
+    calls = [[kvq.DecodeStepHostCall(hin[li], L["io"], ho[li], L["out"], L["kc"], L["vc"],
                                      L["skd"], L["svd"], L["cK"][b], L["cV"][b], state.ctx, w.B,
                                      w.H_q, w.H_kv, w.ctx, state.tau, state.S, state.ws.buf,
                                      state.ws.nbytes, state.err, kvq.OUT_FP16)
@@ -373,7 +420,7 @@ def time_e2e(state, K, dist_ctx, staged=False):
     for i in range(3):
         one(i)
     torch.cuda.synchronize()
-    n = max(1, min(K, 2000 // max(1, w.layers)))
+    n = max(1, min(K, 4000 // max(1, w.layers)))
     barrier(dist_ctx)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(cur)
@@ -385,107 +432,109 @@ def time_e2e(state, K, dist_ctx, staged=False):
     return start.elapsed_time(end), n, h2d, d2h
 
 
-def time_encode(device, hbm_peak):
-    """Prefill encode of one layer (K and V) and its dequant, device time."""
+def decode_report(state, ms, K, per_launch_ms, hbm_peak, peak_kind, sm_mhz, sm_count,
+                  traffic=None):
+    """Throughput and roofline figures of a timed decode workload."""
+    w = state.w
+    launches = K * state.kernels_per_step
+    us_launch = ms / launches * 1e3  # one kvq_decode_step launch per layer
+    bytes_launch = statistics.fmean(state.bytes_per_launch)
+    gbs = bytes_launch / (us_launch / 1e6) / 1e9
+    flops = w.B * w.H_kv * w.ctx * decode_flops_per_token_head(w.d, w.G)
+    fp_peak = fp32_peak_tflops(sm_mhz, sm_count)
+    tfs = flops / (us_launch / 1e6) / 1e12
+    early = [i for i in range(w.layers) if (w.L_K[i], w.L_V[i]) != (w.L_K[-1], w.L_V[-1])]
+    late = [i for i in range(w.layers) if i not in early]
+    by_kind = {}
+    for name, idx in (("early_boost_layers", early), ("other_layers", late)):
+        if idx:
+            t = statistics.fmean(per_launch_ms[i] for i in idx)
+            b = statistics.fmean(state.bytes_per_launch[i] for i in idx)
+            by_kind[name] = {"layers": len(idx), "L_K": w.L_K[idx[0]], "L_V": w.L_V[idx[0]],
+                             "us_per_launch_event_bracketed": t * 1e3,
+                             "gb_per_s": b / (t / 1e3) / 1e9,
+                             "hbm_frac": b / (t / 1e3) / 1e9 / hbm_peak}
+    return {
+        "gb_per_s": state.bytes_per_step * K / (ms / 1e3) / 1e9,
+        "ms_per_step": ms / K,
+        "per_token_latency_ms": ms / K,
+        "bytes_per_step": state.bytes_per_step,
+        "num_splits": state.S,
+        "roofline": {
+            "kernel": "decode_kernel (kvq_decode_step: append of the new token, split-K "
+                      "decode attention and the split combine, one launch per layer)",
+            "bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+            "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
+            "traffic": traffic, "bytes_per_launch": bytes_launch, "us_per_launch": us_launch,
+        },
+        "roofline_fp32": {
+            "achieved": tfs, "peak": fp_peak, "unit": "TFLOP/s", "frac": tfs / fp_peak,
+            "flops_per_launch": flops,
+            "peak_kind": f"FP32 FMA pipe, derived: {FP32_LANES_PER_SM} lanes/SM x {sm_count} "
+                         f"SMs x 2 flop x {sm_mhz:.0f} MHz (sampled)",
+        },
+        "launch_kinds": by_kind,
+    }
+
+
+def time_prefill(device, hbm_peak, reps=3):
+    """The prefill workload in full: kvq_encode of K and V of all 32 layers
+    (16 x 8192 tokens x 8 KV heads each), then kvq_dequant of all of them;
+    CUDA events around whole passes."""
     import torch
     from decode_attention_rand_b200 import kvq, synth
-    w = synth.WORKLOADS["prefill_32layers_b16_t8192_hkv8_d128"]
-    sk, sv = synth.layer_signs(w, 0)
+    w = synth.WORKLOADS[PREFILL]
     items = []
-    for kind, L, mode, s in ((synth.KIND_K, 128, 0, sk), (synth.KIND_V, 64, 1, sv)):
-        c = kvq.codec(w.d, L, mode)
-        p = kvq.alloc_plane(c, w.B, w.H_kv, w.ctx, device)
-        x = synth.kv(w, 0, kind, device=device)
-        y = torch.empty_like(x)
-        items.append((c, p, x, y, torch.from_numpy(s).to(device)))
-    n_vec = 2 * w.B * w.H_kv * w.ctx
-    enc_bytes = sum(x.numel() * 2 + w.B * w.H_kv * w.ctx * row_bytes_total(kvq, w.d, c.L, c.norm_mode)
-                    for c, p, x, y, s in items)
-    reps = 20
-    for c, p, x, y, s in items:
+    for layer in range(w.layers):
+        sk, sv = synth.layer_signs(w, layer)
+        for kind, L, mode, s in ((synth.KIND_K, w.L_K[layer], w.mode_K, sk),
+                                 (synth.KIND_V, w.L_V[layer], w.mode_V, sv)):
+            c = kvq.codec(w.d, L, mode)
+            p = kvq.alloc_plane(c, w.B, w.H_kv, w.ctx, device)
+            x = synth.kv(w, layer, kind, device=device)
+            items.append((c, p, x, torch.from_numpy(s).to(device)))
+    # one fp16 destination per tensor kind, reused by every layer's dequant
+    ys = [torch.empty_like(items[0][2]), torch.empty_like(items[1][2])]
+    n_vec = len(items) * w.B * w.H_kv * w.ctx
+    rows = sum(w.B * w.H_kv * w.ctx * row_bytes_total(kvq, w.d, c.L, c.norm_mode)
+               for c, p, x, s in items)
+    fp16 = sum(x.numel() * 2 for c, p, x, s in items)
+    for c, p, x, s in items:  # warm-up pass
         kvq.encode(c, s, x, p, 0)
-        kvq.dequant(c, s, p, w.ctx, out=y)
+    for i, (c, p, x, s) in enumerate(items):
+        kvq.dequant(c, s, p, w.ctx, out=ys[i % 2])
     torch.cuda.synchronize()
     e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
     e0.record()
     for _ in range(reps):
-        for c, p, x, y, s in items:
+        for c, p, x, s in items:
             kvq.encode(c, s, x, p, 0)
     e1.record()
     for _ in range(reps):
-        for c, p, x, y, s in items:
-            kvq.dequant(c, s, p, w.ctx, out=y)
+        for i, (c, p, x, s) in enumerate(items):
+            kvq.dequant(c, s, p, w.ctx, out=ys[i % 2])
     e2.record()
     torch.cuda.synchronize()
     enc_s = e0.elapsed_time(e1) / 1e3 / reps
     dq_s = e1.elapsed_time(e2) / 1e3 / reps
-    tokens = w.B * w.ctx
-    return {
-        "workload": f"{w.name} (one layer: K and V, {n_vec} head vectors)",
+    tokens = w.layers * w.B * w.ctx
+    out = {
+        "workload": f"{w.name}: K and V of {w.layers} layers, {n_vec} head vectors per pass",
         "tokens_per_s": tokens / enc_s,
         "head_vectors_per_s": n_vec / enc_s,
-        "encode_gb_per_s": enc_bytes / enc_s / 1e9,
-        "encode_frac": enc_bytes / enc_s / 1e9 / hbm_peak,
-        "dequant_gb_per_s": enc_bytes / dq_s / 1e9,
-        "dequant_frac": enc_bytes / dq_s / 1e9 / hbm_peak,
-        "ms_per_layer_encode": enc_s * 1e3,
-        "ms_per_layer_dequant": dq_s * 1e3,
+        "encode_gb_per_s": (fp16 + rows) / enc_s / 1e9,
+        "encode_frac": (fp16 + rows) / enc_s / 1e9 / hbm_peak,
+        "dequant_gb_per_s": (fp16 + rows) / dq_s / 1e9,
+        "dequant_frac": (fp16 + rows) / dq_s / 1e9 / hbm_peak,
+        "ms_per_pass_encode": enc_s * 1e3,
+        "ms_per_pass_dequant": dq_s * 1e3,
+        "bytes_per_pass": fp16 + rows,
+        "launches_per_pass": len(items),
     }
-
-
-def time_decode_layers(device, hbm_peak, sm_mhz):
-    """Decode-kernel time on single layers of the large decode workloads
-    (eager launches, CUDA events; each layer's codes exceed L2)."""
-    import torch
-    from decode_attention_rand_b200 import kvq, synth
-    sm = torch.cuda.get_device_properties(device).multi_processor_count
-    fp_peak = fp32_peak_tflops(sm_mhz, sm)
-    res = []
-    for name, layer in (("mistral7b_32layers_b8_hq32_hkv8_d128_ctx32768", 4),
-                        ("mistral7b_32layers_b8_hq32_hkv8_d128_ctx32768", 0),
-                        ("tinyllama_22layers_b4_hq32_hkv4_d64_ctx65536", 2)):
-        w = synth.WORKLOADS[name]
-        sk, sv = synth.layer_signs(w, layer)
-        skd, svd = torch.from_numpy(sk).to(device), torch.from_numpy(sv).to(device)
-        kc = kvq.codec(w.d, w.L_K[layer], w.mode_K)
-        vc = kvq.codec(w.d, w.L_V[layer], w.mode_V)
-        planes = []
-        for kind, c, sg in ((synth.KIND_K, kc, skd), (synth.KIND_V, vc, svd)):
-            p = kvq.alloc_plane(c, w.B, w.H_kv, w.ctx, device)
-            x = synth.kv(w, layer, kind, device=device)
-            kvq.encode(c, sg, x, p, 0)
-            del x
-            planes.append(p)
-        q = synth.queries(w, layer, device=device)
-        ctx = torch.full((w.B,), w.ctx, dtype=torch.int32, device=device)
-        out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float16, device=device)
-        S = kvq.kvq_decode_num_splits(w.B, w.H_kv, w.ctx, sm)
-        ws = kvq.DecodeWorkspace(w.B, w.H_q, w.d, S, device)
-
-        def run():
-            kvq.decode_attn(q, kc, vc, skd, svd, planes[0], planes[1], ctx, w.ctx, None,
-                            num_splits=S, workspace=ws, out=out, out_dtype=kvq.OUT_FP16)
-        for _ in range(3):
-            run()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n = 20
-        e0.record()
-        for _ in range(n):
-            run()
-        e1.record()
-        torch.cuda.synchronize()
-        t = e0.elapsed_time(e1) / 1e3 / n
-        nb = (w.B * w.H_kv * w.ctx * (row_bytes_total(kvq, w.d, kc.L, kc.norm_mode) +
-                                      row_bytes_total(kvq, w.d, vc.L, vc.norm_mode)) +
-              w.B * w.H_q * w.d * 4)
-        fl = w.B * w.H_kv * w.ctx * decode_flops_per_token_head(w.d, w.G)
-        res.append({"workload": f"{name} layer {layer} (L_K {kc.L}, L_V {vc.L}, {S} splits)",
-                    "us": t * 1e6, "gb_per_s": nb / t / 1e9, "hbm_frac": nb / t / 1e9 / hbm_peak,
-                    "tflop_per_s": fl / t / 1e12, "fp32_frac": fl / t / 1e12 / fp_peak})
-        del planes, q, ws
-        torch.cuda.empty_cache()
-    return res
+    del items, ys
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_case(args):
@@ -523,7 +572,7 @@ def run_case(args):
                             num_splits=S, workspace=ws, out=out, out_dtype=kvq.OUT_FP16)
         what = f"decode {w.name} layer {layer}, {S} splits"
     else:
-        w = synth.WORKLOADS["prefill_32layers_b16_t8192_hkv8_d128"]
+        w = synth.WORKLOADS[PREFILL]
         sk, sv = synth.layer_signs(w, 0)
         isk = args.tensor == "k"
         c = (kvq.codec(w.d, w.L_K[0], w.mode_K) if isk else kvq.codec(w.d, w.L_V[0], w.mode_V))
@@ -609,9 +658,12 @@ class OracleSteps:
         return nbytes, dt
 
     def calibrate(self, per_step_s):
-        """Pick the context slice so that one step takes about per_step_s."""
-        data = self._prepare(self.units[0], self.w.ctx)
-        _, t_full = self._one(self.units[0], data)
+        """Pick the context slice so that one step takes about per_step_s
+        (timed first on a 2048-token slice, then scaled)."""
+        probe = min(self.w.ctx, 2048)
+        data = self._prepare(self.units[0], probe)
+        _, t_probe = self._one(self.units[0], data)
+        t_full = t_probe * self.w.ctx / probe
         if per_step_s is not None and t_full > per_step_s:
             sl = int(self.w.ctx * per_step_s / t_full) // 16 * 16
             self.slice_len = max(16, min(self.w.ctx, sl))
@@ -642,8 +694,10 @@ class OracleSteps:
 
 def cpu_baseline(w, seconds):
     ors = OracleSteps(w)
-    t_full = ors.calibrate(None)
-    n = max(1, int(seconds / max(t_full, 1e-6)))
+    ors.calibrate(seconds / 4)
+    t0 = time.perf_counter()
+    done, secs = ors.run(1)
+    n = max(1, int(seconds / max(time.perf_counter() - t0, 1e-6)))
     done, secs = ors.run(n)
     return {"value": done / secs / 1e9, "unit": "GB/s", "cores": ors.threads, "kind": "oracle",
             "sample": ors.describe(n)}
@@ -697,7 +751,7 @@ def run_reference(args, w):
     a bounded sample each, the whole run kept to a few minutes."""
     ors = OracleSteps(w)
     budget = max(5.0, min(150.0, 2.0 * (args.steps + args.warmup)))  # seconds, whole run
-    ors.calibrate(budget / (args.steps + args.warmup))
+    ors.calibrate(budget / max(1, args.steps + args.warmup))
     ors.run(args.warmup)
     done, secs = ors.run(args.steps)
     gbs = done / secs / 1e9
@@ -711,6 +765,36 @@ def run_reference(args, w):
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def measure(name, device, l2, K, W, ctx, hbm_peak, peak_kind, sm_count, sampler, e2e=False,
+            traffic=None):
+    """Build one decode workload, time K graphed steps (and the e2e path),
+    and return its report plus the timed window and the state's launch count."""
+    from decode_attention_rand_b200 import synth
+    w = synth.WORKLOADS[name]
+    state = DecodeStep(w, device, l2)
+    ms, per_launch, (tw0, tw1) = time_graph(state, K, W, ctx)
+    ms = max_over_ranks(ctx, ms)
+    clocks = sampler.summary(tw0, tw1)
+    rep = decode_report(state, ms, K, per_launch, hbm_peak, peak_kind,
+                        clocks.get("sm_mhz") or SM_MAX_MHZ, sm_count, traffic)
+    rep["workload"] = w.name
+    rep["clocks"] = clocks
+    rep["l2"] = (f"inputs larger than L2: {state.cache_bytes / 1e9:.2f} GB of codes read per "
+                 f"cycle of {state.nbuf} step(s) (L2 {l2 / 2**20:.0f} MiB)")
+    if e2e:
+        e_ms, e_n, h2d, d2h = time_e2e(state, K, ctx)
+        e_ms = max_over_ranks(ctx, e_ms)
+        rep["e2e"] = {"value": ctx["world"] * state.bytes_per_step * e_n / (e_ms / 1e3) / 1e9,
+                      "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "steps": e_n, "transfer": "cudaMemcpyAsync in and out on the stream per call"}
+    err = int(state.err.item())
+    launches = state.kernels_per_step * K
+    state.release()
+    if err != 0:
+        raise RuntimeError(f"{name}: device error word {err}")
+    return rep, launches
 
 
 def main():
@@ -746,98 +830,69 @@ def main():
     hbm_peak, peak_kind = peaks()
     sampler = ClockSampler(bus)
     sampler.start()
+    sm_count = props.multi_processor_count
+    K, W = args.steps, max(args.warmup, 0)
 
-    state = DecodeStep(w, device, l2)
-    total_bytes, per_layer = step_bytes(kvq, w)
-    ms, dec_ms, (tw0, tw1) = time_graph(state, args.steps, args.warmup, ctx)
-    ms = max_over_ranks(ctx, ms)
-    e2e_ms, e2e_n, h2d, d2h = time_e2e(state, args.steps, ctx, staged=True)
-    e2e_ms = max_over_ranks(ctx, e2e_ms)
-    zc_ms, zc_n, _, _ = time_e2e(state, args.steps, ctx)
-    zc_ms = max_over_ranks(ctx, zc_ms)
-    enc = None if args.no_encode else time_encode(device, hbm_peak)
-    big = None if args.no_encode else time_decode_layers(device, hbm_peak, SM_MAX_MHZ)
-    t_end = time.time()
+    head, launches = measure(w.name, device, l2, K, W, ctx, hbm_peak, peak_kind, sm_count,
+                             sampler, e2e=True, traffic=headline_traffic(w.name))
+    extra = {}
+    if not args.no_extra:
+        for key, name in (("decode_tinyllama", TINYLLAMA), ("decode_llama_layer", LLAMA_LAYER)):
+            if name != w.name:
+                extra[key], _ = measure(name, device, l2, K, W, ctx, hbm_peak, peak_kind,
+                                        sm_count, sampler)
+        extra["encode"] = time_prefill(device, hbm_peak)
     sampler.stop()
-    if int(state.err.item()) != 0:
-        raise RuntimeError(f"device error word {int(state.err.item())}")
 
     if ctx["rank"] != 0:
         if ctx["dist"] is not None:
             ctx["dist"].destroy_process_group()
         return 0
-    clocks = sampler.summary(tw0, tw1)
     world = ctx["world"]
-    value = world * total_bytes * args.steps / (ms / 1e3) / 1e9
-    e2e = world * total_bytes * e2e_n / (e2e_ms / 1e3) / 1e9
-    e2e_zc = world * total_bytes * zc_n / (zc_ms / 1e3) / 1e9
-    # the step is one kvq_decode_step launch per layer, so the timed region's
-    # device time over its launches is the kernel's average launch duration;
-    # dec_ms (event nodes around each launch, which add their own dispatch
-    # gaps) is reported beside it
-    dec_ms_isolated = dec_ms
-    dec_ms = ms / (args.steps * w.layers)
-    dec_bytes = statistics.fmean(per_layer)
-    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
-    dec_flops = w.B * w.H_kv * w.ctx * decode_flops_per_token_head(w.d, w.G)
-    sm_mhz = clocks.get("sm_mhz") or SM_MAX_MHZ
-    fp_peak = fp32_peak_tflops(sm_mhz, props.multi_processor_count)
-    fp_achieved = dec_flops / (dec_ms / 1e3) / 1e12
-    traffic = profile_traffic("decode_kernel_llama7b_layer")
-    # the binding roofline of the decode kernel: FP32 FMA pipe when the time
-    # its flops need at peak exceeds the time its bytes need at HBM peak
-    fp_bound = dec_flops / (fp_peak * 1e12) > dec_bytes / (hbm_peak * 1e9)
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": world * head["gb_per_s"], "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {
-            **workload_config(w), "num_splits": state.S, "out": "fp16",
-            "l2": f"inputs larger than L2: {state.nbuf} rotated cache copies "
-                  f"({state.nbuf * sum(per_layer) / 2**20:.0f} MiB per cycle, L2 {l2 / 2**20:.0f} MiB)",
-            "timing": "CUDA graph replay, CUDA events, max over ranks",
-            "bytes_per_step": total_bytes,
+            **workload_config(w), "num_splits": head["num_splits"], "out": "fp16",
+            "l2": head["l2"],
+            "timing": "CUDA graph replay of whole steps, CUDA events, max over ranks",
+            "bytes_per_step": head["bytes_per_step"],
         },
-        "roofline": ({
-            "kernel": "decode_kernel (one kvq_decode_step launch: append, splits and their combine)",
-            "bound": "alu", "achieved": fp_achieved, "peak": fp_peak, "unit": "TFLOP/s",
-            "frac": fp_achieved / fp_peak,
-            "peak_kind": f"FP32 FMA pipe, derived: {FP32_LANES_PER_SM} lanes/SM x "
-                         f"{props.multi_processor_count} SMs x 2 flop x {sm_mhz:.0f} MHz",
-            "traffic": traffic, "flops_per_launch": dec_flops, "bytes_per_launch": dec_bytes,
-            "us_per_launch": dec_ms * 1e3, "us_per_launch_event_bracketed": dec_ms_isolated * 1e3,
-        } if fp_bound else {
-            "kernel": "decode_kernel (one kvq_decode_step launch: append, splits and their combine)",
-            "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-            "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
-            "traffic": traffic, "bytes_per_launch": dec_bytes, "us_per_launch": dec_ms * 1e3,
-            "us_per_launch_event_bracketed": dec_ms_isolated * 1e3,
-        }),
-        "roofline_hbm": {
-            "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-            "peak_kind": f"{peak_kind} copy bandwidth", "traffic": traffic,
-        },
-        "e2e": {"value": e2e, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_n,
-                "transfer": "cudaMemcpyAsync in and out on the stream per call"},
-        "e2e_zero_copy": {"value": e2e_zc, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                          "d2h_bytes_per_step": d2h, "steps": zc_n,
-                          "transfer": "kernel loads / stores of page-locked host memory"},
-        "gpu_launches": state.kernels_per_step * args.steps,
-        "clocks": clocks,
+        "roofline": head["roofline"],
+        "roofline_fp32": head["roofline_fp32"],
+        "launch_kinds": head["launch_kinds"],
+        "per_token_latency_ms": {w.name: head["per_token_latency_ms"]},
+        "e2e": head["e2e"],
+        "gpu_launches": launches,
+        "clocks": head["clocks"],
     }
-    if enc:
-        line["encode"] = enc
-    if big:
-        for r in big:
-            r["fp32_frac"] = r["tflop_per_s"] / fp_peak
-        line["decode_large_layers"] = big
+    for key, rep in extra.items():
+        line[key] = rep
+        if "per_token_latency_ms" in rep:
+            line["per_token_latency_ms"][rep["workload"]] = rep["per_token_latency_ms"]
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
     if ctx["dist"] is not None:
         ctx["dist"].destroy_process_group()
     return 0
+
+
+def headline_traffic(name):
+    """DRAM bytes per decode launch of a workload, from the committed ncu
+    summaries of its layer kinds (weighted by how many layers each kind has),
+    or None when a summary is missing or stale."""
+    from decode_attention_rand_b200 import synth
+    w = synth.WORKLOADS[name]
+    if name == DEFAULT_WORKLOAD:
+        t0 = profile_traffic("decode_kernel_mistral7b_layer0")
+        t4 = profile_traffic("decode_kernel_mistral7b_layer4")
+        if t0 is None or t4 is None:
+            return None
+        n_early = sum(1 for i in range(w.layers) if w.L_K[i] == w.L_K[0])
+        return (n_early * t0 + (w.layers - n_early) * t4) / w.layers
+    return None
 
 
 if __name__ == "__main__":

@@ -4,11 +4,18 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "kvq_internal.h"
 
 namespace {
 
 thread_local char g_err[512] = "";
+
+// kvq_test_control state: launches still to be failed, and the tile-wait
+// limit of decode kernels plus one (0: the default limit).
+std::atomic<int64_t> g_fail_launches{0};
+std::atomic<int64_t> g_wait_limit_p1{0};
 
 int fail(int code, const char* fmt, ...) {
     va_list ap;
@@ -106,6 +113,20 @@ int cuda_status(cudaError_t e, const char* what) {
     return ok();
 }
 
+// A launch that kvq_test_control asked to fail: consumes one and reports it
+// the way a failed launch is reported (nothing is queued).
+bool injected_failure() {
+    int64_t n = g_fail_launches.load();
+    while (n > 0)
+        if (g_fail_launches.compare_exchange_weak(n, n - 1)) return true;
+    return false;
+}
+
+int injected(const char* what) {
+    return fail(KVQ_ECUDA, "%s: cudaErrorLaunchFailure (launch failure injected by "
+                "kvq_test_control)", what);
+}
+
 }  // namespace
 
 namespace kvq {
@@ -114,7 +135,22 @@ int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
 extern "C" {
 
-int32_t kvq_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+int32_t kvq_version(void) { return 1 * 10000 + 1 * 100 + 0; }
+
+int kvq_test_control(int32_t key, int64_t value) {
+    if (value < 0) return fail(KVQ_EINVAL, "kvq_test_control: negative value");
+    switch (key) {
+        case KVQ_TEST_RESET:
+            g_fail_launches.store(0);
+            g_wait_limit_p1.store(0);
+            return ok();
+        case KVQ_TEST_FAIL_LAUNCHES: g_fail_launches.store(value); return ok();
+        case KVQ_TEST_WAIT_LIMIT:
+            g_wait_limit_p1.store((value < 0xFFFFFFFFll ? value : 0xFFFFFFFFll - 1) + 1);
+            return ok();
+        default: return fail(KVQ_EINVAL, "kvq_test_control: unknown key %d", key);
+    }
+}
 
 const char* kvq_last_error(void) { return g_err; }
 
@@ -187,6 +223,7 @@ int kvq_encode(const kvq_codec* codec, const int8_t* signs, const void* x, int32
     const int rc = prep_encode(codec, signs, x, B, H_kv, T, pos0, out, "kvq_encode", "x", &j);
     if (rc) return rc;
     if (j.n_vec == 0) return ok();
+    if (injected_failure()) return injected("kvq_encode");
     return cuda_status(kvq::launch_encode_jobs(&j, 1, sm_count_current(),
                                                static_cast<cudaStream_t>(stream)),
                        "kvq_encode");
@@ -204,6 +241,7 @@ int kvq_encode_kv(const kvq_codec* kc, const int8_t* signs_k, const void* k, con
         return fail(KVQ_EINVAL, "kvq_encode_kv: K head_dim %d differs from V head_dim %d",
                     j[0].c.d, j[1].c.d);
     if (j[0].n_vec == 0) return ok();
+    if (injected_failure()) return injected("kvq_encode_kv");
     return cuda_status(kvq::launch_encode_jobs(j, 2, sm_count_current(),
                                                static_cast<cudaStream_t>(stream)),
                        "kvq_encode_kv");
@@ -225,6 +263,7 @@ int kvq_encode_kv_paged(const kvq_codec* kc, const int8_t* signs_k, const void* 
                     j[0].c.d, j[1].c.d);
     if (j[0].n_vec == 0) return ok();
     j[0].err_word = j[1].err_word = err_word;
+    if (injected_failure()) return injected("kvq_encode_kv_paged");
     return cuda_status(kvq::launch_encode_jobs(j, 2, sm_count_current(),
                                                static_cast<cudaStream_t>(stream)),
                        "kvq_encode_kv_paged");
@@ -246,6 +285,7 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs, const kvq_plane* in
     if (n == 0) return ok();
     if (!signs || !y) return fail(KVQ_EINVAL, "kvq_dequant: NULL signs or y");
     if (!aligned16(y)) return fail(KVQ_EINVAL, "kvq_dequant: y must be 16-byte aligned");
+    if (injected_failure()) return injected("kvq_dequant");
     return cuda_status(kvq::launch_dequant(c, signs, p, n, T, pos0, static_cast<__half*>(y),
                                            sm_count_current(), static_cast<cudaStream_t>(stream)),
                        "kvq_dequant");
@@ -376,7 +416,10 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
         a.enc_k = kvq::encode_args(a.kc, signs_k);
         a.enc_v = kvq::encode_args(a.vc, signs_v);
     }
+    const int64_t wl = g_wait_limit_p1.load();
+    a.wait_limit = wl > 0 ? (uint32_t)(wl - 1) : kvq::kWaitLimit;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (injected_failure()) return injected(what);
     int rc2;
     if (hio && hio->in_bytes > 0) {
         rc2 = cuda_status(cudaMemcpyAsync(const_cast<void*>(q), hio->in_host, (size_t)hio->in_bytes,

@@ -48,7 +48,6 @@ constexpr int kTT = 128;          // tokens per staged tile
 constexpr int kMaxStages = 4;     // ring depth (2..4, chosen per launch)
 constexpr int kTPG = 4;           // tokens per group chunk
 constexpr float kLazyThr = 8.f;   // log2 units
-constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr int kTabRep = 16;       // table replicas (one per half-warp lane)
 constexpr int kTabShift = 7;      // log2(kTabRep * sizeof(float2))
 
@@ -104,9 +103,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0u;
 }
 
-// Bounded wait: false when the limit ran out.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    for (uint32_t it = 0; it < kWaitLimit; ++it)
+// Bounded wait: false when `limit` tries ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint32_t limit = kWaitLimit) {
+    for (uint32_t it = 0; it < limit; ++it)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
@@ -533,7 +533,7 @@ decode_kernel(DecodeArgs A) {
 
         for (int tile = 0; tile < nloop; tile++) {
             const int s = tile % NST;
-            const bool got = mbar_wait_bounded(&full[s], (uint32_t)(tile / NST) & 1u);
+            const bool got = mbar_wait_bounded(&full[s], (uint32_t)(tile / NST) & 1u, A.wait_limit);
             if (!__all_sync(KVQ_FULL_MASK, got)) {
                 if (lane == 0) atomicOr(&sflag[0], 1);
                 break;
@@ -664,7 +664,9 @@ decode_kernel(DecodeArgs A) {
                 const int nxt = issued;
                 const int sn = nxt % NST;
                 bool ok = true;
-                if (nxt >= NST) ok = mbar_wait_bounded(&empty[sn], (uint32_t)((nxt / NST) - 1) & 1u);
+                if (nxt >= NST)
+                    ok = mbar_wait_bounded(&empty[sn], (uint32_t)((nxt / NST) - 1) & 1u,
+                                           A.wait_limit);
                 if (ok) {
                     issue_tile(nxt);
                     issued = nxt + 1;

@@ -76,6 +76,7 @@ struct DecodeArgs {
                              // cluster and combine through distributed shared memory
     // fused append (kvq_decode_step): the new token of every (b, KV head),
     // encoded by the CTA whose split holds position ctx_len[b] - 1
+    uint32_t wait_limit;     // tries before a tile wait gives up (kvq_test_control)
     const __half* k_new;     // [B][H_kv][d] or NULL (no append)
     const __half* v_new;     // [B][H_kv][d]
     EncArgs enc_k, enc_v;    // codec, signs and constants of the two encodes
@@ -94,6 +95,9 @@ cudaError_t launch_decode_d128_g1(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d128_g2(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d128_g4(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d128_g8(const DecodeArgs& a, cudaStream_t stream);
+
+// Default number of tries of a bounded mbarrier wait.
+constexpr uint32_t kWaitLimit = 1u << 22;
 
 // Set the calling thread's kvq_last_error() message; returns `code`.
 int record_error(int code, const char* msg);

@@ -26,6 +26,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "kvq.h")
 KVQ_OK, KVQ_EINVAL, KVQ_EUNSUPPORTED, KVQ_ECUDA, KVQ_ETIMEOUT = 0, -1, -2, -3, -4
 KVQ_NORM_LIN8, KVQ_NORM_LOG4 = 0, 1
 KVQ_DEVERR_CTX_RANGE, KVQ_DEVERR_TIMEOUT, KVQ_DEVERR_PAGE_RANGE = 0x1, 0x2, 0x4
+KVQ_TEST_RESET, KVQ_TEST_FAIL_LAUNCHES, KVQ_TEST_WAIT_LIMIT = 0, 1, 2
 OUT_FP16, OUT_FP32 = 0, 1
 
 
@@ -56,6 +57,7 @@ _lib = None
 _SIGNATURES = {
     "kvq_version": (C.c_int32, []),
     "kvq_last_error": (C.c_char_p, []),
+    "kvq_test_control": (C.c_int, [C.c_int32, C.c_int64]),
     "kvq_angle_bits": (C.c_int32, [C.c_int32]),
     "kvq_row_bytes": (C.c_int64, [C.POINTER(kvq_codec), C.c_int32]),
     "kvq_encode": (C.c_int, [C.POINTER(kvq_codec), C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
@@ -164,6 +166,10 @@ def kvq_version() -> int:
 
 def kvq_last_error() -> str:
     return lib().kvq_last_error().decode()
+
+
+def kvq_test_control(key: int, value: int):
+    _check(lib().kvq_test_control(key, value))
 
 
 def kvq_angle_bits(L: int) -> int:

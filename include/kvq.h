@@ -359,6 +359,27 @@ int kvq_decode_attn_noalloc(const void* q, const kvq_codec* kc,
                             int32_t num_splits, int32_t* err_word, void* out,
                             int32_t out_dtype, void* stream);
 
+/* Test controls for the failure-detection tests.  Failures are made on the
+ * host, or by a device wait that gives up early; nothing here faults, traps
+ * or hangs the GPU.  Process-wide settings, not meant for production use.
+ *   KVQ_TEST_RESET          restores every default (value ignored)
+ *   KVQ_TEST_FAIL_LAUNCHES  value n >= 0: the next n kernel launches of this
+ *                           library are not made; each call that would have
+ *                           made one returns KVQ_ECUDA (as a failed launch
+ *                           does) with nothing queued on its stream
+ *   KVQ_TEST_WAIT_LIMIT     value n >= 0: decode kernels launched from now on
+ *                           give up a wait for a staged tile (or for a free
+ *                           stage) after n tries (n = 0: at once, without
+ *                           trying) and set KVQ_DEVERR_TIMEOUT in err_word; such
+ *                           a CTA contributes nothing to the output.  Copies
+ *                           already issued are still waited for, with the
+ *                           default limit of 2^22 tries, before a CTA exits.
+ * Returns KVQ_OK, or KVQ_EINVAL for an unknown key or a negative value. */
+#define KVQ_TEST_RESET 0
+#define KVQ_TEST_FAIL_LAUNCHES 1
+#define KVQ_TEST_WAIT_LIMIT 2
+int kvq_test_control(int32_t key, int64_t value);
+
 /* Message for the last non-OK status returned on the calling thread
  * (empty string if none).  The pointer stays valid until the next call on
  * the same thread. */

@@ -68,4 +68,4 @@ def test_reference_arm_under_torchrun_prints_once():
     assert d["value"] > 0 and d["unit"] == "GB/s" and d["higher_is_better"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
-    assert d["config"]["workload"].startswith("llama7b_layer")
+    assert d["config"]["workload"].startswith("mistral7b_32layers")

@@ -204,3 +204,130 @@ def test_paged_bad_page_entry_is_reported(dev):
     torch.cuda.synchronize()
     assert int(err.item()) & kvq.KVQ_DEVERR_PAGE_RANGE
     assert torch.isfinite(out).all()
+
+
+# --------------------------------------------------- against the oracle --
+# The tests above pin the paged forms to the contiguous ones; these compare
+# them with the fp64 oracle directly, reading the codes through the page
+# table on the host.
+
+import oracle as O  # noqa: E402
+
+from kvq_testutil import REL_L2_TOL, compare_codes, rel_l2  # noqa: E402
+
+
+def _gather(P, table, b, t0, t1, page_tokens=128):
+    """O.Codes of tokens t0 .. t1-1 of every KV head of sequence b, read
+    through the page table; rows in (h, t) order."""
+    rows = []
+    for w in range(3):
+        per_h = []
+        for h in range(P.H_kv):
+            parts = [P.rows(w)[int(table[b, t // page_tokens]), h, t % page_tokens]
+                     for t in range(t0, t1)]
+            per_h.append(torch.stack(parts) if parts else P.rows(w)[0, h, :0])
+        rows.append(np.ascontiguousarray(torch.cat(per_h).cpu().numpy()))
+    c = P.codec
+    return O.Codes(c.head_dim, c.L, c.norm_mode, *rows)
+
+
+def _oracle_attend_paged(q, Kp, Vp, table, sk, sv, ctx_lens, G, tau):
+    B, H_q, d = q.shape
+    H_kv = H_q // G
+    want = np.zeros((B, H_q, d))
+    for b in range(B):
+        n = int(ctx_lens[b])
+        kcodes, vcodes = _gather(Kp, table, b, 0, n), _gather(Vp, table, b, 0, n)
+        for h in range(H_kv):
+            kh = O.dequant(kcodes.take(slice(h * n, (h + 1) * n)), sk)
+            vh = O.dequant(vcodes.take(slice(h * n, (h + 1) * n)), sv)
+            want[b, h * G:(h + 1) * G] = O.attend(q[b, h * G:(h + 1) * G].astype(np.float64),
+                                                   kh, vh, tau)
+    return want
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("S", [1, 4])
+def test_paged_decode_matches_oracle(dev, S):
+    """Paged decode attention over ragged sequences (a one-token sequence, one
+    ending on a page's first row, one spanning six pages) against textbook
+    attention on the oracle's dequantization of the rows the table maps."""
+    B, H_kv, G, d, max_pages = 3, 2, 4, 128, 6
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=20 + S)
+    H_q = G * H_kv
+    qn = np.random.default_rng(21).standard_normal((B, H_q, d)).astype(np.float16)
+    q = torch.from_numpy(qn).cuda()
+    ctx_lens = [1, 129, 768]
+    ctx = torch.tensor(ctx_lens, dtype=torch.int32, device="cuda")
+    tau = 1 / math.sqrt(d)
+    ws = _ws(B, H_q, d, S)
+    out = torch.empty((B, H_q, d), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.kvq_decode_attn_paged(q, kc, vc, sk, sv, Kp.c(), Vp.c(), ctx, B, H_q, H_kv, 768, tau, S,
+                              ws.buf, ws.nbytes, err, out, kvq.OUT_FP32)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    want = _oracle_attend_paged(qn, Kp, Vp, table, sk.cpu().numpy(), sv.cpu().numpy(), ctx_lens,
+                                G, tau)
+    assert rel_l2(out.cpu().numpy(), want).max() <= REL_L2_TOL
+
+
+@pytest.mark.gpu
+def test_paged_encode_matches_oracle(dev):
+    """kvq_encode_kv_paged over tokens 50 .. 349 (three pages, both page
+    boundaries crossed): the codes the table maps equal the oracle's codes of
+    the same vectors, under the parity rule."""
+    B, H_kv, d, max_pages = 2, 3, 128, 4
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=25)
+    rng = np.random.default_rng(26)
+    kn = rng.standard_normal((B, H_kv, 300, d)).astype(np.float16)
+    kn[..., 5] *= 20
+    vn = rng.standard_normal((B, H_kv, 300, d)).astype(np.float16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.kvq_encode_kv_paged(kc, sk, torch.from_numpy(kn).cuda(), Kp.c(), vc, sv,
+                            torch.from_numpy(vn).cuda(), Vp.c(), B, H_kv, 300, 50, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for P, x, s, c in ((Kp, kn, sk, kc), (Vp, vn, sv, vc)):
+        want = O.encode(x, s.cpu().numpy(), c.L, c.norm_mode)
+        for b in range(B):
+            got = _gather(P, table, b, 50, 350)
+            rows = slice(b * H_kv * 300, (b + 1) * H_kv * 300)
+            compare_codes((got.angles, got.norms, got.params), want.take(rows))
+
+
+@pytest.mark.gpu
+def test_paged_decode_step_matches_oracle(dev):
+    """The fused paged step with appends on a page's first row (ctx 129), its
+    last row (ctx 256) and mid-page (ctx 300): the appended rows equal the
+    oracle's codes of the new vectors, and the output equals textbook
+    attention over the oracle's dequantization of the mapped rows."""
+    B, H_kv, G, d, max_pages = 3, 2, 4, 128, 4
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=27)
+    H_q = G * H_kv
+    rng = np.random.default_rng(28)
+    qn = rng.standard_normal((B, H_q, d)).astype(np.float16)
+    kn = rng.standard_normal((B, H_kv, d)).astype(np.float16)
+    kn[..., 9] *= 20
+    vn = rng.standard_normal((B, H_kv, d)).astype(np.float16)
+    ctx_lens = [129, 256, 300]
+    ctx = torch.tensor(ctx_lens, dtype=torch.int32, device="cuda")
+    S, tau = 3, 1 / math.sqrt(d)
+    ws = _ws(B, H_q, d, S)
+    out = torch.empty((B, H_q, d), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.kvq_decode_step_paged(torch.from_numpy(qn).cuda(), torch.from_numpy(kn).cuda(),
+                              torch.from_numpy(vn).cuda(), kc, vc, sk, sv, Kp.c(), Vp.c(), ctx,
+                              B, H_q, H_kv, 512, tau, S, ws.buf, ws.nbytes, err, out,
+                              kvq.OUT_FP32)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for P, x, s, c in ((Kp, kn, sk, kc), (Vp, vn, sv, vc)):
+        want = O.encode(x, s.cpu().numpy(), c.L, c.norm_mode)
+        for b, n in enumerate(ctx_lens):
+            got = _gather(P, table, b, n - 1, n)
+            compare_codes((got.angles, got.norms, got.params),
+                          want.take(slice(b * H_kv, (b + 1) * H_kv)))
+    want = _oracle_attend_paged(qn, Kp, Vp, table, sk.cpu().numpy(), sv.cpu().numpy(), ctx_lens,
+                                G, tau)
+    assert rel_l2(out.cpu().numpy(), want).max() <= REL_L2_TOL

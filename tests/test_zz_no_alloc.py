@@ -52,29 +52,68 @@ def _rel_l2(a, b):
     return ((a - b).norm(dim=1) / b.norm(dim=1).clamp_min(1e-30)).max().item()
 
 
-@pytest.mark.parametrize("name,ctx_lens", [
-    ("llama7b_layer_b1_hq32_hkv8_d128_ctx4096", None),
-    ("tiny_b1_hq4_hkv2_d128_ctx256", [200]),
+def _noalloc(w, kc, vc, skd, svd, Kp, Vp, q, ctx, tau, S, err, like):
+    out = torch.full_like(like, float("nan"))
+    kvq.kvq_decode_attn_noalloc(q, kc, vc, skd, svd, Kp.c(), Vp.c(), ctx, w.B, w.H_q, w.H_kv,
+                                w.ctx, tau, S, err, out, kvq.OUT_FP32)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("name,ctx_lens,splits", [
+    # 16 splits of 8 KV heads: one cluster per KV head, partials in shared memory
+    ("llama7b_layer_b1_hq32_hkv8_d128_ctx4096", None, None),
+    # 20 splits (more than a cluster takes): partials and completion counters
+    # in the built-in scratch array, merged by the last CTA of each KV head
+    ("llama7b_layer_b1_hq32_hkv8_d128_ctx4096", None, 20),
+    ("tiny_b1_hq4_hkv2_d128_ctx256", [200], None),
 ])
-def test_noalloc_matches_workspace_entry_point(ready, name, ctx_lens):
+def test_noalloc_matches_workspace_entry_point(ready, name, ctx_lens, splits):
+    """Same kernel, same splits, same inputs: the output is bit-identical to
+    kvq_decode_attn with a caller workspace, on two calls in a row."""
     dev = ready
     w = synth.WORKLOADS[name]
     kc, vc, skd, svd, Kp, Vp, q = _layer(w, 0, dev)
     ctx_vals = ctx_lens or [w.ctx] * w.B
     ctx = torch.tensor(ctx_vals, dtype=torch.int32, device=dev)
     sm = torch.cuda.get_device_properties(dev).multi_processor_count
-    S = kvq.kvq_decode_num_splits(w.B, w.H_kv, w.ctx, sm)
+    S = splits or kvq.kvq_decode_num_splits(w.B, w.H_kv, w.ctx, sm)
     tau = 1.0 / math.sqrt(w.d)
     ref = kvq.decode_attn(q, kc, vc, skd, svd, Kp, Vp, ctx, w.ctx, tau, num_splits=S,
                           out_dtype=kvq.OUT_FP32)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     for call in range(2):
-        out = torch.full_like(ref, float("nan"))
-        kvq.kvq_decode_attn_noalloc(q, kc, vc, skd, svd, Kp.c(), Vp.c(), ctx, w.B, w.H_q, w.H_kv,
-                                    w.ctx, tau, S, err, out, kvq.OUT_FP32)
-        torch.cuda.synchronize()
-        assert torch.isfinite(out).all(), call
-        assert _rel_l2(out, ref) <= REL_L2_TOL, (call, _rel_l2(out, ref))
+        out = _noalloc(w, kc, vc, skd, svd, Kp, Vp, q, ctx, tau, S, err, ref)
+        assert torch.equal(out, ref), call
+    assert int(err.item()) == 0
+    assert _rel_l2(out, ref) <= REL_L2_TOL
+
+
+def test_noalloc_scratch_reuse_across_calls(ready):
+    """Calls in a row share the array and find the previous call's partials
+    and counters there: 20 splits, then 7 splits over a shorter context (its
+    counters are fewer and its partials land elsewhere), a call rejected for
+    its size, 20 splits again with another query; each equals its
+    workspace-entry-point twin."""
+    dev = ready
+    w = synth.WORKLOADS["llama7b_layer_b1_hq32_hkv8_d128_ctx4096"]
+    kc, vc, skd, svd, Kp, Vp, q = _layer(w, 0, dev)
+    tau = 1.0 / math.sqrt(w.d)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    q2 = torch.flip(q, dims=[1]).contiguous()
+    plan = [(20, w.ctx, q), (7, 1500, q), (None, w.ctx, q), (20, w.ctx, q2)]
+    for S, n, qq in plan:
+        ctx = torch.tensor([n], dtype=torch.int32, device=dev)
+        if S is None:
+            out = torch.zeros((1, w.H_q, w.d), dtype=torch.float32, device=dev)
+            with pytest.raises(kvq.KvqError):
+                kvq.kvq_decode_attn_noalloc(qq, kc, vc, skd, svd, Kp.c(), Vp.c(), ctx, 1, w.H_q,
+                                            w.H_kv, w.ctx, tau, 65535, err, out, kvq.OUT_FP32)
+            continue
+        ref = kvq.decode_attn(qq, kc, vc, skd, svd, Kp, Vp, ctx, w.ctx, tau, num_splits=S,
+                              out_dtype=kvq.OUT_FP32)
+        out = _noalloc(w, kc, vc, skd, svd, Kp, Vp, qq, ctx, tau, S, err, ref)
+        assert torch.equal(out, ref), (S, n)
     assert int(err.item()) == 0
 
 
