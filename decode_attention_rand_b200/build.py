@@ -23,7 +23,8 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 OUT = os.path.join(HERE, "libkvq.so")
 BUILD = os.path.join(ROOT, "_build")
-SOURCES = ["kvq_abi.cu", "kvq_encode.cu", "kvq_dequant.cu", "kvq_decode.cu", "kvq_noalloc.cu"] + [
+SOURCES = ["kvq_abi.cu", "kvq_encode.cu", "kvq_dequant.cu", "kvq_decode.cu", "kvq_noalloc.cu",
+           "kvq_decode_generic.cu"] + [
     f"kvq_decode_d{d}_g{g}.cu" for d in (64, 128) for g in (1, 2, 4, 8)]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -43,7 +44,9 @@ def source_digest(extra_flags=()) -> str:
         h.update(os.path.basename(f).encode() + b"\0")
         with open(f, "rb") as fh:
             h.update(fh.read())
-    h.update(" ".join([*FLAGS, *extra_flags]).encode())
+    # the flags without the include directory's absolute path (it differs
+    # between checkouts of the same sources)
+    h.update(" ".join([f for f in (*FLAGS, *extra_flags) if not os.path.isabs(f)]).encode())
     return h.hexdigest()
 
 

@@ -378,12 +378,6 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
         return fail(KVQ_EINVAL, "%s: out_dtype must be 0 (fp16) or 1 (fp32)", what);
     if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
         return fail(KVQ_EINVAL, "%s: softmax_scale is not finite", what);
-    const int G = H_q / H_kv;
-    if (!kvq::decode_supported(a.kc.d, G, a.kc.L, a.vc.L, a.kc.mode, a.vc.mode))
-        return fail(KVQ_EUNSUPPORTED,
-                    "%s: no kernel for head_dim %d, G %d, L_K %d, L_V %d "
-                    "(built: head_dim 64/128, G 1/2/4/8, L <= 256)",
-                    what, a.kc.d, G, a.kc.L, a.vc.L);
     const int64_t need = kvq_decode_workspace_bytes(B, H_q, a.kc.d, num_splits);
     if (!workspace || ws_bytes < need)
         return fail(KVQ_EINVAL, "%s: workspace of %lld bytes is below the %lld needed", what,

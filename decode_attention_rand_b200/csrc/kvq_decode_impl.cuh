@@ -26,8 +26,19 @@
 //   - consumer warps take blocks of consecutive tokens; a group of NL lanes
 //     owns four tokens, each lane PP pairs of them and the matching pairs of
 //     all G query heads of the KV head (GQA), so every unpacked code serves G
-//     heads; partial scores meet in a transpose-reduce over the group, the
-//     softmax weights travel back the same way;
+//     heads;
+//   - the work per pair is kept to a handful of instructions: a key norm
+//     byte becomes the float 1 + c 2^-15 in one byte permute, and with the
+//     key table holding 2^15 (cos, sin), fma(f, U, -U) is c (cos, sin)
+//     rounded once (no int-to-float conversion); a value norm nibble is
+//     or-ed into the mantissa of 1.0 (f = 1 + c/16) and one FMA gives the
+//     exponent LO + c (HI - LO)/15; table bases are folded into the load
+//     address where the tables fit in static shared memory;
+//   - partial scores meet in a transpose-reduce over the group in which every
+//     lane sends the same register each round: a lane's query heads and token
+//     order are permuted once, by its lane bits, so no per-round select is
+//     needed; the softmax weights reach the value pass through a small
+//     per-warp buffer in shared memory as (p, p) pairs;
 //   - angle codes have compile-time widths (BK, BV in 5..8; 0 = runtime) so
 //     a code becomes a table offset in two integer operations; bin-centre
 //     cos/sin tables are replicated 16 times so a half-warp's 64-bit lookups
@@ -38,6 +49,8 @@
 //     (batch, KV head) to finish (atomic counter, no waiting) merges the
 //     splits, divides by l, applies the inverse FWHT and D_V / sqrt(d).
 #pragma once
+
+#include <mutex>
 
 #include "kvq_encode_impl.cuh"
 #include "kvq_internal.h"
@@ -51,6 +64,12 @@ constexpr float kLazyThr = 8.f;   // log2 units
 constexpr int kTabRep = 16;       // table replicas (one per half-warp lane)
 constexpr int kTabShift = 7;      // log2(kTabRep * sizeof(float2))
 
+// True when the two replicated cos/sin tables of fixed code widths (bk, bv)
+// fit in static shared memory (48 KB).
+constexpr bool decode_static_tables(int bk, int bv) {
+    return bk > 0 && bv > 0 && ((1 << bk) + (1 << bv)) * kTabRep * 8 <= 48 * 1024;
+}
+
 template <int D, int G>
 struct DecCfg {
     static constexpr int P = D / 2;
@@ -63,6 +82,7 @@ struct DecCfg {
     static constexpr int NG = WARPS * GPW;                     // groups per CTA
     static constexpr int V = kTPG * G;                         // partial sums per lane
     static constexpr int VF = V / NL;                          // final sums per lane
+    static constexpr int PBUF = TW * G * 2;                    // floats of (p, p) per warp
     static_assert(VF >= 1, "group too wide");
     static_assert(PP % 4 == 0, "codes are unpacked four at a time");
     static_assert(kTT % (TW * WARPS) == 0, "blocks must tile the stage");
@@ -192,41 +212,20 @@ __device__ __forceinline__ float4 dsmem_f32x4(uint32_t addr) {
 
 // ------------------------------------------------------- group exchange --
 
-// Transpose-reduce over the NL lanes of a group: on return v[0..VF) holds the
-// group sums of entries lg*VF + e.
+// Reduce over the NL lanes of a group, halving the live entries each round:
+// every lane adds its partner's v[i + half] to its own v[i].  For the result
+// to be a transpose-reduce, slot i of lane lg must hold logical entry
+// i ^ (lg * VF) (the caller arranges that once, by permuting the query heads
+// and token order it computes into each slot); then on return v[0..VF) holds
+// the group sums of the logical entries lg * VF + e.
 template <int V, int NL>
-__device__ __forceinline__ void transpose_reduce(float (&v)[V], int lg) {
+__device__ __forceinline__ void xor_reduce(float (&v)[V]) {
 #pragma unroll
     for (int r = 0; (NL >> (r + 1)) >= 1; r++) {
         const int o = NL >> (r + 1);
         const int half = V >> (r + 1);
-        const bool upper = (lg & o) != 0;
 #pragma unroll
-        for (int i = 0; i < half; i++) {
-            const float send = upper ? v[i] : v[i + half];
-            const float keep = upper ? v[i + half] : v[i];
-            v[i] = keep + __shfl_xor_sync(KVQ_FULL_MASK, send, o);
-        }
-    }
-}
-
-// Inverse of transpose_reduce: from v[0..VF) (entries lg*VF + e) rebuild all
-// V entries in every lane of the group.
-template <int V, int NL>
-__device__ __forceinline__ void transpose_gather(float (&v)[V], int lg) {
-    constexpr int VF = V / NL;
-#pragma unroll
-    for (int r = 0; (1 << r) < NL; r++) {
-        const int o = 1 << r;
-        const int cur = VF << r;
-        const bool upper = (lg & o) != 0;
-#pragma unroll
-        for (int i = 0; i < cur; i++) {
-            const float mine = v[i];
-            const float other = __shfl_xor_sync(KVQ_FULL_MASK, mine, o);
-            v[i] = upper ? other : mine;
-            v[i + cur] = upper ? mine : other;
-        }
+        for (int i = 0; i < half; i++) v[i] += __shfl_xor_sync(KVQ_FULL_MASK, v[i + half], o);
     }
 }
 
@@ -296,11 +295,6 @@ __device__ __forceinline__ void load_bytes(const uint8_t* p, uint32_t (&w)[(NBYT
     }
 }
 
-__device__ __forceinline__ float2 lds_f2(uint32_t smem_addr) {
-    float2 v;
-    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(smem_addr));
-    return v;
-}
 
 // ------------------------------------------------------------- kernel ---
 
@@ -320,16 +314,25 @@ decode_kernel(DecodeArgs A) {
     constexpr int EPQ = D / 32;
     constexpr int CONSUMERS = WARPS * 32;
 
+    // cos/sin tables: in static shared memory when both widths are fixed and
+    // the tables fit (their address is then a constant of the load), in the
+    // dynamic allocation otherwise
+    constexpr bool kStatic = decode_static_tables(BK, BV);
+    __shared__ __align__(128) float2 s_tab[kStatic ? ((1 << BK) + (1 << BV)) * kTabRep : 1];
     extern __shared__ __align__(16) unsigned char smem[];
     const int NST = A.nstages;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);           // [kMaxStages]
     uint64_t* empty = full + kMaxStages;                          // [kMaxStages]
     int* sflag = reinterpret_cast<int*>(smem + 16 * kMaxStages);  // timeout, last
     const int nK = 1 << A.kc.bits, nV = 1 << A.vc.bits;
-    float2* tabK = reinterpret_cast<float2*>(smem + 16 * kMaxStages + 16);  // [2^bK][16]
-    float2* tabV = tabK + nK * kTabRep;                           // [2^bV][16]
-    float* qs = reinterpret_cast<float*>(tabV + nV * kTabRep);    // [G][D]
+    unsigned char* dyn = smem + 16 * kMaxStages + 16;
+    // key table: 2^15 (cos, sin) [2^bK][16]; value table: (cos, sin) [2^bV][16]
+    float2* tabK = kStatic ? s_tab : reinterpret_cast<float2*>(dyn);
+    float2* tabV = tabK + nK * kTabRep;
+    if (!kStatic) dyn += sizeof(float2) * kTabRep * (size_t)(nK + nV);
+    float* qs = reinterpret_cast<float*>(dyn);                    // [G][D]
     uint32_t* encst = reinterpret_cast<uint32_t*>(qs + G * D);    // [2][kEncStageWords]
+    float* pbuf_all = reinterpret_cast<float*>(encst + 2 * kEncStageWords);  // [WARPS][PBUF]
     unsigned char* stages = smem + A.stage_offset;                // [kStages][stage]
 
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -449,7 +452,9 @@ decode_kernel(DecodeArgs A) {
             const int a = isK ? e : e - nK;
             float s, c;
             sincospif((float)(2 * a + 1) / (float)(isK ? A.kc.L : A.vc.L) - 1.f, &s, &c);
-            tabK[e * kTabRep] = make_float2(c, s);
+            // key entries scaled by 2^15 (exact): see the norm decoding below
+            const float sc = isK ? 32768.f : 1.f;
+            tabK[e * kTabRep] = make_float2(c * sc, s * sc);
         }
         named_barrier(2, nthr);
 #pragma unroll 1
@@ -516,19 +521,31 @@ decode_kernel(DecodeArgs A) {
 #pragma unroll
     for (int e = 0; e < VF; e++) lpart[e] = 0.f;
 
+    // Slot (j, h) of this lane's partial scores holds the logical entry
+    // (j ^ JX, h ^ HX) (token slot, head) so that xor_reduce needs no selects;
+    // after it, final entry e is logical M + e: token slot (M + e) / G, head
+    // (M + e) % G, with softmax reference mh[e].
+    const int M = lg * VF;
+    const int HX = M % G, JX = M / G;
+    float mh[VF];
+#pragma unroll
+    for (int e = 0; e < VF; e++) mh[e] = -INFINITY;
+    float* pbuf = pbuf_all + warp * Cfg::PBUF;  // [TW][G] (p, p) of this warp's block
+
     {
         f32x2 q2[G][PP];
 #pragma unroll
         for (int h = 0; h < G; h++)
 #pragma unroll
             for (int k = 0; k < PP; k++) {
-                const float2 qq = reinterpret_cast<const float2*>(qs + h * D)[lg * PP + k];
+                const float2 qq = reinterpret_cast<const float2*>(qs + (h ^ HX) * D)[lg * PP + k];
                 q2[h][k] = pack2(qq.x, qq.y);
             }
         const int bitsK = BK > 0 ? BK : A.kc.bits, bitsV = BV > 0 ? BV : A.vc.bits;
         const int cbK = lg * PP * bitsK, cbV = lg * PP * bitsV;
         const uint32_t lane_off = (uint32_t)(lane & 15) * 8u;
-        const uint32_t tK = smem_u32(tabK), tV = smem_u32(tabV);
+        const unsigned char* tKb = reinterpret_cast<const unsigned char*>(tabK);
+        const unsigned char* tVb = reinterpret_cast<const unsigned char*>(tabV);
         const int awK = A.kc.angle_words, awV = A.vc.angle_words;
 
         for (int tile = 0; tile < nloop; tile++) {
@@ -550,12 +567,12 @@ decode_kernel(DecodeArgs A) {
             const int ntok = (int)((t1 - tt0) < kTT ? (t1 - tt0) : kTT);
 
             for (int blk = warp; blk * TW < ntok; blk += WARPS) {
-                // token of slot j of this group: consecutive rows across the warp
-                // -- scores: partial dot products of this lane's pairs --------
+                // -- scores: this lane's partial dot products, slot (j, h) --
+                // token slot j ^ JX (rows consecutive across the warp), head h ^ HX
                 float part[V];
 #pragma unroll
                 for (int j = 0; j < kTPG; j++) {
-                    const int t = blk * TW + j * GPW + grp;
+                    const int t = blk * TW + (j ^ JX) * GPW + grp;
                     uint32_t off[PP];
                     angle_offsets<PP, BK>(sKa + t * awK, cbK, bitsK, lane_off, off);
                     uint32_t nw[(PP + 3) / 4];
@@ -565,31 +582,30 @@ decode_kernel(DecodeArgs A) {
                     for (int h = 0; h < G; h++) dot[h] = 0ull;
 #pragma unroll
                     for (int k = 0; k < PP; k++) {
-                        const float cf = (float)((nw[k / 4] >> (8 * (k % 4))) & 0xFFu);
-                        const float2 cs = lds_f2(tK + off[k]);
-                        const f32x2 xy = pack2(cf * cs.x, cf * cs.y);
+                        // norm byte c -> f = 1 + c 2^-15 (bytes 0x3F 0x80 c 0x00);
+                        // the key table holds U = 2^15 (cos, sin), so
+                        // fma(f, U, -U) = (f - 1) U = c (cos, sin), rounded once
+                        const float f = __uint_as_float(
+                            __byte_perm(nw[k / 4], 0x3F800000u, 0x7604u | ((k % 4) << 4)));
+                        const float2 U = *reinterpret_cast<const float2*>(tKb + off[k]);
+                        const f32x2 xy = pack2(fmaf(f, U.x, -U.x), fmaf(f, U.y, -U.y));
 #pragma unroll
                         for (int h = 0; h < G; h++) dot[h] = fma2(q2[h][k], xy, dot[h]);
                     }
 #pragma unroll
                     for (int h = 0; h < G; h++) part[j * G + h] = lo2(dot[h]) + hi2(dot[h]);
                 }
-                transpose_reduce<V, NL>(part, lg);
+                xor_reduce<V, NL>(part);
                 // -- scale by M/255 * tau * log2(e), mask, lazy softmax reference
                 bool need = false;
 #pragma unroll
                 for (int e = 0; e < VF; e++) {
-                    const int idx = lg * VF + e;
-                    const int j = idx / G, h = idx % G;
-                    const int t = blk * TW + j * GPW + grp;
-                    const float M = half_bits_to_float(sKp[t]);
-                    float sv = part[e] * (M * (1.f / 255.f)) * A.scale_log2;
+                    const int t = blk * TW + ((M + e) / G) * GPW + grp;
+                    const float Mk = half_bits_to_float(sKp[t]);
+                    float sv = part[e] * (Mk * (1.f / 255.f)) * A.scale_log2;
                     sv = t < ntok ? sv : -INFINITY;
                     part[e] = sv;
-                    float mh = mref[0];
-#pragma unroll
-                    for (int hh = 1; hh < G; hh++) mh = (hh == h) ? mref[hh] : mh;
-                    need |= sv > mh + kLazyThr;
+                    need |= sv > mh[e] + kLazyThr;
                 }
                 if (__any_sync(KVQ_FULL_MASK, need)) {
                     float mx[G];
@@ -597,7 +613,7 @@ decode_kernel(DecodeArgs A) {
                     for (int h = 0; h < G; h++) mx[h] = -INFINITY;
 #pragma unroll
                     for (int e = 0; e < VF; e++) {
-                        const int h = (lg * VF + e) % G;
+                        const int h = (M + e) % G;
 #pragma unroll
                         for (int hh = 0; hh < G; hh++)
                             if (hh == h) mx[hh] = fmaxf(mx[hh], part[e]);
@@ -612,44 +628,69 @@ decode_kernel(DecodeArgs A) {
                         for (int k = 0; k < PP; k++) acc[h][k] = mul2(acc[h][k], al2);
 #pragma unroll
                         for (int e = 0; e < VF; e++)
-                            if ((lg * VF + e) % G == h) lpart[e] *= al;
+                            if ((M + e) % G == h) lpart[e] *= al;
                         mref[h] = mn;
                     }
+#pragma unroll
+                    for (int e = 0; e < VF; e++) {
+                        const int h = (M + e) % G;
+                        float m = mref[0];
+#pragma unroll
+                        for (int hh = 1; hh < G; hh++) m = (hh == h) ? mref[hh] : m;
+                        mh[e] = m;
+                    }
                 }
+                // -- softmax weights to this warp's buffer as (p, p) pairs --
+                __syncwarp();  // the previous block's value pass is done with it
 #pragma unroll
                 for (int e = 0; e < VF; e++) {
-                    const int h = (lg * VF + e) % G;
-                    float mh = mref[0];
-#pragma unroll
-                    for (int hh = 1; hh < G; hh++) mh = (hh == h) ? mref[hh] : mh;
-                    const float p = part[e] == -INFINITY ? 0.f : ex2(part[e] - mh);
-                    part[e] = p;
+                    const int idx = M + e;
+                    const float p = part[e] == -INFINITY ? 0.f : ex2(part[e] - mh[e]);
                     lpart[e] += p;
+                    reinterpret_cast<float2*>(pbuf)[((idx / G) * GPW + grp) * G + idx % G] =
+                        make_float2(p, p);
                 }
-                transpose_gather<V, NL>(part, lg);
+                __syncwarp();
                 // -- values: acc[h] += p[t][h] * r^ (cos, sin), rotated domain --
 #pragma unroll
                 for (int j = 0; j < kTPG; j++) {
-                    const int t = blk * TW + j * GPW + grp;
+                    const int tl = j * GPW + grp;
+                    const int t = blk * TW + tl;
+                    f32x2 pw[G];
+                    if constexpr (G == 1) {
+                        const float2 v = reinterpret_cast<const float2*>(pbuf)[tl];
+                        pw[0] = pack2(v.x, v.y);
+                    } else {
+#pragma unroll
+                        for (int h2 = 0; h2 < G / 2; h2++) {
+                            const float4 v = reinterpret_cast<const float4*>(pbuf + tl * G * 2)[h2];
+                            pw[2 * h2] = pack2(v.x, v.y);
+                            pw[2 * h2 + 1] = pack2(v.z, v.w);
+                        }
+                    }
                     uint32_t off[PP];
                     angle_offsets<PP, BV>(sVa + t * awV, cbV, bitsV, lane_off, off);
                     uint32_t nw[(PP / 2 + 3) / 4];
                     load_bytes<PP / 2>(sVn + t * (P / 2) + lg * (PP / 2), nw);
                     const uint32_t pr = sVp[t];
-                    float LO = half_bits_to_float((uint16_t)(pr & 0xFFFF));
-                    float step = (half_bits_to_float((uint16_t)(pr >> 16)) - LO) * (1.f / 15.f);
+                    const float LO = half_bits_to_float((uint16_t)(pr & 0xFFFF));
+                    // log2 r^ = LO + c (HI - LO)/15 = f A + B with f = 1 + c/16,
+                    // A = 16 (HI - LO)/15, B = LO - A
+                    float A16 = (half_bits_to_float((uint16_t)(pr >> 16)) - LO) * (16.f / 15.f);
+                    float B16 = LO - A16;
                     // rows past the context hold stale bytes: make their r^ finite
                     // (their softmax weight is already 0)
-                    LO = t < ntok ? LO : -64.f;
-                    step = t < ntok ? step : 0.f;
-                    f32x2 pw[G];
-#pragma unroll
-                    for (int h = 0; h < G; h++) pw[h] = pack2(part[j * G + h], part[j * G + h]);
+                    A16 = t < ntok ? A16 : 0.f;
+                    B16 = t < ntok ? B16 : -64.f;
 #pragma unroll
                     for (int k = 0; k < PP; k++) {
-                        const float cf = (float)((nw[k / 8] >> (4 * (k % 8))) & 0xFu);
-                        const float r = ex2(fmaf(cf, step, LO));
-                        const float2 cs = lds_f2(tV + off[k]);
+                        // nibble k of the word -> mantissa bits 19..22 of 1.0
+                        const int sh = 4 * (k % 8);
+                        const uint32_t w = nw[k / 8];
+                        const uint32_t mant = sh <= 19 ? (w << (19 - sh)) : (w >> (sh - 19));
+                        const float f = __uint_as_float((mant & 0x00780000u) | 0x3F800000u);
+                        const float r = ex2(fmaf(f, A16, B16));
+                        const float2 cs = *reinterpret_cast<const float2*>(tVb + off[k]);
                         const f32x2 xy = pack2(r * cs.x, r * cs.y);
 #pragma unroll
                         for (int h = 0; h < G; h++) acc[h][k] = fma2(pw[h], xy, acc[h][k]);
@@ -927,14 +968,17 @@ decode_kernel(DecodeArgs A) {
 
 // ------------------------------------------------------------------ host --
 
-// Shared-memory plan of one launch (ring depth 4, 3 or 2, whichever fits);
-// returns 0 bytes when even two stages do not fit.
-template <int D, int G>
-inline size_t decode_smem_plan(DecodeArgs& a) {
+// Shared-memory plan of one launch (ring depth 4, 3 or 2, whichever fits in
+// `avail` bytes of dynamic shared memory); returns 0 bytes when even two
+// stages do not fit.
+template <int D, int G, int BK, int BV>
+inline size_t decode_smem_plan(DecodeArgs& a, size_t avail) {
     using Cfg = DecCfg<D, G>;
-    size_t off = 16 * kMaxStages + 16 +
-                 sizeof(float2) * kTabRep * (size_t)((1 << a.kc.bits) + (1 << a.vc.bits)) +
-                 sizeof(float) * G * D + sizeof(uint32_t) * 2 * kEncStageWords;
+    size_t off = 16 * kMaxStages + 16;
+    if (!decode_static_tables(BK, BV))
+        off += sizeof(float2) * kTabRep * (size_t)((1 << a.kc.bits) + (1 << a.vc.bits));
+    off += sizeof(float) * G * D + sizeof(uint32_t) * 2 * kEncStageWords +
+           sizeof(float) * Cfg::WARPS * Cfg::PBUF;
     off = (off + 15) / 16 * 16;
     a.stage_offset = (int)off;
     const int rb[6] = {a.kc.angle_words * 4, a.kc.norm_bytes, a.kc.param_bytes,
@@ -953,7 +997,7 @@ inline size_t decode_smem_plan(DecodeArgs& a) {
     for (int ns = kMaxStages; ns >= 2; ns--) {
         size_t ring = (size_t)ns * sb;
         if (ring < merge) ring = merge;
-        if (off + ring <= 227 * 1024) {
+        if (off + ring <= avail) {
             a.nstages = ns;
             return off + ring;
         }
@@ -964,39 +1008,58 @@ inline size_t decode_smem_plan(DecodeArgs& a) {
 // Largest cluster the combine uses (non-portable beyond 8 CTAs).
 constexpr int kMaxClusterSplits = 16;
 
+// Per-device launch facts of one kernel instance, set up once under a lock:
+// SM count, the dynamic shared memory left beside its static tables, and how
+// many clusters of S CTAs can be resident at once for a given dynamic size
+// (the generic-width instance's size varies with the code widths).
+struct DecodeLaunchCache {
+    std::mutex lock;
+    bool init[64] = {};
+    int sm_count[64] = {};
+    size_t avail[64] = {};
+    struct Entry {
+        int dev, S;
+        size_t smem;
+        int n;
+    };
+    Entry entries[256];
+    int n_entries = 0;
+};
+
 template <int D, int G, int BK, int BV>
 inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
     using Cfg = DecCfg<D, G>;
     auto kernel = decode_kernel<D, G, BK, BV>;
-    const size_t smem = decode_smem_plan<D, G>(a);
-    if (smem == 0) return cudaErrorInvalidConfiguration;
-    static bool attr_done[64] = {};
-    static int sm_count[64] = {};
-    // per device and split count: how many clusters of that many CTAs can be
-    // resident at once (-1 unknown)
-    static int cluster_max[64][kMaxClusterSplits + 1];
-    static bool cluster_init[64] = {};
+    static DecodeLaunchCache cache;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const bool cache = dev >= 0 && dev < 64;
-    if (!cache || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        int n = 0;
-        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        if (cache) {
-            sm_count[dev] = n;
-            if (!cluster_init[dev]) {
-                for (int k = 0; k <= kMaxClusterSplits; k++) cluster_max[dev][k] = -1;
-                cluster_init[dev] = true;
-            }
-            attr_done[dev] = true;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    size_t avail;
+    int sm_count;
+    {
+        std::lock_guard<std::mutex> g(cache.lock);
+        if (!cache.init[dev]) {
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, kernel);
+            if (e != cudaSuccess) return e;
+            const size_t dyn = 227 * 1024 - fa.sharedSizeBytes;
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+            if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+            int n = 0;
+            e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            cache.sm_count[dev] = n;
+            cache.avail[dev] = dyn;
+            cache.init[dev] = true;
         }
+        avail = cache.avail[dev];
+        sm_count = cache.sm_count[dev];
     }
+    const size_t smem = decode_smem_plan<D, G, BK, BV>(a, avail);
+    if (smem == 0) return cudaErrorInvalidConfiguration;
     dim3 grid((unsigned)a.num_splits, (unsigned)a.H_kv, (unsigned)a.B);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -1017,20 +1080,27 @@ inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
     // occupancy calculator rather than count SMs
     const int S = a.num_splits;
     a.cluster = 0;
-    if (cache && S <= kMaxClusterSplits &&
-        (int64_t)a.B * a.H_kv * S <= (int64_t)sm_count[dev]) {
-        if (cluster_max[dev][S] < 0) {
+    if (S <= kMaxClusterSplits && (int64_t)a.B * a.H_kv * S <= (int64_t)sm_count) {
+        int n = -1;
+        {
+            std::lock_guard<std::mutex> g(cache.lock);
+            for (int i = 0; i < cache.n_entries; i++)
+                if (cache.entries[i].dev == dev && cache.entries[i].S == S &&
+                    cache.entries[i].smem == smem)
+                    n = cache.entries[i].n;
+        }
+        if (n < 0) {
             cfg.attrs = attr;
             cfg.numAttrs = 1;
-            int n = 0;
             const cudaError_t q = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
             if (q != cudaSuccess) {
                 (void)cudaGetLastError();
                 n = 0;
             }
-            cluster_max[dev][S] = n;
+            std::lock_guard<std::mutex> g(cache.lock);
+            if (cache.n_entries < 256) cache.entries[cache.n_entries++] = {dev, S, smem, n};
         }
-        a.cluster = (int64_t)a.B * a.H_kv <= (int64_t)cluster_max[dev][S];
+        a.cluster = (int64_t)a.B * a.H_kv <= (int64_t)n;
     }
     cfg.attrs = a.cluster ? attr : attr + 1;
     cfg.numAttrs = a.cluster ? 2 : 1;

@@ -82,11 +82,12 @@ struct DecodeArgs {
     EncArgs enc_k, enc_v;    // codec, signs and constants of the two encodes
 };
 
-// True when the decode kernels are built for this (head_dim, G, L_K, L_V)
-// and norm-mode combination.
-bool decode_supported(int d, int G, int LK, int LV, int mode_k, int mode_v);
+// True when the staged decode kernel is built for this (head_dim, G, L_K,
+// L_V) and norm-mode combination; the generic kernel takes every other one.
+bool decode_fast_supported(int d, int G, int LK, int LV, int mode_k, int mode_v);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_generic(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d64_g1(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d64_g2(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d64_g4(const DecodeArgs& a, cudaStream_t stream);

@@ -114,8 +114,8 @@ typedef enum { KVQ_NORM_LIN8 = 0, KVQ_NORM_LOG4 = 1 } kvq_norm_mode;
                                      page 0 was read or written instead       */
 
 /* One codec: per layer and separately for K and V ("per-layer early-boost").
- * head_dim: power of two, 4..256 for encode/dequant; 64 or 128 for decode.
- * L: 2..65536 for encode/dequant; 2..256 for decode. */
+ * head_dim: power of two, 4..256.  L: 2..65536.  Every call takes every
+ * codec (decode: either norm mode for K and for V). */
 typedef struct {
     int32_t head_dim;
     int32_t L;
@@ -194,8 +194,12 @@ int kvq_encode_kv(const kvq_codec* kc, const int8_t* signs_k, const void* k,
                   const void* v, const kvq_plane* V, int32_t B, int32_t H_kv,
                   int32_t T, int64_t pos0, void* stream);
 
-/* Dequantize tokens pos0 .. pos0+T-1 of a plane back to fp16:
- *   y  device fp16 [B][H_kv][T][head_dim], 16-byte aligned (x^ above). */
+/* Dequantize tokens pos0 .. pos0+T-1 of a plane back to fp16: the
+ * reconstruction of the TurboAngle abstract's codec (each pair's norm from
+ * its norm code, its angle the centre of its bin, then the inverse of the
+ * random rotation), x^ = D H z^ / sqrt(d) as defined above.
+ *   y  device fp16 [B][H_kv][T][head_dim], 16-byte aligned, caller-owned.
+ * Arguments are checked as for kvq_encode; T == 0 is a no-op. */
 int kvq_dequant(const kvq_codec* codec, const int8_t* signs,
                 const kvq_plane* in, int32_t B, int32_t H_kv, int32_t T,
                 int64_t pos0, void* y, void* stream);
@@ -216,10 +220,14 @@ int64_t kvq_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t head_dim,
                                    int32_t num_splits);
 
 /* Split-K decode attention over the compressed cache, one layer, one new
- * query per sequence.
+ * query per sequence: attention scores read straight from the codes, never
+ * from a dequantized cache (TurboAngle abstract for the codec; the
+ * on-the-fly reconstruction principle of the OCTOPUS page, "TL;DR" and "Why
+ * it matters"), with the formulas of "Decode attention" above.
  *   q          device fp16 [B][H_q][head_dim]
- *   kc, vc     K and V codecs (same head_dim; kc LIN8, vc LOG4 in the
- *              kernels built here, other mode pairs return EUNSUPPORTED)
+ *   kc, vc     K and V codecs (same head_dim, any L and norm modes; head_dim
+ *              64/128, G 1/2/4/8, L <= 256 with LIN8 K and LOG4 V run in the
+ *              staged kernel, every other codec in the generic kernel)
  *   signs_k/v  device int8 [head_dim] diagonals used when K / V were encoded
  *   K, V       planes holding the cache; tokens 0 .. ctx_len[b]-1 are read
  *   ctx_len    device int32 [B]; values are clipped to [0, min(max_ctx,
@@ -261,7 +269,9 @@ int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc,
  * kvq_decode_attn.  The TurboAngle abstract encodes K and V on arrival and
  * attends from codes; doing both in one launch is this library's choice:
  * the split that holds the new token encodes it while its first tiles are
- * in flight, the other splits never wait for it.
+ * in flight, the other splits never wait for it.  (For codecs the staged
+ * kernel does not take, see kvq_decode_attn, the append is its own small
+ * launch just before the decode, with the same results.)
  *   k_new, v_new  device fp16 [B][H_kv][head_dim], 16-byte aligned
  * Everything else as for kvq_decode_attn.  A ctx_len outside the range
  * above appends nothing (and is clipped and reported as there). */

@@ -164,9 +164,6 @@ def _decode_rc(**kw):
 
 @pytest.mark.parametrize("kw,status,msg", [
     (dict(H_q=6, H_kv=4), kvq.KVQ_EINVAL, "multiple"),
-    (dict(H_q=32, H_kv=2), kvq.KVQ_EUNSUPPORTED, "no kernel"),
-    (dict(kc=(32, 128, 0), vc=(32, 64, 1)), kvq.KVQ_EUNSUPPORTED, "no kernel"),
-    (dict(kc=(128, 512, 0)), kvq.KVQ_EUNSUPPORTED, "no kernel"),
     (dict(vc=(64, 64, 1)), kvq.KVQ_EINVAL, "head_dim differ"),
     (dict(V=_plane(48)), kvq.KVQ_EINVAL, "capacity differ"),
     (dict(S=0), kvq.KVQ_EINVAL, "num_splits"),
@@ -179,6 +176,27 @@ def _decode_rc(**kw):
 def test_decode_rejects_bad_arguments(kw, status, msg):
     assert _decode_rc(**kw) == status
     assert msg in kvq.kvq_last_error()
+
+
+@pytest.mark.parametrize("kw", [
+    dict(H_q=32, H_kv=2),                          # G 16
+    dict(H_q=6, H_kv=2),                           # G 3
+    dict(kc=(4, 2, 0), vc=(4, 3, 1)),              # the smallest head
+    dict(kc=(32, 128, 0), vc=(32, 64, 1)),
+    dict(kc=(256, 65536, 1), vc=(256, 5000, 0)),   # log K norms, linear V norms
+    dict(kc=(128, 512, 0)),
+])
+def test_decode_accepts_every_codec(kw):
+    """Decode takes every codec encode takes (head_dim 4..256, any G, L up to
+    65536, either norm mode for K and V): the arguments pass every check and
+    the call reaches its launch (here made to fail on the host, so nothing
+    runs)."""
+    kvq.kvq_test_control(kvq.KVQ_TEST_FAIL_LAUNCHES, 1)
+    try:
+        assert _decode_rc(**kw) == kvq.KVQ_ECUDA
+        assert "injected" in kvq.kvq_last_error()
+    finally:
+        kvq.kvq_test_control(kvq.KVQ_TEST_RESET, 0)
 
 
 @pytest.mark.parametrize("k,v,msg", [

@@ -244,7 +244,8 @@ def test_dequant_sweep(dev, d, L):
 # ------------------------------------------------------------------ decode --
 
 def run_decode_case(B, H_q, H_kv, d, ctx_lens, LK, LV, seed=0, splits=None, cap=None,
-                    out_dtype=kvq.OUT_FP32, q_scale=1.0, tau=None):
+                    out_dtype=kvq.OUT_FP32, q_scale=1.0, tau=None, mode_k=O.MODE_LIN8,
+                    mode_v=O.MODE_LOG4):
     maxc = max(ctx_lens) if len(ctx_lens) else 0
     cap = cap or max(16, (maxc + 15) // 16 * 16)
     G = H_q // H_kv
@@ -252,10 +253,10 @@ def run_decode_case(B, H_q, H_kv, d, ctx_lens, LK, LV, seed=0, splits=None, cap=
     xk = _rand_x(B, H_kv, cap, d, seed=seed + 1)
     xv = _rand_x(B, H_kv, cap, d, seed=seed + 2, outliers=False)
     q = (np.random.default_rng(seed + 3).standard_normal((B, H_q, d)) * q_scale).astype(np.float16)
-    kc, vc = kvq.codec(d, LK, O.MODE_LIN8), kvq.codec(d, LV, O.MODE_LOG4)
+    kc, vc = kvq.codec(d, LK, mode_k), kvq.codec(d, LV, mode_v)
     Kp, Vp = kvq.alloc_plane(kc, B, H_kv, cap), kvq.alloc_plane(vc, B, H_kv, cap)
-    kcodes = O.encode(xk, sk, LK, O.MODE_LIN8)
-    vcodes = O.encode(xv, sv, LV, O.MODE_LOG4)
+    kcodes = O.encode(xk, sk, LK, mode_k)
+    vcodes = O.encode(xv, sv, LV, mode_v)
     for b in range(B):
         for h in range(H_kv):
             sl = slice((b * H_kv + h) * cap, (b * H_kv + h + 1) * cap)
@@ -291,6 +292,30 @@ def test_decode_gqa_sweep(dev, d, G):
     assert e.max() <= REL_L2_TOL, e.max()
 
 
+@pytest.mark.parametrize("d,G,LK,LV,mk,mv", [
+    (4, 1, 2, 3, O.MODE_LIN8, O.MODE_LOG4),        # the smallest head
+    (8, 3, 16, 16, O.MODE_LIN8, O.MODE_LOG4),      # G not a power of two
+    (16, 2, 128, 64, O.MODE_LOG4, O.MODE_LIN8),    # norm modes swapped
+    (32, 4, 1000, 24, O.MODE_LIN8, O.MODE_LOG4),
+    (64, 16, 128, 64, O.MODE_LIN8, O.MODE_LOG4),   # G 16: two head chunks
+    (128, 4, 512, 64, O.MODE_LIN8, O.MODE_LOG4),   # L past the staged kernel's 256
+    (128, 6, 65536, 5000, O.MODE_LOG4, O.MODE_LOG4),  # sincospif past the 4096 table
+    (256, 4, 128, 64, O.MODE_LIN8, O.MODE_LOG4),
+    (256, 1, 4096, 2, O.MODE_LIN8, O.MODE_LIN8),
+])
+def test_decode_every_codec(dev, d, G, LK, LV, mk, mv):
+    """Decode over codecs outside the staged kernel's set (the generic
+    kernel) against the oracle: ragged lengths, an empty sequence, two split
+    counts."""
+    H_kv = 2
+    for splits in (None, 3):
+        got, want, err = run_decode_case(4, G * H_kv, H_kv, d, [1, 77, 300, 0], LK, LV,
+                                         seed=d + G + LK, splits=splits, mode_k=mk, mode_v=mv)
+        assert err == 0
+        assert rel_l2(got, want)[:3].max() <= REL_L2_TOL, (splits, rel_l2(got, want))
+        assert np.all(got[3] == 0)
+
+
 @pytest.mark.parametrize("LK,LV", [(256, 256), (128, 64), (32, 5), (2, 2), (200, 33)])
 def test_decode_codebooks(dev, LK, LV):
     got, want, _ = run_decode_case(2, 8, 2, 128, [129, 64], LK, LV, seed=LK + LV)
@@ -309,24 +334,26 @@ def test_decode_split_invariance(dev):
         assert rel_l2(o, outs[0]).max() < 1e-5
 
 
-@pytest.mark.parametrize("ctx_lens,splits,H_kv,G", [
-    ([300, 129, 1, 0], None, 2, 4),   # ragged, a one-token sequence, an empty one
-    ([256, 128], 2, 2, 4),            # new token on the first row of a tile / of a split
-    ([257, 200], 3, 2, 4),
-    ([4096], None, 8, 4),             # the Llama-shaped layer
-    ([1000, 513], 1, 1, 8),           # one split: the held tile is not the first
+@pytest.mark.parametrize("ctx_lens,splits,H_kv,G,d,LK,LV", [
+    ([300, 129, 1, 0], None, 2, 4, 128, 128, 64),  # ragged, a one-token sequence, an empty one
+    ([256, 128], 2, 2, 4, 128, 128, 64),  # new token on the first row of a tile / of a split
+    ([257, 200], 3, 2, 4, 128, 128, 64),
+    ([4096], None, 8, 4, 128, 128, 64),   # the Llama-shaped layer
+    ([1000, 513], 1, 1, 8, 128, 128, 64),  # one split: the held tile is not the first
+    ([300, 129, 1, 0], 3, 2, 3, 256, 128, 64),  # the generic kernel (append launched first)
+    ([200, 64], None, 2, 4, 32, 512, 32),
 ])
-def test_decode_step_equals_append_then_decode(dev, ctx_lens, splits, H_kv, G):
+def test_decode_step_equals_append_then_decode(dev, ctx_lens, splits, H_kv, G, d, LK, LV):
     """kvq_decode_step writes the new token's codes exactly as kvq_encode_kv
     does and returns exactly what kvq_decode_attn returns on the appended
     cache; the appended cache also matches the oracle."""
-    d, B = 128, len(ctx_lens)
+    B = len(ctx_lens)
     H_q = G * H_kv
     cap = (max(ctx_lens) + 16 + 15) // 16 * 16
     sk, sv = _signs(31, d), _signs(32, d)
     k = _rand_x(B, H_kv, cap, d, seed=33)
     v = _rand_x(B, H_kv, cap, d, seed=34, outliers=False)
-    kc, vc = kvq.codec(d, 128, O.MODE_LIN8), kvq.codec(d, 64, O.MODE_LOG4)
+    kc, vc = kvq.codec(d, LK, O.MODE_LIN8), kvq.codec(d, LV, O.MODE_LOG4)
     skd, svd = _dev_signs(sk), _dev_signs(sv)
     kd, vd = torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda()
     # reference: every position encoded; step: the new positions blanked first
@@ -356,8 +383,8 @@ def test_decode_step_equals_append_then_decode(dev, ctx_lens, splits, H_kv, G):
         assert torch.equal(Ks.rows(w), Kr.rows(w)), ("K", w)
         assert torch.equal(Vs.rows(w), Vr.rows(w)), ("V", w)
     assert torch.equal(out_s, out_r)
-    compare_codes(plane_rows(Ks, t_range=(0, cap)), O.encode(k, sk, 128, O.MODE_LIN8))
-    compare_codes(plane_rows(Vs, t_range=(0, cap)), O.encode(v, sv, 64, O.MODE_LOG4))
+    compare_codes(plane_rows(Ks, t_range=(0, cap)), O.encode(k, sk, LK, O.MODE_LIN8))
+    compare_codes(plane_rows(Vs, t_range=(0, cap)), O.encode(v, sv, LV, O.MODE_LOG4))
 
 
 def test_decode_step_prepared_call_equals_call(dev):

@@ -80,3 +80,43 @@ def test_codec_error_matches_oracle_and_falls_with_L():
             e = np.linalg.norm(xh.reshape(-1, x.shape[-1]) - xd, axis=1) / np.linalg.norm(xd, axis=1)
             # the GPU rounds its dequantized vectors to fp16
             assert r[key] == pytest.approx(e.mean(), rel=2e-3, abs=2e-4), (key, r["L_K"])
+
+
+def test_bits_per_element_other_norm_modes():
+    """4-bit log K norms (and 8-bit linear V norms) count 4 (8) bits per pair
+    and carry their own fp16 parameters: LOG4 two per vector, LIN8 one."""
+    lin, log = kvq.KVQ_NORM_LIN8, kvq.KVQ_NORM_LOG4
+    b = quality.bits_per_element(128, 128, 64, log, log)
+    assert b["norms"] == pytest.approx((4 + 4) / 4)
+    assert b["params"] == pytest.approx((32 + 32) / 256)
+    assert b["stored"] == pytest.approx(b["total"])
+    b = quality.bits_per_element(64, 128, 64, log, lin)
+    assert b["norms"] == pytest.approx((4 + 8) / 4)
+    assert b["params"] == pytest.approx((32 + 16) / 128)
+    assert b["stored"] == pytest.approx(b["total"])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mk,mv", [(kvq.KVQ_NORM_LOG4, kvq.KVQ_NORM_LOG4),
+                                   (kvq.KVQ_NORM_LOG4, kvq.KVQ_NORM_LIN8)])
+def test_norm_mode_sweep_matches_oracle(mk, mv):
+    """The other norm pairings, at a codebook past 256: the tool's
+    dequantization errors equal the oracle's, and the attention error (the
+    decode kernels now take every codec) is reported."""
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    import oracle as O
+    from decode_attention_rand_b200 import build as kbuild
+    kbuild.build()
+    w = synth.WORKLOADS["tiny_b1_hq4_hkv2_d128_ctx256"]
+    r = quality.codec_error(w, 0, 1024, 1024, mode_k=mk, mode_v=mv)
+    assert r["attn_rel_l2_mean"] is not None and r["attn_rel_l2_mean"] < 0.5
+    sk, sv = synth.layer_signs(w, 0)
+    k = synth.kv(w, 0, synth.KIND_K, device="cuda").cpu().numpy()
+    v = synth.kv(w, 0, synth.KIND_V, device="cuda").cpu().numpy()
+    for x, s, mode, key in ((k, sk, mk, "k_rel_l2_mean"), (v, sv, mv, "v_rel_l2_mean")):
+        xh = O.dequant(O.encode(x, s, 1024, mode), s).reshape(x.shape)
+        xd = x.astype(np.float64).reshape(-1, x.shape[-1])
+        e = np.linalg.norm(xh.reshape(-1, x.shape[-1]) - xd, axis=1) / np.linalg.norm(xd, axis=1)
+        assert r[key] == pytest.approx(e.mean(), rel=2e-3, abs=2e-4), key
