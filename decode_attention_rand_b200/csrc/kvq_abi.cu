@@ -143,7 +143,9 @@ int kvq_test_control(int32_t key, int64_t value) {
         case KVQ_TEST_RESET:
             g_fail_launches.store(0);
             g_wait_limit_p1.store(0);
+            kvq::set_debug_checks(-1);
             return ok();
+        case KVQ_TEST_DEBUG_CHECKS: kvq::set_debug_checks(value ? 1 : 0); return ok();
         case KVQ_TEST_FAIL_LAUNCHES: g_fail_launches.store(value); return ok();
         case KVQ_TEST_WAIT_LIMIT:
             g_wait_limit_p1.store((value < 0xFFFFFFFFll ? value : 0xFFFFFFFFll - 1) + 1);
@@ -224,6 +226,7 @@ int kvq_encode(const kvq_codec* codec, const int8_t* signs, const void* x, int32
     if (rc) return rc;
     if (j.n_vec == 0) return ok();
     if (injected_failure()) return injected("kvq_encode");
+    kvq::ProfileRange range("kvq_encode");
     return cuda_status(kvq::launch_encode_jobs(&j, 1, sm_count_current(),
                                                static_cast<cudaStream_t>(stream)),
                        "kvq_encode");
@@ -242,6 +245,7 @@ int kvq_encode_kv(const kvq_codec* kc, const int8_t* signs_k, const void* k, con
                     j[0].c.d, j[1].c.d);
     if (j[0].n_vec == 0) return ok();
     if (injected_failure()) return injected("kvq_encode_kv");
+    kvq::ProfileRange range("kvq_encode_kv");
     return cuda_status(kvq::launch_encode_jobs(j, 2, sm_count_current(),
                                                static_cast<cudaStream_t>(stream)),
                        "kvq_encode_kv");
@@ -264,6 +268,7 @@ int kvq_encode_kv_paged(const kvq_codec* kc, const int8_t* signs_k, const void* 
     if (j[0].n_vec == 0) return ok();
     j[0].err_word = j[1].err_word = err_word;
     if (injected_failure()) return injected("kvq_encode_kv_paged");
+    kvq::ProfileRange range("kvq_encode_kv_paged");
     return cuda_status(kvq::launch_encode_jobs(j, 2, sm_count_current(),
                                                static_cast<cudaStream_t>(stream)),
                        "kvq_encode_kv_paged");
@@ -286,6 +291,7 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs, const kvq_plane* in
     if (!signs || !y) return fail(KVQ_EINVAL, "kvq_dequant: NULL signs or y");
     if (!aligned16(y)) return fail(KVQ_EINVAL, "kvq_dequant: y must be 16-byte aligned");
     if (injected_failure()) return injected("kvq_dequant");
+    kvq::ProfileRange range("kvq_dequant");
     return cuda_status(kvq::launch_dequant(c, signs, p, n, T, pos0, static_cast<__half*>(y),
                                            sm_count_current(), static_cast<cudaStream_t>(stream)),
                        "kvq_dequant");
@@ -414,10 +420,15 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
     a.wait_limit = wl > 0 ? (uint32_t)(wl - 1) : kvq::kWaitLimit;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (injected_failure()) return injected(what);
+    kvq::ProfileRange range(what);
     int rc2;
     if (hio && hio->in_bytes > 0) {
         rc2 = cuda_status(cudaMemcpyAsync(const_cast<void*>(q), hio->in_host, (size_t)hio->in_bytes,
                                           cudaMemcpyHostToDevice, st), what);
+        if (rc2) return rc2;
+    }
+    if (kvq::debug_checks_on()) {
+        rc2 = cuda_status(kvq::launch_cache_check(a, st), what);
         if (rc2) return rc2;
     }
     rc2 = cuda_status(kvq::launch_decode(a, st), what);

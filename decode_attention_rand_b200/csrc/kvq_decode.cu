@@ -4,7 +4,22 @@
 // (kvq_decode_generic.cu) for every other codec.
 #include "kvq_internal.h"
 
+#include <atomic>
+
 namespace kvq {
+
+int device_sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = cache[dev].load();
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            return 148;
+        cache[dev].store(n);
+    }
+    return n;
+}
 
 bool decode_fast_supported(int d, int G, int LK, int LV, int mode_k, int mode_v) {
     if (d != 64 && d != 128) return false;

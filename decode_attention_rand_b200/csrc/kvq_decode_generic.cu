@@ -369,6 +369,20 @@ __global__ void __launch_bounds__(64) append_kernel(DecodeArgs A) {
 }
 
 template <int D>
+cudaError_t launch_append_d(const DecodeArgs& a, cudaStream_t stream) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)a.H_kv, (unsigned)a.B, 1);
+    cfg.blockDim = dim3(64);
+    return cudaLaunchKernelEx(&cfg, append_kernel<D>, a);
+}
+
+template <int D>
 cudaError_t launch_generic_d(const DecodeArgs& a, cudaStream_t stream) {
     using Cfg = GenCfg<D>;
     const int G = a.H_q / a.H_kv;
@@ -391,10 +405,7 @@ cudaError_t launch_generic_d(const DecodeArgs& a, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (a.k_new) {
-        cfg.gridDim = dim3((unsigned)a.H_kv, (unsigned)a.B, 1);
-        cfg.blockDim = dim3(64);
-        cfg.dynamicSmemBytes = 0;
-        e = cudaLaunchKernelEx(&cfg, append_kernel<D>, a);
+        e = launch_append_d<D>(a, stream);
         if (e != cudaSuccess) return e;
     }
     cfg.gridDim = dim3((unsigned)a.num_splits, (unsigned)(a.H_kv * chunks), (unsigned)a.B);
@@ -406,6 +417,19 @@ cudaError_t launch_generic_d(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t launch_append(const DecodeArgs& a, cudaStream_t stream) {
+    switch (a.kc.d) {
+        case 4: return launch_append_d<4>(a, stream);
+        case 8: return launch_append_d<8>(a, stream);
+        case 16: return launch_append_d<16>(a, stream);
+        case 32: return launch_append_d<32>(a, stream);
+        case 64: return launch_append_d<64>(a, stream);
+        case 128: return launch_append_d<128>(a, stream);
+        case 256: return launch_append_d<256>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_decode_generic(const DecodeArgs& a, cudaStream_t stream) {
     switch (a.kc.d) {

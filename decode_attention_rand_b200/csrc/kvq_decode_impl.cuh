@@ -70,10 +70,15 @@ constexpr bool decode_static_tables(int bk, int bv) {
     return bk > 0 && bv > 0 && ((1 << bk) + (1 << bv)) * kTabRep * 8 <= 48 * 1024;
 }
 
-template <int D, int G>
+// CTAS: resident CTAs per SM the instance is built for.  With one, a lane
+// owns 32 / G pairs (at most 16) of each token; with two, half as many (at
+// least 4), which halves its query and accumulator registers (4 G PP of
+// them) so that two 8-warp CTAs fit beside each other on an SM.
+template <int D, int G, int CTAS = 1>
 struct DecCfg {
     static constexpr int P = D / 2;
-    static constexpr int PP = (32 / G) > 16 ? 16 : (32 / G);  // pairs per lane
+    static constexpr int PP_MAX = CTAS == 1 ? 32 / G : (16 / G < 4 ? 4 : 16 / G);
+    static constexpr int PP = PP_MAX > 16 ? 16 : PP_MAX;        // pairs per lane
     static constexpr int NL = P / PP;                          // lanes per token group
     static constexpr int GPW = 32 / NL;                        // groups per warp
     static constexpr int TW = GPW * kTPG;                      // tokens per warp block
@@ -229,34 +234,79 @@ __device__ __forceinline__ void xor_reduce(float (&v)[V]) {
     }
 }
 
-// Byte offsets (entry * 128 + lane16 * 8) into a 16x replicated float2
-// table for the PP angle codes of this lane: bits [cb, cb + PP*B) of a row.
-// B > 0: compile-time width; B == 0: runtime width `bits`.
+// Loads from the shared window at a 32-bit address (smem_u32); volatile, so
+// that they stay behind the mbarrier wait that made the staged bytes valid.
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint2 lds_u64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint4 lds_u128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1+%2];" : "=h"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u8 %0, [%1+%2];" : "=h"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+__device__ __forceinline__ float2 lds_f2(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ float4 lds_f4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(a), "n"(OFF));
+    return v;
+}
+
+// Shared addresses of the 16x replicated float2 table entries of this lane's
+// PP angle codes: table + lane16 * 8 + code * 128, the codes being bits
+// [cb, cb + PP*B) of the row at shared address `row` (wa = its first word:
+// the row address plus 4 (cb >> 5); sh = cb & 31).  B > 0: compile-time
+// width; B == 0: runtime width `bits`.
 template <int PP, int B>
-__device__ __forceinline__ void angle_offsets(const uint32_t* row, int cb, int bits,
-                                              uint32_t lane_off, uint32_t (&off)[PP]) {
+__device__ __forceinline__ void angle_addrs(uint32_t wa, int sh, int bits, uint32_t tab_lane,
+                                            uint32_t (&off)[PP]) {
     if constexpr (B > 0) {
         constexpr int NB = PP * B;             // chunk bits
         constexpr int NW = (NB + 31) / 32;     // normalised words
         constexpr uint32_t mask = ((1u << B) - 1u) << kTabShift;
+        uint32_t w[NW + 2];
+        w[0] = lds_u32<0>(wa);
+        if constexpr (NW >= 1) w[1] = lds_u32<4>(wa);
+        if constexpr (NW >= 2) w[2] = lds_u32<8>(wa);
+        if constexpr (NW >= 3) w[3] = lds_u32<12>(wa);
+        if constexpr (NW >= 4) w[4] = lds_u32<16>(wa);
+        static_assert(NW <= 4, "at most 128 code bits per lane");
         uint32_t n[NW + 1];
-        const int w0 = cb >> 5;
-        if constexpr (NB % 32 == 0) {
 #pragma unroll
-            for (int i = 0; i < NW; i++) n[i] = row[w0 + i];
-        } else {
-            const int sh = cb & 31;
-            uint32_t w[NW + 1];
-#pragma unroll
-            for (int i = 0; i <= NW; i++) w[i] = row[w0 + i];
-#pragma unroll
-            for (int i = 0; i < NW; i++) n[i] = __funnelshift_r(w[i], w[i + 1], sh);
-        }
+        for (int i = 0; i < NW; i++) n[i] = __funnelshift_r(w[i], w[i + 1], sh);
         n[NW] = 0u;
 #pragma unroll
         for (int k = 0; k < PP; k++) {
-            constexpr int dummy = 0;
-            (void)dummy;
             const int pos = k * B;             // compile-time after unrolling
             const int wi = pos >> 5, bi = pos & 31;
             uint32_t x;
@@ -265,41 +315,45 @@ __device__ __forceinline__ void angle_offsets(const uint32_t* row, int cb, int b
             } else {
                 x = __funnelshift_r(n[wi], n[wi + 1], bi - kTabShift);
             }
-            off[k] = (x & mask) | lane_off;
+            off[k] = (x & mask) + tab_lane;
         }
     } else {
         const uint32_t mask = (1u << bits) - 1u;
 #pragma unroll
         for (int q = 0; q < PP / 4; q++) {
-            const int pos = cb + q * 4 * bits;
-            const uint32_t win = __funnelshift_r(row[pos >> 5], row[(pos >> 5) + 1], pos & 31);
+            const int pos = sh + q * 4 * bits;  // from the first word of the lane
+            const uint32_t a = wa + 4u * (uint32_t)(pos >> 5);
+            const uint32_t win = __funnelshift_r(lds_u32<0>(a), lds_u32<4>(a), pos & 31);
 #pragma unroll
             for (int k = 0; k < 4; k++)
-                off[4 * q + k] = (((win >> (k * bits)) & mask) << kTabShift) | lane_off;
+                off[4 * q + k] = (((win >> (k * bits)) & mask) << kTabShift) + tab_lane;
         }
     }
 }
 
+// NBYTES bytes (1, 2, 4, 8, 16) at shared address a as little-endian words.
 template <int NBYTES>
-__device__ __forceinline__ void load_bytes(const uint8_t* p, uint32_t (&w)[(NBYTES + 3) / 4]) {
+__device__ __forceinline__ void lds_bytes(uint32_t a, uint32_t (&w)[(NBYTES + 3) / 4]) {
     if constexpr (NBYTES == 16) {
-        const uint4 q = *reinterpret_cast<const uint4*>(p);
+        const uint4 q = lds_u128(a);
         w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
     } else if constexpr (NBYTES == 8) {
-        const uint2 q = *reinterpret_cast<const uint2*>(p);
+        const uint2 q = lds_u64(a);
         w[0] = q.x; w[1] = q.y;
     } else if constexpr (NBYTES == 4) {
-        w[0] = *reinterpret_cast<const uint32_t*>(p);
+        w[0] = lds_u32(a);
+    } else if constexpr (NBYTES == 2) {
+        w[0] = lds_u16(a);
     } else {
-        w[0] = *reinterpret_cast<const uint16_t*>(p);
+        static_assert(NBYTES == 1, "1, 2, 4, 8 or 16 bytes");
+        w[0] = lds_u8(a);
     }
 }
 
-
 // ------------------------------------------------------------- kernel ---
 
-template <int D, int G, int BK, int BV>
-__global__ void __launch_bounds__(DecCfg<D, G>::THREADS, 1)
+template <int D, int G, int BK, int BV, int CTAS>
+__global__ void __launch_bounds__(DecCfg<D, G, CTAS>::THREADS, CTAS)
 decode_kernel(DecodeArgs A) {
     // A kernel launched after this one as its programmatic dependent (the
     // next layer's or step's decode) may start its setup once every CTA here
@@ -307,7 +361,7 @@ decode_kernel(DecodeArgs A) {
     // which returns only when this grid has completed and its writes are
     // visible, so it overlaps its barrier setup and tables with this tail.
     asm volatile("griddepcontrol.launch_dependents;");
-    using Cfg = DecCfg<D, G>;
+    using Cfg = DecCfg<D, G, CTAS>;
     constexpr int P = Cfg::P, PP = Cfg::PP, NL = Cfg::NL, GPW = Cfg::GPW, NG = Cfg::NG;
     constexpr int WARPS = Cfg::WARPS, TW = Cfg::TW;
     constexpr int V = Cfg::V, VF = Cfg::VF;
@@ -398,7 +452,9 @@ decode_kernel(DecodeArgs A) {
     // the tables and rotate q; the tile holding it, and the ones after, are
     // copied in only after it is written.  Without an append all warps share
     // the tables and q.
-    const bool fused = A.k_new != nullptr;
+    // the two-CTA instance carries no append code (its registers would not
+    // fit); its kvq_decode_step runs the append as a launch of its own first
+    const bool fused = CTAS == 1 && A.k_new != nullptr;
     const int w0 = fused ? 2 : 0;  // first warp of the table / q' work
     int64_t ctx_in = 0;
     bool append = false;           // warps 0 and 1 of a fused launch
@@ -413,7 +469,7 @@ decode_kernel(DecodeArgs A) {
         for (; issued < NST - 1 && issued < ntiles_max && issued < hold; issued++) issue_tile(issued);
     }
     if (fused && warp < 2) {
-        if (append) {
+        if constexpr (CTAS == 1) if (append) {
             // the same encode_tile as kvq_encode, one vector per warp
             using ECfg = EncCfg<D>;
             EncArgs E = warp == 0 ? A.enc_k : A.enc_v;
@@ -543,10 +599,15 @@ decode_kernel(DecodeArgs A) {
             }
         const int bitsK = BK > 0 ? BK : A.kc.bits, bitsV = BV > 0 ? BV : A.vc.bits;
         const int cbK = lg * PP * bitsK, cbV = lg * PP * bitsV;
+        // all staged data is addressed by 32-bit shared-window offsets; row
+        // strides are compile-time constants for the fixed code widths
+        const int rbK = 4 * (BK > 0 ? (P * BK + 31) / 32 : A.kc.angle_words);
+        const int rbV = 4 * (BV > 0 ? (P * BV + 31) / 32 : A.vc.angle_words);
         const uint32_t lane_off = (uint32_t)(lane & 15) * 8u;
-        const unsigned char* tKb = reinterpret_cast<const unsigned char*>(tabK);
-        const unsigned char* tVb = reinterpret_cast<const unsigned char*>(tabV);
-        const int awK = A.kc.angle_words, awV = A.vc.angle_words;
+        const uint32_t tKl = smem_u32(tabK) + lane_off, tVl = smem_u32(tabV) + lane_off;
+        const uint32_t wK = 4u * (uint32_t)(cbK >> 5), wV = 4u * (uint32_t)(cbV >> 5);
+        const int shK = cbK & 31, shV = cbV & 31;
+        const uint32_t stages32 = smem_u32(stages);
 
         for (int tile = 0; tile < nloop; tile++) {
             const int s = tile % NST;
@@ -556,13 +617,11 @@ decode_kernel(DecodeArgs A) {
                 break;
             }
             if (__any_sync(KVQ_FULL_MASK, *((volatile int*)&sflag[0]) != 0)) break;
-            const unsigned char* st = stages + (size_t)s * A.stage_bytes;
-            const uint32_t* sKa = reinterpret_cast<const uint32_t*>(st + A.lay[0]);
-            const uint8_t* sKn = st + A.lay[1];
-            const uint16_t* sKp = reinterpret_cast<const uint16_t*>(st + A.lay[2]);
-            const uint32_t* sVa = reinterpret_cast<const uint32_t*>(st + A.lay[3]);
-            const uint8_t* sVn = st + A.lay[4];
-            const uint32_t* sVp = reinterpret_cast<const uint32_t*>(st + A.lay[5]);
+            const uint32_t st = stages32 + (uint32_t)(s * A.stage_bytes);
+            const uint32_t sKa = st + A.lay[0] + wK, sKn = st + A.lay[1] + lg * PP;
+            const uint32_t sKp = st + A.lay[2];
+            const uint32_t sVa = st + A.lay[3] + wV, sVn = st + A.lay[4] + lg * (PP / 2);
+            const uint32_t sVp = st + A.lay[5];
             const int64_t tt0 = t0 + (int64_t)tile * kTT;
             const int ntok = (int)((t1 - tt0) < kTT ? (t1 - tt0) : kTT);
 
@@ -574,9 +633,9 @@ decode_kernel(DecodeArgs A) {
                 for (int j = 0; j < kTPG; j++) {
                     const int t = blk * TW + (j ^ JX) * GPW + grp;
                     uint32_t off[PP];
-                    angle_offsets<PP, BK>(sKa + t * awK, cbK, bitsK, lane_off, off);
+                    angle_addrs<PP, BK>(sKa + (uint32_t)(t * rbK), shK, bitsK, tKl, off);
                     uint32_t nw[(PP + 3) / 4];
-                    load_bytes<PP>(sKn + t * P + lg * PP, nw);
+                    lds_bytes<PP>(sKn + (uint32_t)(t * P), nw);
                     f32x2 dot[G];
 #pragma unroll
                     for (int h = 0; h < G; h++) dot[h] = 0ull;
@@ -587,7 +646,7 @@ decode_kernel(DecodeArgs A) {
                         // fma(f, U, -U) = (f - 1) U = c (cos, sin), rounded once
                         const float f = __uint_as_float(
                             __byte_perm(nw[k / 4], 0x3F800000u, 0x7604u | ((k % 4) << 4)));
-                        const float2 U = *reinterpret_cast<const float2*>(tKb + off[k]);
+                        const float2 U = lds_f2(off[k]);
                         const f32x2 xy = pack2(fmaf(f, U.x, -U.x), fmaf(f, U.y, -U.y));
 #pragma unroll
                         for (int h = 0; h < G; h++) dot[h] = fma2(q2[h][k], xy, dot[h]);
@@ -601,7 +660,7 @@ decode_kernel(DecodeArgs A) {
 #pragma unroll
                 for (int e = 0; e < VF; e++) {
                     const int t = blk * TW + ((M + e) / G) * GPW + grp;
-                    const float Mk = half_bits_to_float(sKp[t]);
+                    const float Mk = half_bits_to_float((uint16_t)lds_u16(sKp + 2u * (uint32_t)t));
                     float sv = part[e] * (Mk * (1.f / 255.f)) * A.scale_log2;
                     sv = t < ntok ? sv : -INFINITY;
                     part[e] = sv;
@@ -669,10 +728,10 @@ decode_kernel(DecodeArgs A) {
                         }
                     }
                     uint32_t off[PP];
-                    angle_offsets<PP, BV>(sVa + t * awV, cbV, bitsV, lane_off, off);
+                    angle_addrs<PP, BV>(sVa + (uint32_t)(t * rbV), shV, bitsV, tVl, off);
                     uint32_t nw[(PP / 2 + 3) / 4];
-                    load_bytes<PP / 2>(sVn + t * (P / 2) + lg * (PP / 2), nw);
-                    const uint32_t pr = sVp[t];
+                    lds_bytes<PP / 2>(sVn + (uint32_t)(t * (P / 2)), nw);
+                    const uint32_t pr = lds_u32(sVp + 4u * (uint32_t)t);
                     const float LO = half_bits_to_float((uint16_t)(pr & 0xFFFF));
                     // log2 r^ = LO + c (HI - LO)/15 = f A + B with f = 1 + c/16,
                     // A = 16 (HI - LO)/15, B = LO - A
@@ -690,7 +749,7 @@ decode_kernel(DecodeArgs A) {
                         const uint32_t mant = sh <= 19 ? (w << (19 - sh)) : (w >> (sh - 19));
                         const float f = __uint_as_float((mant & 0x00780000u) | 0x3F800000u);
                         const float r = ex2(fmaf(f, A16, B16));
-                        const float2 cs = *reinterpret_cast<const float2*>(tVb + off[k]);
+                        const float2 cs = lds_f2(off[k]);
                         const f32x2 xy = pack2(r * cs.x, r * cs.y);
 #pragma unroll
                         for (int h = 0; h < G; h++) acc[h][k] = fma2(pw[h], xy, acc[h][k]);
@@ -971,9 +1030,9 @@ decode_kernel(DecodeArgs A) {
 // Shared-memory plan of one launch (ring depth 4, 3 or 2, whichever fits in
 // `avail` bytes of dynamic shared memory); returns 0 bytes when even two
 // stages do not fit.
-template <int D, int G, int BK, int BV>
+template <int D, int G, int BK, int BV, int CTAS>
 inline size_t decode_smem_plan(DecodeArgs& a, size_t avail) {
-    using Cfg = DecCfg<D, G>;
+    using Cfg = DecCfg<D, G, CTAS>;
     size_t off = 16 * kMaxStages + 16;
     if (!decode_static_tables(BK, BV))
         off += sizeof(float2) * kTabRep * (size_t)((1 << a.kc.bits) + (1 << a.vc.bits));
@@ -1026,10 +1085,10 @@ struct DecodeLaunchCache {
     int n_entries = 0;
 };
 
-template <int D, int G, int BK, int BV>
+template <int D, int G, int BK, int BV, int CTAS>
 inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
-    using Cfg = DecCfg<D, G>;
-    auto kernel = decode_kernel<D, G, BK, BV>;
+    using Cfg = DecCfg<D, G, CTAS>;
+    auto kernel = decode_kernel<D, G, BK, BV, CTAS>;
     static DecodeLaunchCache cache;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1043,7 +1102,10 @@ inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
             cudaFuncAttributes fa;
             e = cudaFuncGetAttributes(&fa, kernel);
             if (e != cudaSuccess) return e;
-            const size_t dyn = 227 * 1024 - fa.sharedSizeBytes;
+            // per CTA: 227 KB, or half the SM's 228 KB less the 1 KB the
+            // system reserves per CTA when two share the SM
+            const size_t dyn = (CTAS == 1 ? 227 * 1024 : 228 * 1024 / 2 - 1024) -
+                               fa.sharedSizeBytes;
             e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
             if (e != cudaSuccess) return e;
             e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -1058,7 +1120,7 @@ inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
         avail = cache.avail[dev];
         sm_count = cache.sm_count[dev];
     }
-    const size_t smem = decode_smem_plan<D, G, BK, BV>(a, avail);
+    const size_t smem = decode_smem_plan<D, G, BK, BV, CTAS>(a, avail);
     if (smem == 0) return cudaErrorInvalidConfiguration;
     dim3 grid((unsigned)a.num_splits, (unsigned)a.H_kv, (unsigned)a.B);
     cudaLaunchConfig_t cfg = {};
@@ -1109,19 +1171,48 @@ inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// The append of kvq_decode_step as its own launch (kvq_decode_generic.cu),
+// for the instances that carry no append code.
+cudaError_t launch_append(const DecodeArgs& a, cudaStream_t stream);
+
+// The two-CTA instance of fixed widths (bk, bv): for G up to 4 with codes of
+// 5..7 bits (its tables then fit in static shared memory beside a ring of
+// tiles in half an SM), when the launch needs more than one wave of one-CTA
+// launches (a single wave is latency-bound and keeps the fused append).
+inline bool decode_two_ctas(const DecodeArgs& a, int G, int sm_count) {
+    return G <= 4 && a.kc.bits >= 5 && a.kc.bits <= 7 && a.vc.bits >= 5 && a.vc.bits <= 7 &&
+           (int64_t)a.B * a.H_kv * a.num_splits > (int64_t)sm_count;
+}
+
 // Fast kernels for code widths 5..8 (codebooks of 17..256 entries), the
 // runtime-width kernel for anything else.
 template <int D, int G>
 inline cudaError_t launch_decode_dg(const DecodeArgs& a, cudaStream_t stream) {
     const int bk = a.kc.bits, bv = a.vc.bits;
+    if constexpr (G <= 4) {
+        if (decode_two_ctas(a, G, device_sm_count())) {
+            DecodeArgs b = a;
+            if (a.k_new) {
+                const cudaError_t e = launch_append(a, stream);
+                if (e != cudaSuccess) return e;
+                b.k_new = b.v_new = nullptr;
+            }
+#define KVQ_BB2(X, Y) \
+    if (bk == X && bv == Y) return launch_decode_kernel<D, G, X, Y, 2>(b, stream);
+            KVQ_BB2(5, 5) KVQ_BB2(5, 6) KVQ_BB2(5, 7)
+            KVQ_BB2(6, 5) KVQ_BB2(6, 6) KVQ_BB2(6, 7)
+            KVQ_BB2(7, 5) KVQ_BB2(7, 6) KVQ_BB2(7, 7)
+#undef KVQ_BB2
+        }
+    }
 #define KVQ_BB(X, Y) \
-    if (bk == X && bv == Y) return launch_decode_kernel<D, G, X, Y>(a, stream);
+    if (bk == X && bv == Y) return launch_decode_kernel<D, G, X, Y, 1>(a, stream);
     KVQ_BB(5, 5) KVQ_BB(5, 6) KVQ_BB(5, 7) KVQ_BB(5, 8)
     KVQ_BB(6, 5) KVQ_BB(6, 6) KVQ_BB(6, 7) KVQ_BB(6, 8)
     KVQ_BB(7, 5) KVQ_BB(7, 6) KVQ_BB(7, 7) KVQ_BB(7, 8)
     KVQ_BB(8, 5) KVQ_BB(8, 6) KVQ_BB(8, 7) KVQ_BB(8, 8)
 #undef KVQ_BB
-    return launch_decode_kernel<D, G, 0, 0>(a, stream);
+    return launch_decode_kernel<D, G, 0, 0, 1>(a, stream);
 }
 
 }  // namespace kvq

@@ -97,6 +97,23 @@ cudaError_t launch_decode_d128_g2(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d128_g4(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d128_g8(const DecodeArgs& a, cudaStream_t stream);
 
+// KVQ_DEBUG cache integrity check (kvq_debug.cu): on when the environment
+// variable is set (or by kvq_test_control); launched before each decode.
+bool debug_checks_on();
+void set_debug_checks(int on);  // 1 on, 0 off, -1 back to the environment
+cudaError_t launch_cache_check(const DecodeArgs& a, cudaStream_t stream);
+
+// KVQ_PROFILE: an NVTX range around each call's launches when the environment
+// variable is set.
+struct ProfileRange {
+    bool on;
+    explicit ProfileRange(const char* name);
+    ~ProfileRange();
+};
+
+// SM count of the current device (cached per device; 148 if unknown).
+int device_sm_count();
+
 // Default number of tries of a bounded mbarrier wait.
 constexpr uint32_t kWaitLimit = 1u << 22;
 

@@ -26,7 +26,8 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "kvq.h")
 KVQ_OK, KVQ_EINVAL, KVQ_EUNSUPPORTED, KVQ_ECUDA, KVQ_ETIMEOUT = 0, -1, -2, -3, -4
 KVQ_NORM_LIN8, KVQ_NORM_LOG4 = 0, 1
 KVQ_DEVERR_CTX_RANGE, KVQ_DEVERR_TIMEOUT, KVQ_DEVERR_PAGE_RANGE = 0x1, 0x2, 0x4
-KVQ_TEST_RESET, KVQ_TEST_FAIL_LAUNCHES, KVQ_TEST_WAIT_LIMIT = 0, 1, 2
+KVQ_DEVERR_BAD_CODE = 0x8
+KVQ_TEST_RESET, KVQ_TEST_FAIL_LAUNCHES, KVQ_TEST_WAIT_LIMIT, KVQ_TEST_DEBUG_CHECKS = 0, 1, 2, 3
 OUT_FP16, OUT_FP32 = 0, 1
 
 

@@ -86,6 +86,13 @@
  *   out) are OR-ed into *err_word (KVQ_DEVERR_* bits) when err_word is not
  *   NULL; the kernels never trap.
  * Inputs must be finite; NaN or Inf inputs give unspecified codes.
+ *
+ * Environment: KVQ_DEBUG (set, not "0") makes every decode call first check
+ * the cache rows it reads (tokens 0 .. ctx_len[b]-1) for values the encoder
+ * never writes and report them as KVQ_DEVERR_BAD_CODE in err_word; it costs a
+ * second read of the cache and is meant for debugging.  KVQ_PROFILE (set, not
+ * "0") brackets the launches of every call with an NVTX range named after the
+ * call, for profilers.  Both are read once, at the first call.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -112,6 +119,10 @@ typedef enum { KVQ_NORM_LIN8 = 0, KVQ_NORM_LOG4 = 1 } kvq_norm_mode;
 #define KVQ_DEVERR_TIMEOUT 0x2    /* an mbarrier wait hit its iteration cap  */
 #define KVQ_DEVERR_PAGE_RANGE 0x4 /* a page-table entry outside [0, num_pages):
                                      page 0 was read or written instead       */
+#define KVQ_DEVERR_BAD_CODE 0x8   /* KVQ_DEBUG checks: a cache row holds a value
+                                     the encoder never writes (an angle code
+                                     >= L, a non-finite fp16 parameter, LOG4
+                                     HI < LO, LIN8 M < 0)                    */
 
 /* One codec: per layer and separately for K and V ("per-layer early-boost").
  * head_dim: power of two, 4..256.  L: 2..65536.  Every call takes every
@@ -384,10 +395,14 @@ int kvq_decode_attn_noalloc(const void* q, const kvq_codec* kc,
  *                           a CTA contributes nothing to the output.  Copies
  *                           already issued are still waited for, with the
  *                           default limit of 2^22 tries, before a CTA exits.
+ *   KVQ_TEST_DEBUG_CHECKS   value 1 / 0: the KVQ_DEBUG checks on / off for
+ *                           the rest of the process, whatever the environment
+ *                           says (KVQ_TEST_RESET returns to the environment)
  * Returns KVQ_OK, or KVQ_EINVAL for an unknown key or a negative value. */
 #define KVQ_TEST_RESET 0
 #define KVQ_TEST_FAIL_LAUNCHES 1
 #define KVQ_TEST_WAIT_LIMIT 2
+#define KVQ_TEST_DEBUG_CHECKS 3
 int kvq_test_control(int32_t key, int64_t value);
 
 /* Message for the last non-OK status returned on the calling thread

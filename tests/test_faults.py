@@ -173,3 +173,76 @@ def test_injected_failure_queues_nothing_and_library_recovers(dev, controls):
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
     assert math.isfinite(float(out.abs().max()))
+
+
+def test_profile_ranges_do_not_change_results_on_host():
+    """KVQ_PROFILE brackets each call's launches with an NVTX range; a call
+    made with it set (in a fresh process, where it is read) returns what it
+    returns without it (here: the argument errors and the launch outcome on a
+    machine without a GPU are unchanged)."""
+    import subprocess
+    import sys
+    code = (
+        "import ctypes as C; from decode_attention_rand_b200 import kvq\n"
+        "kc, vc = kvq.codec(128, 128, 0), kvq.codec(128, 64, 1)\n"
+        f"K = kvq.kvq_plane({FAKE}, {FAKE}, {FAKE}, 256)\n"
+        f"rc = kvq.lib().kvq_encode(C.byref(kc), {FAKE}, {FAKE}, 1, 2, 10, 250, C.byref(K), None)\n"
+        "print(rc, kvq.kvq_last_error())\n"
+    )
+    outs = []
+    for env in ({"KVQ_PROFILE": "1"}, {"KVQ_PROFILE": "0"}):
+        import os
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                           env={**os.environ, **env}, timeout=300,
+                           cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+        assert r.returncode == 0, r.stderr[-2000:]
+        outs.append(r.stdout.strip())
+    assert outs[0] == outs[1] and outs[0].startswith(str(kvq.KVQ_EINVAL))
+
+
+@pytest.mark.gpu
+def test_debug_checks_report_corrupted_rows(dev, controls):
+    """With the KVQ_DEBUG checks on, a clean cache reports nothing; a NaN
+    parameter (the streaming encoder's in-doubt marker, never left in a
+    finished cache) or an angle code >= L (L = 100 leaves codes 100..127
+    unused) sets KVQ_DEVERR_BAD_CODE; a decode step does not check the row it
+    is about to append."""
+    d, B, H_kv, G, n = 128, 2, 2, 4, 300
+    rng = np.random.default_rng(41)
+    kc, vc = kvq.codec(d, 100, kvq.KVQ_NORM_LIN8), kvq.codec(d, 64, kvq.KVQ_NORM_LOG4)
+    sk = torch.from_numpy(np.where(rng.integers(0, 2, d) == 0, 1, -1).astype(np.int8)).cuda()
+    sv = torch.from_numpy(np.where(rng.integers(0, 2, d) == 0, 1, -1).astype(np.int8)).cuda()
+    K, V = kvq.alloc_plane(kc, B, H_kv, 320), kvq.alloc_plane(vc, B, H_kv, 320)
+    kvq.encode(kc, sk, torch.from_numpy(rng.standard_normal((B, H_kv, 320, d)).astype(np.float16)).cuda(), K, 0)
+    kvq.encode(vc, sv, torch.from_numpy(rng.standard_normal((B, H_kv, 320, d)).astype(np.float16)).cuda(), V, 0)
+    q = torch.from_numpy(rng.standard_normal((B, G * H_kv, d)).astype(np.float16)).cuda()
+    ctx = torch.full((B,), n, dtype=torch.int32, device="cuda")
+    kvq.kvq_test_control(kvq.KVQ_TEST_DEBUG_CHECKS, 1)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def run():
+        err.zero_()
+        kvq.decode_attn(q, kc, vc, sk, sv, K, V, ctx, n, num_splits=2, err_word=err)
+        torch.cuda.synchronize()
+        return int(err.item())
+    assert run() == 0
+    V.rows(2)[1, 1, 17] = torch.tensor([0x00, 0x7E, 0x00, 0x3C], dtype=torch.uint8)  # LO = NaN
+    assert run() & kvq.KVQ_DEVERR_BAD_CODE
+    kvq.encode(vc, sv, torch.from_numpy(rng.standard_normal((B, H_kv, 320, d)).astype(np.float16)).cuda(), V, 0)
+    assert run() == 0
+    K.rows(0)[0, 0, 5, 0] = 0x7F  # pair 0's 7-bit code = 127 >= L
+    assert run() & kvq.KVQ_DEVERR_BAD_CODE
+    # rows past the context are not looked at
+    kvq.encode(kc, sk, torch.from_numpy(rng.standard_normal((B, H_kv, 320, d)).astype(np.float16)).cuda(), K, 0)
+    K.rows(2)[:, :, n:] = 0xFF  # NaN M beyond ctx
+    assert run() == 0
+    # the row a step appends holds garbage until the step writes it
+    K.rows(2)[:, :, n - 1] = 0xFF
+    err.zero_()
+    kvq.decode_step(q, q[:, :H_kv].contiguous(), q[:, :H_kv].contiguous(), kc, vc, sk, sv, K, V,
+                    ctx, n, num_splits=2, err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    kvq.kvq_test_control(kvq.KVQ_TEST_DEBUG_CHECKS, 0)
+    K.rows(2)[0, 0, 3] = 0xFF
+    assert run() == 0  # checks off: not looked at

@@ -316,6 +316,20 @@ def test_decode_every_codec(dev, d, G, LK, LV, mk, mv):
         assert np.all(got[3] == 0)
 
 
+@pytest.mark.parametrize("G,LK,LV", [(4, 128, 64), (2, 32, 128), (1, 64, 32), (4, 100, 20)])
+def test_decode_multi_wave(dev, G, LK, LV):
+    """Launches of more than one wave of CTAs (here 8 x 4 x 6 = 192 > 148)
+    with G up to 4 and 5..7-bit codes run the two-CTAs-per-SM instance
+    (fewer pairs per lane); against the oracle."""
+    B, H_kv = 8, 4
+    got, want, err = run_decode_case(B, G * H_kv, H_kv, 128, [700, 1, 129, 513, 0, 640, 64, 333],
+                                     LK, LV, seed=G + LK, splits=6)
+    assert err == 0
+    e = rel_l2(got, want)
+    assert e[[0, 1, 2, 3, 5, 6, 7]].max() <= REL_L2_TOL, e
+    assert np.all(got[4] == 0)
+
+
 @pytest.mark.parametrize("LK,LV", [(256, 256), (128, 64), (32, 5), (2, 2), (200, 33)])
 def test_decode_codebooks(dev, LK, LV):
     got, want, _ = run_decode_case(2, 8, 2, 128, [129, 64], LK, LV, seed=LK + LV)
@@ -341,6 +355,7 @@ def test_decode_split_invariance(dev):
     ([4096], None, 8, 4, 128, 128, 64),   # the Llama-shaped layer
     ([1000, 513], 1, 1, 8, 128, 128, 64),  # one split: the held tile is not the first
     ([300, 129, 1, 0], 3, 2, 3, 256, 128, 64),  # the generic kernel (append launched first)
+    ([4096, 3000, 1], 20, 4, 4, 128, 128, 64),  # multi-wave: two CTAs per SM, append first
     ([200, 64], None, 2, 4, 32, 512, 32),
 ])
 def test_decode_step_equals_append_then_decode(dev, ctx_lens, splits, H_kv, G, d, LK, LV):
