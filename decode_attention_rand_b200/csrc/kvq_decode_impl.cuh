@@ -564,50 +564,60 @@ decode_kernel(DecodeArgs A) {
     }
 
     const int grp = lane / NL, lg = lane % NL;
+    // Slot (j, h) of a lane's partial scores holds the logical entry
+    // (j ^ JX, h ^ HX) (token slot, head) so that xor_reduce needs no selects;
+    // after it, final entry e is logical M + e: token slot (M + e) / G, head
+    // (M + e) % G, with softmax reference mh[e].
+    const int M = lg * VF;
+    const int HX = M % G, JX = M / G;
+    const int bitsK = BK > 0 ? BK : A.kc.bits, bitsV = BV > 0 ? BV : A.vc.bits;
+    const int cbK = lg * PP * bitsK, cbV = lg * PP * bitsV;
+    // all staged data is addressed by 32-bit shared-window offsets; row
+    // strides are compile-time constants for the fixed code widths
+    const int rbK = 4 * (BK > 0 ? (P * BK + 31) / 32 : A.kc.angle_words);
+    const int rbV = 4 * (BV > 0 ? (P * BV + 31) / 32 : A.vc.angle_words);
+    const uint32_t lane_off = (uint32_t)(lane & 15) * 8u;
+    const uint32_t tKl = smem_u32(tabK) + lane_off, tVl = smem_u32(tabV) + lane_off;
+    const uint32_t wK = 4u * (uint32_t)(cbK >> 5), wV = 4u * (uint32_t)(cbV >> 5);
+    const int shK = cbK & 31, shV = cbV & 31;
+    const uint32_t stages32 = smem_u32(stages);
+    // ---- merge the NG group states of this CTA (reuses the stage memory) --
+    // accumulators as [G][PP][NG * 2 NL + pad]: a warp writes one (h, k) row
+    // segment of 32 consecutive float2 (no bank conflicts), and the pad puts
+    // the next k row on the other half of the banks for the summing pass
+    constexpr int ROW = NG * 2 * NL + 16;
+    float* gm = reinterpret_cast<float*>(stages);  // [NG][G]  running maxima
+    float* gl = gm + NG * G;                      // [NG][G]  denominators, then weights
+    float* gacc = gl + NG * G;                    // [G][PP][ROW]
+    float* hml = gacc + G * PP * ROW;             // [G][2]   CTA max and denominator
+
     const int gidx = warp * GPW + grp;
-    f32x2 acc[G][PP];
+    float2 acc[G][PP];
     float mref[G];
     float lpart[VF];
 #pragma unroll
     for (int h = 0; h < G; h++) {
         mref[h] = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < PP; k++) acc[h][k] = 0ull;
+        for (int k = 0; k < PP; k++) acc[h][k] = make_float2(0.f, 0.f);
     }
 #pragma unroll
     for (int e = 0; e < VF; e++) lpart[e] = 0.f;
 
-    // Slot (j, h) of this lane's partial scores holds the logical entry
-    // (j ^ JX, h ^ HX) (token slot, head) so that xor_reduce needs no selects;
-    // after it, final entry e is logical M + e: token slot (M + e) / G, head
-    // (M + e) % G, with softmax reference mh[e].
-    const int M = lg * VF;
-    const int HX = M % G, JX = M / G;
-    float mh[VF];
+    float mh[VF];  // softmax reference of final entry e
 #pragma unroll
     for (int e = 0; e < VF; e++) mh[e] = -INFINITY;
     float* pbuf = pbuf_all + warp * Cfg::PBUF;  // [TW][G] (p, p) of this warp's block
 
     {
-        f32x2 q2[G][PP];
+        float2 q2[G][PP];
 #pragma unroll
         for (int h = 0; h < G; h++)
 #pragma unroll
             for (int k = 0; k < PP; k++) {
                 const float2 qq = reinterpret_cast<const float2*>(qs + (h ^ HX) * D)[lg * PP + k];
-                q2[h][k] = pack2(qq.x, qq.y);
+                q2[h][k] = qq;
             }
-        const int bitsK = BK > 0 ? BK : A.kc.bits, bitsV = BV > 0 ? BV : A.vc.bits;
-        const int cbK = lg * PP * bitsK, cbV = lg * PP * bitsV;
-        // all staged data is addressed by 32-bit shared-window offsets; row
-        // strides are compile-time constants for the fixed code widths
-        const int rbK = 4 * (BK > 0 ? (P * BK + 31) / 32 : A.kc.angle_words);
-        const int rbV = 4 * (BV > 0 ? (P * BV + 31) / 32 : A.vc.angle_words);
-        const uint32_t lane_off = (uint32_t)(lane & 15) * 8u;
-        const uint32_t tKl = smem_u32(tabK) + lane_off, tVl = smem_u32(tabV) + lane_off;
-        const uint32_t wK = 4u * (uint32_t)(cbK >> 5), wV = 4u * (uint32_t)(cbV >> 5);
-        const int shK = cbK & 31, shV = cbV & 31;
-        const uint32_t stages32 = smem_u32(stages);
 
         for (int tile = 0; tile < nloop; tile++) {
             const int s = tile % NST;
@@ -636,23 +646,24 @@ decode_kernel(DecodeArgs A) {
                     angle_addrs<PP, BK>(sKa + (uint32_t)(t * rbK), shK, bitsK, tKl, off);
                     uint32_t nw[(PP + 3) / 4];
                     lds_bytes<PP>(sKn + (uint32_t)(t * P), nw);
-                    f32x2 dot[G];
-#pragma unroll
-                    for (int h = 0; h < G; h++) dot[h] = 0ull;
+                    float2 dot[G];
 #pragma unroll
                     for (int k = 0; k < PP; k++) {
                         // norm byte c -> f = 1 + c 2^-15 (bytes 0x3F 0x80 c 0x00);
                         // the key table holds U = 2^15 (cos, sin), so
-                        // fma(f, U, -U) = (f - 1) U = c (cos, sin), rounded once
+                        // fma(f, U, -U) = (f - 1) U = c (cos, sin), rounded once;
+                        // the first pair starts the accumulators (no zeroing)
                         const float f = __uint_as_float(
                             __byte_perm(nw[k / 4], 0x3F800000u, 0x7604u | ((k % 4) << 4)));
                         const float2 U = lds_f2(off[k]);
-                        const f32x2 xy = pack2(fmaf(f, U.x, -U.x), fmaf(f, U.y, -U.y));
+                        const float2 xy =
+                            __ffma2_rn(make_float2(f, f), U, make_float2(-U.x, -U.y));
 #pragma unroll
-                        for (int h = 0; h < G; h++) dot[h] = fma2(q2[h][k], xy, dot[h]);
+                        for (int h = 0; h < G; h++)
+                            dot[h] = k == 0 ? __fmul2_rn(q2[h][k], xy) : __ffma2_rn(q2[h][k], xy, dot[h]);
                     }
 #pragma unroll
-                    for (int h = 0; h < G; h++) part[j * G + h] = lo2(dot[h]) + hi2(dot[h]);
+                    for (int h = 0; h < G; h++) part[j * G + h] = dot[h].x + dot[h].y;
                 }
                 xor_reduce<V, NL>(part);
                 // -- scale by M/255 * tau * log2(e), mask, lazy softmax reference
@@ -682,9 +693,9 @@ decode_kernel(DecodeArgs A) {
                         mx[h] = group_max<NL>(mx[h]);
                         const float mn = fmaxf(mref[h], mx[h]);
                         const float al = (mn == -INFINITY) ? 0.f : ex2(mref[h] - mn);
-                        const f32x2 al2 = pack2(al, al);
+                        const float2 al2 = make_float2(al, al);
 #pragma unroll
-                        for (int k = 0; k < PP; k++) acc[h][k] = mul2(acc[h][k], al2);
+                        for (int k = 0; k < PP; k++) acc[h][k] = __fmul2_rn(acc[h][k], al2);
 #pragma unroll
                         for (int e = 0; e < VF; e++)
                             if ((M + e) % G == h) lpart[e] *= al;
@@ -715,16 +726,16 @@ decode_kernel(DecodeArgs A) {
                 for (int j = 0; j < kTPG; j++) {
                     const int tl = j * GPW + grp;
                     const int t = blk * TW + tl;
-                    f32x2 pw[G];
+                    float2 pw[G];
                     if constexpr (G == 1) {
                         const float2 v = reinterpret_cast<const float2*>(pbuf)[tl];
-                        pw[0] = pack2(v.x, v.y);
+                        pw[0] = v;
                     } else {
 #pragma unroll
                         for (int h2 = 0; h2 < G / 2; h2++) {
                             const float4 v = reinterpret_cast<const float4*>(pbuf + tl * G * 2)[h2];
-                            pw[2 * h2] = pack2(v.x, v.y);
-                            pw[2 * h2 + 1] = pack2(v.z, v.w);
+                            pw[2 * h2] = make_float2(v.x, v.y);
+                            pw[2 * h2 + 1] = make_float2(v.z, v.w);
                         }
                     }
                     uint32_t off[PP];
@@ -750,9 +761,9 @@ decode_kernel(DecodeArgs A) {
                         const float f = __uint_as_float((mant & 0x00780000u) | 0x3F800000u);
                         const float r = ex2(fmaf(f, A16, B16));
                         const float2 cs = lds_f2(off[k]);
-                        const f32x2 xy = pack2(r * cs.x, r * cs.y);
+                        const float2 xy = __fmul2_rn(make_float2(r, r), cs);
 #pragma unroll
-                        for (int h = 0; h < G; h++) acc[h][k] = fma2(pw[h], xy, acc[h][k]);
+                        for (int h = 0; h < G; h++) acc[h][k] = __ffma2_rn(pw[h], xy, acc[h][k]);
                     }
                 }
             }
@@ -793,21 +804,12 @@ decode_kernel(DecodeArgs A) {
         for (int h = 0; h < G; h++) {
             mref[h] = -INFINITY;
 #pragma unroll
-            for (int k = 0; k < PP; k++) acc[h][k] = 0ull;
+            for (int k = 0; k < PP; k++) acc[h][k] = make_float2(0.f, 0.f);
         }
 #pragma unroll
         for (int e = 0; e < VF; e++) lpart[e] = 0.f;
     }
 
-    // ---- merge the NG group states of this CTA (reuses the stage memory) --
-    // accumulators as [G][PP][NG * 2 NL + pad]: a warp writes one (h, k) row
-    // segment of 32 consecutive float2 (no bank conflicts), and the pad puts
-    // the next k row on the other half of the banks for the summing pass
-    constexpr int ROW = NG * 2 * NL + 16;
-    float* gm = reinterpret_cast<float*>(stages);  // [NG][G]  running maxima
-    float* gl = gm + NG * G;                      // [NG][G]  denominators, then weights
-    float* gacc = gl + NG * G;                    // [G][PP][ROW]
-    float* hml = gacc + G * PP * ROW;             // [G][2]   CTA max and denominator
     {
         float lh[G];
 #pragma unroll
@@ -833,7 +835,7 @@ decode_kernel(DecodeArgs A) {
 #pragma unroll
             for (int k = 0; k < PP; k++)
                 reinterpret_cast<float2*>(gacc + (h * PP + k) * ROW)[gidx * NL + lg] =
-                    make_float2(lo2(acc[h][k]), hi2(acc[h][k]));
+                    acc[h][k];
     }
     __syncthreads();
     // per head: the CTA max, each group's weight 2^(m_g - max), the denominator
