@@ -88,10 +88,15 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extra", action="store_true",
                    help="headline workload only (no TinyLlama / Llama-layer steps, no prefill)")
-    p.add_argument("--case", default=None, choices=["decode_layer", "encode_layer", "dequant_layer"],
-                   help="run one kernel case only (for profiler captures): the decode of "
-                        "--layer of --workload, or the prefill encode (or dequant) of 8 batch "
-                        "entries of one layer; --steps launches after 3 warm-up launches")
+    p.add_argument("--case", default=None,
+                   choices=["decode_layer", "step_layer", "encode_layer", "dequant_layer"],
+                   help="run one kernel case only (for profiler captures): the decode (or the "
+                        "append + decode step) of --layer of --workload, or the prefill encode "
+                        "(or dequant) of 8 batch entries of one layer; --steps launches after 3 "
+                        "warm-up launches")
+    p.add_argument("--L", type=int, default=None,
+                   help="with --case: codebook size for K and V instead of the workload's "
+                        "(sizes outside the fast kernels' set select the general kernels)")
     p.add_argument("--layer", type=int, default=0)
     p.add_argument("--tensor", default="k", choices=["k", "v"],
                    help="encode_layer / dequant_layer case: the layer's K (8-bit linear norms) "
@@ -546,13 +551,13 @@ def run_case(args):
     kvq.lib()
     device = torch.device("cuda", 0)
     steps = max(1, min(args.steps, 20))
-    if args.case == "decode_layer":
+    if args.case in ("decode_layer", "step_layer"):
         w = synth.WORKLOADS[args.workload]
         layer = args.layer
         sk, sv = synth.layer_signs(w, layer)
         skd, svd = torch.from_numpy(sk).to(device), torch.from_numpy(sv).to(device)
-        kc = kvq.codec(w.d, w.L_K[layer], w.mode_K)
-        vc = kvq.codec(w.d, w.L_V[layer], w.mode_V)
+        kc = kvq.codec(w.d, args.L or w.L_K[layer], w.mode_K)
+        vc = kvq.codec(w.d, args.L or w.L_V[layer], w.mode_V)
         planes = []
         for kind, c, sg in ((synth.KIND_K, kc, skd), (synth.KIND_V, vc, svd)):
             p = kvq.alloc_plane(c, w.B, w.H_kv, w.ctx, device)
@@ -567,15 +572,29 @@ def run_case(args):
         S = kvq.kvq_decode_num_splits(w.B, w.H_kv, w.ctx, sm)
         ws = kvq.DecodeWorkspace(w.B, w.H_q, w.d, S, device)
 
-        def run():
-            kvq.decode_attn(q, kc, vc, skd, svd, planes[0], planes[1], ctx, w.ctx, None,
-                            num_splits=S, workspace=ws, out=out, out_dtype=kvq.OUT_FP16)
-        what = f"decode {w.name} layer {layer}, {S} splits"
+        if args.case == "decode_layer":
+            def run():
+                kvq.decode_attn(q, kc, vc, skd, svd, planes[0], planes[1], ctx, w.ctx, None,
+                                num_splits=S, workspace=ws, out=out, out_dtype=kvq.OUT_FP16)
+            what = f"decode {w.name} layer {layer}, {S} splits"
+        else:
+            # every launch appends the same new token at position ctx - 1
+            kn = synth.kv(w, layer, synth.KIND_K, device=device, T=1, salt=7)[:, :, 0].contiguous()
+            vn = synth.kv(w, layer, synth.KIND_V, device=device, T=1, salt=7)[:, :, 0].contiguous()
+
+            def run():
+                kvq.decode_step(q, kn, vn, kc, vc, skd, svd, planes[0], planes[1], ctx, w.ctx,
+                                None, num_splits=S, workspace=ws, out=out,
+                                out_dtype=kvq.OUT_FP16)
+            what = f"append + decode step {w.name} layer {layer}, {S} splits"
+        if args.L:
+            what += f", L_K = L_V = {args.L}"
     else:
         w = synth.WORKLOADS[PREFILL]
         sk, sv = synth.layer_signs(w, 0)
         isk = args.tensor == "k"
-        c = (kvq.codec(w.d, w.L_K[0], w.mode_K) if isk else kvq.codec(w.d, w.L_V[0], w.mode_V))
+        c = (kvq.codec(w.d, args.L or w.L_K[0], w.mode_K) if isk
+             else kvq.codec(w.d, args.L or w.L_V[0], w.mode_V))
         nb = 8
         p = kvq.alloc_plane(c, nb, w.H_kv, w.ctx, device)
         x = synth.kv(w, 0, synth.KIND_K if isk else synth.KIND_V, device=device, b_range=(0, nb))

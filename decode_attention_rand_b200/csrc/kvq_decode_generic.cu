@@ -340,13 +340,18 @@ decode_generic_kernel(DecodeArgs A, int chunks) {
 // The new token of every (b, KV head) at position ctx_len[b] - 1, written
 // exactly as kvq_encode_kv writes it (the same encode_tile): warp 0 encodes
 // the K vector, warp 1 the V vector.
+//
+// Its dependent (the decode) may start once every CTA here has passed the
+// wait for the kernels before it: by then everything those kernels wrote (q,
+// ctx_len, the cache) is complete and visible, and the decode needs to wait
+// for this kernel only before it copies in the tile holding the new rows.
 template <int D>
 __global__ void __launch_bounds__(64) append_kernel(DecodeArgs A) {
-    asm volatile("griddepcontrol.launch_dependents;");
     __shared__ uint32_t est[2][kEncStageWords];
     const int kvh = blockIdx.x, b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     gen_griddep_wait();
+    asm volatile("griddepcontrol.launch_dependents;");
     const int64_t lim = A.max_ctx < A.K.capacity ? A.max_ctx : A.K.capacity;
     const int64_t ctx = A.ctx_len[b];
     if (ctx < 1 || ctx > lim) return;  // nothing to append (the decode reports the clip)

@@ -443,10 +443,12 @@ decode_kernel(DecodeArgs A) {
     // tile t + NST - 1 is issued once tile t - 1 is released, so NST - 1 tiles
     // are in flight ahead of the one being consumed
     // Launched as a programmatic dependent of the previous kernel on the
-    // stream (typically the append of this step), the kernel may start
+    // stream (the previous layer's or step's decode), the kernel may start
     // before that one ends: nothing it reads from global memory (codes, q,
     // ctx_len, signs) is touched before griddepcontrol.wait; the barrier setup
-    // and the cos/sin tables overlap the previous kernel's tail.
+    // and the cos/sin tables overlap the previous kernel's tail.  After a
+    // separate append launch (append_pending) everything but the new row is
+    // already final when the kernel starts, so only that row's tile waits.
     // Fused append (kvq_decode_step): the split holding the new token (position
     // ctx_len[b] - 1) encodes it with warps 0 and 1 while the other warps build
     // the tables and rotate q; the tile holding it, and the ones after, are
@@ -455,6 +457,9 @@ decode_kernel(DecodeArgs A) {
     // the two-CTA instance carries no append code (its registers would not
     // fit); its kvq_decode_step runs the append as a launch of its own first
     const bool fused = CTAS == 1 && A.k_new != nullptr;
+    // append_kernel ran just before (see DecodeArgs::append_pending): only the
+    // tile holding the new row waits for it, every other read starts at once
+    const bool pending = A.append_pending != 0;
     const int w0 = fused ? 2 : 0;  // first warp of the table / q' work
     int64_t ctx_in = 0;
     bool append = false;           // warps 0 and 1 of a fused launch
@@ -463,10 +468,23 @@ decode_kernel(DecodeArgs A) {
         ctx_in = A.ctx_len[b];
         append = ctx_in >= 1 && ctx_in <= lim && ctx_in - 1 >= t0 && ctx_in - 1 < t1m;
     }
+    int hold = ntiles_max;  // (thread 0) first tile that waits for the append
     if (tid == 0) {
-        griddep_wait();
-        const int hold = append ? (int)((ctx_in - 1 - t0) / kTT) : ntiles_max;
+        if (pending) {
+            const int64_t c = A.ctx_len[b];
+            if (c >= 1 && c <= lim && c - 1 >= t0 && c - 1 < t1m) hold = (int)((c - 1 - t0) / kTT);
+        } else {
+            griddep_wait();
+            if (append) hold = (int)((ctx_in - 1 - t0) / kTT);
+        }
         for (; issued < NST - 1 && issued < ntiles_max && issued < hold; issued++) issue_tile(issued);
+        if (pending && issued < NST - 1 && issued < ntiles_max) {
+            griddep_wait();
+            hold = ntiles_max;
+            for (; issued < NST - 1 && issued < ntiles_max; issued++) issue_tile(issued);
+        }
+        // from here on only a pending append's tile waits (in the refill)
+        if (!pending || hold >= ntiles_max) hold = 1 << 30;
     }
     if (fused && warp < 2) {
         if constexpr (CTAS == 1) if (append) {
@@ -516,7 +534,7 @@ decode_kernel(DecodeArgs A) {
 #pragma unroll 1
         for (int idx = t; idx < (nK + nV) * kTabRep; idx += nthr)
             if (idx % kTabRep) tabK[idx] = tabK[idx - idx % kTabRep];
-        griddep_wait();
+        if (!pending) griddep_wait();
         ctx_in = A.ctx_len[b];
         for (int h = warp - w0; h < G; h += WARPS - w0) {
             const __half* qh = A.q + ((int64_t)b * A.H_q + (int64_t)kvh * G + h) * D;
@@ -779,6 +797,10 @@ decode_kernel(DecodeArgs A) {
                     ok = mbar_wait_bounded(&empty[sn], (uint32_t)((nxt / NST) - 1) & 1u,
                                            A.wait_limit);
                 if (ok) {
+                    if (nxt >= hold) {
+                        griddep_wait();  // the append's rows are written
+                        hold = 1 << 30;
+                    }
                     issue_tile(nxt);
                     issued = nxt + 1;
                 } else {
@@ -1198,6 +1220,7 @@ inline cudaError_t launch_decode_dg(const DecodeArgs& a, cudaStream_t stream) {
                 const cudaError_t e = launch_append(a, stream);
                 if (e != cudaSuccess) return e;
                 b.k_new = b.v_new = nullptr;
+                b.append_pending = 1;
             }
 #define KVQ_BB2(X, Y) \
     if (bk == X && bv == Y) return launch_decode_kernel<D, G, X, Y, 2>(b, stream);

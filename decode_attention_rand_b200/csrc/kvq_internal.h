@@ -77,6 +77,12 @@ struct DecodeArgs {
     // fused append (kvq_decode_step): the new token of every (b, KV head),
     // encoded by the CTA whose split holds position ctx_len[b] - 1
     uint32_t wait_limit;     // tries before a tile wait gives up (kvq_test_control)
+    // 1: the new token's rows are being written by append_kernel, the launch
+    // this one is a programmatic dependent of; that kernel starts its
+    // dependents only once everything before it has completed, so this one
+    // reads q and ctx_len at once and waits for the append (griddepcontrol)
+    // only before copying in the tile that holds the new row
+    int append_pending;
     const __half* k_new;     // [B][H_kv][d] or NULL (no append)
     const __half* v_new;     // [B][H_kv][d]
     EncArgs enc_k, enc_v;    // codec, signs and constants of the two encodes

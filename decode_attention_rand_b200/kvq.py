@@ -425,7 +425,9 @@ def decode_step(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v,
                 num_splits=None, workspace: DecodeWorkspace | None = None, err_word=None, out=None,
                 out_dtype: int = OUT_FP32, stream=None):
     """Append k_new / v_new [B, H_kv, d] at position ctx_len[b] - 1 and attend
-    q over positions 0 .. ctx_len[b] - 1, in one kernel."""
+    q over positions 0 .. ctx_len[b] - 1: one kernel, or an append launch
+    followed by the decode where the decode instance carries no append code
+    (the two-CTAs-per-SM and runtime-width kernels)."""
     import torch
     B, H_q, d = q.shape
     if softmax_scale is None:
