@@ -303,7 +303,9 @@ class DecodeStep:
             L = dict(kc=kc, vc=vc, skd=skd, svd=svd, planes=planes, io=io, q=q, knew=knew,
                      vnew=vnew, out=out, cK=[p[0].c() for p in planes],
                      cV=[p[1].c() for p in planes])
-            # one kernel: append the new K and V at position ctx - 1, then attend
+            # append the new K and V at position ctx - 1, then attend: one kernel,
+            # or an append launch and the decode (the library decides per codec
+            # and launch shape)
             L["calls"] = [kvq.DecodeStepCall(q, knew, vnew, kc, vc, skd, svd, L["cK"][b],
                                              L["cV"][b], self.ctx, w.B, w.H_q, w.H_kv, w.ctx,
                                              self.tau, self.S, self.ws.buf, self.ws.nbytes,
@@ -311,7 +313,7 @@ class DecodeStep:
                           for b in range(self.nbuf)]
             self.layers.append(L)
         torch.cuda.synchronize(device)
-        self.kernels_per_step = w.layers  # one fused append + decode launch per layer
+        self.calls_per_step = w.layers  # one kvq_decode_step call per layer
         self.bytes_per_step, self.bytes_per_launch = total, per_layer
         self.cache_bytes = cache_bytes * self.nbuf
 
@@ -344,7 +346,7 @@ def time_graph(state, K, W, dist_ctx):
     for i in range(W):
         state.step(i)
     torch.cuda.synchronize()
-    per_graph = max(1, math.ceil(256 / max(1, state.kernels_per_step)))
+    per_graph = max(1, math.ceil(256 / max(1, state.calls_per_step)))
     unit = max(1, min(K, state.nbuf * max(1, math.ceil(per_graph / state.nbuf))))
     n_full, rem = divmod(K, unit)
     g_unit = torch.cuda.CUDAGraph()
@@ -359,7 +361,7 @@ def time_graph(state, K, W, dist_ctx):
                 state.step(n_full * unit + i, stream=torch.cuda.current_stream())
     # external events become event-record nodes of the graph, so each decode
     # launch is timed inside the replay
-    n_ev = max(1, min(unit, 4 if state.kernels_per_step > 1 else 16))
+    n_ev = max(1, min(unit, 4 if state.calls_per_step > 1 else 16))
     evs = [[[torch.cuda.Event(enable_timing=True, external=True),
              torch.cuda.Event(enable_timing=True, external=True)]
             for _ in state.layers] for _ in range(n_ev)]
@@ -396,6 +398,28 @@ def time_graph(state, K, W, dist_ctx):
                 per_layer[li].append(evs[i][li][0].elapsed_time(evs[i][li][1]))
     del g_unit, g_rem, g_ev
     return ms, [statistics.fmean(x) for x in per_layer], (t_wall0, t_wall1)
+
+
+def kernel_launches_per_step(state):
+    """Kernels of one step, counted from a CUDA graph of it (kernel nodes of
+    the captured, never replayed, graph)."""
+    import torch
+    from cuda.bindings import runtime as rt
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    stream = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=stream):
+        state.step(0, stream=torch.cuda.current_stream())
+    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    err, _, n = rt.cudaGraphGetNodes(graph, 0)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    count = sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
+    del g
+    return count
 
 
 def time_e2e(state, K, dist_ctx):
@@ -441,8 +465,10 @@ def decode_report(state, ms, K, per_launch_ms, hbm_peak, peak_kind, sm_mhz, sm_c
                   traffic=None):
     """Throughput and roofline figures of a timed decode workload."""
     w = state.w
-    launches = K * state.kernels_per_step
-    us_launch = ms / launches * 1e3  # one kvq_decode_step launch per layer
+    calls = K * state.calls_per_step
+    # per layer: the decode kernel, with the append fused in or hidden behind
+    # its first tiles; the roofline takes the whole layer's time (conservative)
+    us_launch = ms / calls * 1e3
     bytes_launch = statistics.fmean(state.bytes_per_launch)
     gbs = bytes_launch / (us_launch / 1e6) / 1e9
     flops = w.B * w.H_kv * w.ctx * decode_flops_per_token_head(w.d, w.G)
@@ -466,8 +492,9 @@ def decode_report(state, ms, K, per_launch_ms, hbm_peak, peak_kind, sm_mhz, sm_c
         "bytes_per_step": state.bytes_per_step,
         "num_splits": state.S,
         "roofline": {
-            "kernel": "decode_kernel (kvq_decode_step: append of the new token, split-K "
-                      "decode attention and the split combine, one launch per layer)",
+            "kernel": "decode_kernel (split-K decode attention with the split combine; "
+                      "kvq_decode_step runs it per layer with the new token's append fused in, "
+                      "or after an append_kernel launch it hides; time per layer)",
             "bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
             "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
             "traffic": traffic, "bytes_per_launch": bytes_launch, "us_per_launch": us_launch,
@@ -809,7 +836,7 @@ def measure(name, device, l2, K, W, ctx, hbm_peak, peak_kind, sm_count, sampler,
                       "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "steps": e_n, "transfer": "cudaMemcpyAsync in and out on the stream per call"}
     err = int(state.err.item())
-    launches = state.kernels_per_step * K
+    launches = kernel_launches_per_step(state) * K
     state.release()
     if err != 0:
         raise RuntimeError(f"{name}: device error word {err}")

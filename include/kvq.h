@@ -368,8 +368,10 @@ int kvq_decode_step_paged(const void* q, const void* k_new, const void* v_new,
  * KVQ_EINVAL before any launch (fewer splits reduce it).  The first call on a
  * device looks up the array's device address (with that device current):
  * make it before any stream capture.  Each call first clears the completion
- * counters with an asynchronous memset on `stream`; the call allocates
- * nothing.  All calls share the one array, so calls whose kernels overlap on
+ * counters with an asynchronous memset on `stream`, then runs the checks and
+ * the launch of kvq_decode_attn: a call that those checks reject returns
+ * KVQ_EINVAL with the memset already queued (harmless: every complete decode
+ * leaves the counters at zero anyway).  The call allocates nothing.  All calls share the one array, so calls whose kernels overlap on
  * the GPU race on it and must be ordered by the caller. */
 int kvq_decode_attn_noalloc(const void* q, const kvq_codec* kc,
                             const kvq_codec* vc, const int8_t* signs_k,
