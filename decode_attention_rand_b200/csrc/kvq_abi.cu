@@ -406,6 +406,11 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
     const int64_t gran = paged ? 128 : 16;
     sl = (sl + gran - 1) / gran * gran;
     a.split_len = sl < gran ? gran : sl;
+    // the kernels count a split's tokens in 32 bits (2^30 tokens of codes are
+    // already more than a GPU holds)
+    if (a.split_len > (1ll << 30))
+        return fail(KVQ_EINVAL, "%s: a split of %lld tokens exceeds 2^30; raise num_splits", what,
+                    (long long)a.split_len);
     a.ws = static_cast<float*>(workspace);
     a.err_word = err_word;
     a.out = out;

@@ -268,6 +268,26 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
     asm volatile("ld.shared.u8 %0, [%1+%2];" : "=h"(v) : "r"(a), "n"(OFF));
     return v;
 }
+// Softmax weights handed from the score pass to the value pass of a warp:
+// explicit shared accesses with a memory clobber, ordered by the __syncwarp
+// on either side of the hand-off.
+__device__ __forceinline__ void sts_pp(uint32_t a, float p) {
+    asm volatile("st.shared.v2.f32 [%0], {%1, %1};" ::"r"(a), "f"(p) : "memory");
+}
+template <int OFF = 0>
+__device__ __forceinline__ float4 lds_pp4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(a), "n"(OFF)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ float2 lds_pp2(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a) : "memory");
+    return v;
+}
 __device__ __forceinline__ float2 lds_f2(uint32_t a) {
     float2 v;
     asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
@@ -563,6 +583,7 @@ decode_kernel(DecodeArgs A) {
         ctx = ctx < 0 ? 0 : lim;
     }
     const int64_t t1 = t1m < ctx ? t1m : ctx;
+    const int span = t1 > t0 ? (int)(t1 - t0) : 0;  // a split is far shorter than 2^31 tokens
     const int ntiles = t1 > t0 ? (int)((t1 - t0 + kTT - 1) / kTT) : 0;
     // every issued tile is consumed (tiles past the context are fully masked)
     const int nloop = ntiles > (NST - 1 < ntiles_max ? NST - 1 : ntiles_max)
@@ -625,7 +646,8 @@ decode_kernel(DecodeArgs A) {
     float mh[VF];  // softmax reference of final entry e
 #pragma unroll
     for (int e = 0; e < VF; e++) mh[e] = -INFINITY;
-    float* pbuf = pbuf_all + warp * Cfg::PBUF;  // [TW][G] (p, p) of this warp's block
+    // [TW][G] (p, p) of this warp's block
+    const uint32_t pbuf = smem_u32(pbuf_all + warp * Cfg::PBUF);
 
     {
         float2 q2[G][PP];
@@ -650,8 +672,8 @@ decode_kernel(DecodeArgs A) {
             const uint32_t sKp = st + A.lay[2];
             const uint32_t sVa = st + A.lay[3] + wV, sVn = st + A.lay[4] + lg * (PP / 2);
             const uint32_t sVp = st + A.lay[5];
-            const int64_t tt0 = t0 + (int64_t)tile * kTT;
-            const int ntok = (int)((t1 - tt0) < kTT ? (t1 - tt0) : kTT);
+            const int left = span - tile * kTT;  // tokens of the split from this tile on
+            const int ntok = left < kTT ? left : kTT;
 
             for (int blk = warp; blk * TW < ntok; blk += WARPS) {
                 // -- scores: this lane's partial dot products, slot (j, h) --
@@ -735,8 +757,7 @@ decode_kernel(DecodeArgs A) {
                     const int idx = M + e;
                     const float p = part[e] == -INFINITY ? 0.f : ex2(part[e] - mh[e]);
                     lpart[e] += p;
-                    reinterpret_cast<float2*>(pbuf)[((idx / G) * GPW + grp) * G + idx % G] =
-                        make_float2(p, p);
+                    sts_pp(pbuf + 8u * (uint32_t)(((idx / G) * GPW + grp) * G + idx % G), p);
                 }
                 __syncwarp();
                 // -- values: acc[h] += p[t][h] * r^ (cos, sin), rotated domain --
@@ -746,14 +767,24 @@ decode_kernel(DecodeArgs A) {
                     const int t = blk * TW + tl;
                     float2 pw[G];
                     if constexpr (G == 1) {
-                        const float2 v = reinterpret_cast<const float2*>(pbuf)[tl];
-                        pw[0] = v;
+                        pw[0] = lds_pp2(pbuf + 8u * (uint32_t)tl);
                     } else {
-#pragma unroll
-                        for (int h2 = 0; h2 < G / 2; h2++) {
-                            const float4 v = reinterpret_cast<const float4*>(pbuf + tl * G * 2)[h2];
-                            pw[2 * h2] = make_float2(v.x, v.y);
-                            pw[2 * h2 + 1] = make_float2(v.z, v.w);
+                        const uint32_t pa = pbuf + 8u * (uint32_t)(tl * G);
+                        float4 v = lds_pp4<0>(pa);
+                        pw[0] = make_float2(v.x, v.y);
+                        pw[1] = make_float2(v.z, v.w);
+                        if constexpr (G >= 4) {
+                            v = lds_pp4<16>(pa);
+                            pw[2] = make_float2(v.x, v.y);
+                            pw[3] = make_float2(v.z, v.w);
+                        }
+                        if constexpr (G >= 8) {
+                            v = lds_pp4<32>(pa);
+                            pw[4] = make_float2(v.x, v.y);
+                            pw[5] = make_float2(v.z, v.w);
+                            v = lds_pp4<48>(pa);
+                            pw[6] = make_float2(v.x, v.y);
+                            pw[7] = make_float2(v.z, v.w);
                         }
                     }
                     uint32_t off[PP];

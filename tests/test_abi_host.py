@@ -172,6 +172,7 @@ def _decode_rc(**kw):
     (dict(out_dtype=3), kvq.KVQ_EINVAL, "out_dtype"),
     (dict(scale=float("nan")), kvq.KVQ_EINVAL, "softmax_scale"),
     (dict(max_ctx=-1), kvq.KVQ_EINVAL, "negative"),
+    (dict(max_ctx=1 << 31, S=1), kvq.KVQ_EINVAL, "exceeds 2^30"),
 ])
 def test_decode_rejects_bad_arguments(kw, status, msg):
     assert _decode_rc(**kw) == status
