@@ -307,7 +307,7 @@ __device__ __forceinline__ float4 lds_f4(uint32_t a) {
 // [cb, cb + PP*B) of the row at shared address `row` (wa = its first word:
 // the row address plus 4 (cb >> 5); sh = cb & 31).  B > 0: compile-time
 // width; B == 0: runtime width `bits`.
-template <int PP, int B>
+template <int PP, int B, bool TABC = false>
 __device__ __forceinline__ void angle_addrs(uint32_t wa, int sh, int bits, uint32_t tab_lane,
                                             uint32_t (&off)[PP]) {
     if constexpr (B > 0) {
@@ -335,7 +335,10 @@ __device__ __forceinline__ void angle_addrs(uint32_t wa, int sh, int bits, uint3
             } else {
                 x = __funnelshift_r(n[wi], n[wi + 1], bi - kTabShift);
             }
-            off[k] = (x & mask) + tab_lane;
+            // with a table at a compile-time address the lane's replica offset
+            // (below bit kTabShift) is or-ed in with the mask, and the base
+            // is left to the load's immediate (see tab_f2)
+            off[k] = TABC ? ((x & mask) | tab_lane) : ((x & mask) + tab_lane);
         }
     } else {
         const uint32_t mask = (1u << bits) - 1u;
@@ -349,6 +352,14 @@ __device__ __forceinline__ void angle_addrs(uint32_t wa, int sh, int bits, uint3
                 off[4 * q + k] = (((win >> (k * bits)) & mask) << kTabShift) + tab_lane;
         }
     }
+}
+
+// Table entry at byte offset `off` of a table in static shared memory: a
+// plain shared load, so the compiler can carry the table base in the load's
+// immediate.  The tables are written before the barrier that precedes every
+// lookup.
+__device__ __forceinline__ float2 tab_f2(const float2* tab, uint32_t off) {
+    return *reinterpret_cast<const float2*>(reinterpret_cast<const char*>(tab) + off);
 }
 
 // NBYTES bytes (1, 2, 4, 8, 16) at shared address a as little-endian words.
@@ -398,7 +409,8 @@ decode_kernel(DecodeArgs A) {
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);           // [kMaxStages]
     uint64_t* empty = full + kMaxStages;                          // [kMaxStages]
     int* sflag = reinterpret_cast<int*>(smem + 16 * kMaxStages);  // timeout, last
-    const int nK = 1 << A.kc.bits, nV = 1 << A.vc.bits;
+    // table sizes: compile-time for fixed widths (so are the table addresses)
+    const int nK = 1 << (BK > 0 ? BK : A.kc.bits), nV = 1 << (BV > 0 ? BV : A.vc.bits);
     unsigned char* dyn = smem + 16 * kMaxStages + 16;
     // key table: 2^15 (cos, sin) [2^bK][16]; value table: (cos, sin) [2^bV][16]
     float2* tabK = kStatic ? s_tab : reinterpret_cast<float2*>(dyn);
@@ -616,7 +628,11 @@ decode_kernel(DecodeArgs A) {
     const int rbK = 4 * (BK > 0 ? (P * BK + 31) / 32 : A.kc.angle_words);
     const int rbV = 4 * (BV > 0 ? (P * BV + 31) / 32 : A.vc.angle_words);
     const uint32_t lane_off = (uint32_t)(lane & 15) * 8u;
-    const uint32_t tKl = smem_u32(tabK) + lane_off, tVl = smem_u32(tabV) + lane_off;
+    // static tables: both table addresses are compile-time constants (tabV
+    // follows 2^BK key entries), so lookups take the lane offset alone
+    constexpr bool kTabC = kStatic;
+    const uint32_t tKl = kTabC ? lane_off : smem_u32(tabK) + lane_off;
+    const uint32_t tVl = kTabC ? lane_off : smem_u32(tabV) + lane_off;
     const uint32_t wK = 4u * (uint32_t)(cbK >> 5), wV = 4u * (uint32_t)(cbV >> 5);
     const int shK = cbK & 31, shV = cbV & 31;
     const uint32_t stages32 = smem_u32(stages);
@@ -683,7 +699,7 @@ decode_kernel(DecodeArgs A) {
                 for (int j = 0; j < kTPG; j++) {
                     const int t = blk * TW + (j ^ JX) * GPW + grp;
                     uint32_t off[PP];
-                    angle_addrs<PP, BK>(sKa + (uint32_t)(t * rbK), shK, bitsK, tKl, off);
+                    angle_addrs<PP, BK, kTabC>(sKa + (uint32_t)(t * rbK), shK, bitsK, tKl, off);
                     uint32_t nw[(PP + 3) / 4];
                     lds_bytes<PP>(sKn + (uint32_t)(t * P), nw);
                     float2 dot[G];
@@ -695,7 +711,7 @@ decode_kernel(DecodeArgs A) {
                         // the first pair starts the accumulators (no zeroing)
                         const float f = __uint_as_float(
                             __byte_perm(nw[k / 4], 0x3F800000u, 0x7604u | ((k % 4) << 4)));
-                        const float2 U = lds_f2(off[k]);
+                        const float2 U = kTabC ? tab_f2(tabK, off[k]) : lds_f2(off[k]);
                         const float2 xy =
                             __ffma2_rn(make_float2(f, f), U, make_float2(-U.x, -U.y));
 #pragma unroll
@@ -788,7 +804,7 @@ decode_kernel(DecodeArgs A) {
                         }
                     }
                     uint32_t off[PP];
-                    angle_addrs<PP, BV>(sVa + (uint32_t)(t * rbV), shV, bitsV, tVl, off);
+                    angle_addrs<PP, BV, kTabC>(sVa + (uint32_t)(t * rbV), shV, bitsV, tVl, off);
                     uint32_t nw[(PP / 2 + 3) / 4];
                     lds_bytes<PP / 2>(sVn + (uint32_t)(t * (P / 2)), nw);
                     const uint32_t pr = lds_u32(sVp + 4u * (uint32_t)t);
@@ -809,7 +825,7 @@ decode_kernel(DecodeArgs A) {
                         const uint32_t mant = sh <= 19 ? (w << (19 - sh)) : (w >> (sh - 19));
                         const float f = __uint_as_float((mant & 0x00780000u) | 0x3F800000u);
                         const float r = ex2(fmaf(f, A16, B16));
-                        const float2 cs = lds_f2(off[k]);
+                        const float2 cs = kTabC ? tab_f2(tabV, off[k]) : lds_f2(off[k]);
                         const float2 xy = __fmul2_rn(make_float2(r, r), cs);
 #pragma unroll
                         for (int h = 0; h < G; h++) acc[h][k] = __ffma2_rn(pw[h], xy, acc[h][k]);
