@@ -186,8 +186,10 @@ struct DqFastCfg {
     static constexpr int S = D == 64 ? 6 : D == 128 ? 7 : 8;
 };
 
+constexpr int kDqFastBlocksPerSM = 3;  // registers for one tile ahead in flight
+
 template <int D, int B>
-__global__ void __launch_bounds__(kDqWarps * 32, 4)
+__global__ void __launch_bounds__(kDqWarps * 32, kDqFastBlocksPerSM)
 dequant_fast_kernel(DqArgs A) {
     using Cfg = DqFastCfg<D>;
     constexpr int NL = Cfg::NL, VPW = Cfg::VPW, S = Cfg::S;
@@ -221,36 +223,54 @@ dequant_fast_kernel(DqArgs A) {
     const int wbase = (lg * 16 * B) >> 5, sh = (lg * 16 * B) & 31;
     const uint32_t n_tiles = (uint32_t)((A.n_vec + VPW - 1) / VPW);
     const uint32_t stride = gridDim.x * kDqWarps;
-    for (uint32_t wt = blockIdx.x * kDqWarps + warp; wt < n_tiles; wt += stride) {
+    // The code rows of a warp tile are loaded one iteration ahead: the loads
+    // of tile wt + stride are in flight while tile wt is transformed.
+    struct Rows {
+        uint32_t w[5];   // angle words from the lane's first one
+        uint4 nq;        // norm bytes (LIN8: 16, LOG4: 8 in .x/.y)
+        uint32_t pr;     // parameters (LIN8: fp16 M, LOG4: fp16 LO | HI << 16)
+    };
+    auto fetch = [&](uint32_t wt, Rows& R) {
         const uint32_t v = wt * VPW + grp;
-        const bool valid = (int64_t)v < A.n_vec;
-        const uint32_t vv = valid ? v : 0u;
+        const uint32_t vv = (int64_t)v < A.n_vec ? v : 0u;
         const uint32_t vt = fast_div(vv, A.tdiv);
         const int64_t row =
             (int64_t)vt * A.in.capacity + A.pos0 + (int64_t)(vv - vt * (uint32_t)A.T);
-        // angle codes: up to five words, aligned to the lane's first bit
-        uint32_t W[4];
-        {
-            const uint32_t* ar = reinterpret_cast<const uint32_t*>(A.in.angles) + row * AW;
-            uint32_t w[5];
+        const uint32_t* ar = reinterpret_cast<const uint32_t*>(A.in.angles) + row * AW;
 #pragma unroll
-            for (int j = 0; j < 5; j++) w[j] = wbase + j < AW ? ar[wbase + j] : 0u;
-#pragma unroll
-            for (int j = 0; j < 4; j++) W[j] = __funnelshift_r(w[j], w[j + 1], sh);
+        for (int j = 0; j < 5; j++) R.w[j] = wbase + j < AW ? ar[wbase + j] : 0u;
+        if (lin8) {
+            R.nq = *reinterpret_cast<const uint4*>(A.in.norms + row * (D / 2) + lg * 16);
+            R.pr = reinterpret_cast<const uint16_t*>(A.in.params)[row];
+        } else {
+            const uint2 q2 = *reinterpret_cast<const uint2*>(A.in.norms + row * (D / 4) + lg * 8);
+            R.nq = make_uint4(q2.x, q2.y, 0u, 0u);
+            R.pr = reinterpret_cast<const uint32_t*>(A.in.params)[row];
         }
+    };
+    Rows nxt;
+    uint32_t wt = blockIdx.x * kDqWarps + warp;
+    if (wt < n_tiles) fetch(wt, nxt);
+    for (; wt < n_tiles; wt += stride) {
+        const Rows cur = nxt;
+        if (wt + stride < n_tiles) fetch(wt + stride, nxt);
+        const uint32_t v = wt * VPW + grp;
+        const bool valid = (int64_t)v < A.n_vec;
+        // angle codes aligned to the lane's first bit
+        uint32_t W[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) W[j] = __funnelshift_r(cur.w[j], cur.w[j + 1], sh);
         // norms: r / sqrt(d) of each pair
         float r[16];
         if (lin8) {
-            const uint4 nq = *reinterpret_cast<const uint4*>(A.in.norms + row * (D / 2) + lg * 16);
-            const uint32_t nw[4] = {nq.x, nq.y, nq.z, nq.w};
-            const float sc = half_bits_to_float(reinterpret_cast<const uint16_t*>(A.in.params)[row]) *
-                             (1.f / 255.f) * isd;
+            const uint32_t nw[4] = {cur.nq.x, cur.nq.y, cur.nq.z, cur.nq.w};
+            const float sc = half_bits_to_float((uint16_t)cur.pr) * (1.f / 255.f) * isd;
 #pragma unroll
             for (int k = 0; k < 16; k++)
                 r[k] = (float)((nw[k >> 2] >> (8 * (k & 3))) & 0xFFu) * sc;
         } else {
-            const uint2 nq = *reinterpret_cast<const uint2*>(A.in.norms + row * (D / 4) + lg * 8);
-            const uint32_t pr = reinterpret_cast<const uint32_t*>(A.in.params)[row];
+            const uint2 nq = make_uint2(cur.nq.x, cur.nq.y);
+            const uint32_t pr = cur.pr;
             const float LO = half_bits_to_float((uint16_t)(pr & 0xFFFF));
             const float step = (half_bits_to_float((uint16_t)(pr >> 16)) - LO) * (1.f / 15.f);
             // 2^(LO + c step) / sqrt(d) = 2^(LO - S/2 + c step)
@@ -291,7 +311,9 @@ static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStre
     constexpr int VPW = DqFastCfg<D>::VPW;
     const int64_t tiles = (a.n_vec + VPW - 1) / VPW;
     int64_t blocks = (tiles + kDqWarps - 1) / kDqWarps;
-    const int64_t cap = (int64_t)sm_count * 8;
+    // one wave of resident blocks, each striding over the tiles (no partly
+    // filled last wave)
+    const int64_t cap = (int64_t)sm_count * kDqFastBlocksPerSM;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     const dim3 g((unsigned)blocks), b(kDqWarps * 32);
