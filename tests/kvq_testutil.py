@@ -100,6 +100,24 @@ def plane_rows(plane, b_range=None, h_range=None, t_range=None):
     return tuple(out)
 
 
+def paged_rows(plane, table, b: int, t0: int, t1: int):
+    """Host copy of tokens t0 .. t1-1 of every KV head of sequence b of a
+    kvq.PagedPlane, read through the page table `table` [B][max_pages]:
+    (angles, norms, params), each uint8 [n, row] in (h, t) order."""
+    import torch
+    pt = plane.page_tokens
+    t = torch.arange(t0, t1)
+    pages = torch.as_tensor(np.asarray(table)[b], dtype=torch.long)[t // pt]
+    dev = plane.rows(0).device
+    pages, offs = pages.to(dev), (t % pt).to(dev)
+    out = []
+    for w in range(3):
+        r = plane.rows(w)
+        rows = [r[pages, h, offs] for h in range(plane.H_kv)]
+        out.append(np.ascontiguousarray(torch.cat(rows).cpu().numpy()))
+    return tuple(out)
+
+
 def put_rows(plane, codes: "O.Codes", b, h, t0: int):
     """Write oracle-encoded rows (tokens t0.. of sequence (b, h)) into a plane."""
     import torch

@@ -213,20 +213,13 @@ def test_paged_bad_page_entry_is_reported(dev):
 
 import oracle as O  # noqa: E402
 
-from kvq_testutil import REL_L2_TOL, compare_codes, rel_l2  # noqa: E402
+from kvq_testutil import REL_L2_TOL, compare_codes, paged_rows, rel_l2  # noqa: E402
 
 
-def _gather(P, table, b, t0, t1, page_tokens=128):
+def _gather(P, table, b, t0, t1):
     """O.Codes of tokens t0 .. t1-1 of every KV head of sequence b, read
     through the page table; rows in (h, t) order."""
-    rows = []
-    for w in range(3):
-        per_h = []
-        for h in range(P.H_kv):
-            parts = [P.rows(w)[int(table[b, t // page_tokens]), h, t % page_tokens]
-                     for t in range(t0, t1)]
-            per_h.append(torch.stack(parts) if parts else P.rows(w)[0, h, :0])
-        rows.append(np.ascontiguousarray(torch.cat(per_h).cpu().numpy()))
+    rows = paged_rows(P, table, b, t0, t1)
     c = P.codec
     return O.Codes(c.head_dim, c.L, c.norm_mode, *rows)
 
@@ -319,6 +312,45 @@ def test_paged_decode_step_matches_oracle(dev):
     kvq.kvq_decode_step_paged(torch.from_numpy(qn).cuda(), torch.from_numpy(kn).cuda(),
                               torch.from_numpy(vn).cuda(), kc, vc, sk, sv, Kp.c(), Vp.c(), ctx,
                               B, H_q, H_kv, 512, tau, S, ws.buf, ws.nbytes, err, out,
+                              kvq.OUT_FP32)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for P, x, s, c in ((Kp, kn, sk, kc), (Vp, vn, sv, vc)):
+        want = O.encode(x, s.cpu().numpy(), c.L, c.norm_mode)
+        for b, n in enumerate(ctx_lens):
+            got = _gather(P, table, b, n - 1, n)
+            compare_codes((got.angles, got.norms, got.params),
+                          want.take(slice(b * H_kv, (b + 1) * H_kv)))
+    want = _oracle_attend_paged(qn, Kp, Vp, table, sk.cpu().numpy(), sv.cpu().numpy(), ctx_lens,
+                                G, tau)
+    assert rel_l2(out.cpu().numpy(), want).max() <= REL_L2_TOL
+
+
+@pytest.mark.gpu
+def test_paged_multi_wave_step_matches_oracle(dev):
+    """A paged step of more than one wave of CTAs (3 x 2 x 28 = 168 > 148
+    SMs, G 4, 7/6-bit codes): the two-CTAs-per-SM decode after its own append
+    launch, the decode waiting for the append only before the tile that holds
+    the new row.  Appends on a page's first row, mid-page and the last row of
+    the last page; codes and output against the oracle."""
+    B, H_kv, G, d, max_pages = 3, 2, 4, 128, 28
+    kc, vc, sk, sv, k, v, Kc, Vc, Kp, Vp, table = _setup(B, H_kv, d, max_pages, seed=31)
+    H_q = G * H_kv
+    rng = np.random.default_rng(32)
+    qn = rng.standard_normal((B, H_q, d)).astype(np.float16)
+    kn = rng.standard_normal((B, H_kv, d)).astype(np.float16)
+    kn[..., 11] *= 20
+    vn = rng.standard_normal((B, H_kv, d)).astype(np.float16)
+    cap = max_pages * 128
+    ctx_lens = [3073, 2000, cap]
+    ctx = torch.tensor(ctx_lens, dtype=torch.int32, device="cuda")
+    S, tau = 28, 1 / math.sqrt(d)
+    ws = _ws(B, H_q, d, S)
+    out = torch.empty((B, H_q, d), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvq.kvq_decode_step_paged(torch.from_numpy(qn).cuda(), torch.from_numpy(kn).cuda(),
+                              torch.from_numpy(vn).cuda(), kc, vc, sk, sv, Kp.c(), Vp.c(), ctx,
+                              B, H_q, H_kv, cap, tau, S, ws.buf, ws.nbytes, err, out,
                               kvq.OUT_FP32)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
