@@ -57,6 +57,7 @@ LLAMA_LAYER = "llama7b_layer_b1_hq32_hkv8_d128_ctx4096"
 PREFILL = "prefill_32layers_b16_t8192_hkv8_d128"
 METRIC = "decode-attn effective HBM GB/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0    # B200 HBM3e, nominal (the measured copy is the roofline)
 SM_COUNT_B200 = 148
 FP32_LANES_PER_SM = 128     # FP32 FMA lanes per SM (4 sub-partitions x 32)
 SM_MAX_MHZ = 1965.0
@@ -497,6 +498,7 @@ def decode_report(state, ms, K, per_launch_ms, hbm_peak, peak_kind, sm_mhz, sm_c
                       "or after an append_kernel launch it hides; time per layer)",
             "bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
             "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} copy bandwidth",
+            "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS,
             "traffic": traffic, "bytes_per_launch": bytes_launch, "us_per_launch": us_launch,
         },
         "roofline_fp32": {
@@ -556,8 +558,10 @@ def time_prefill(device, hbm_peak, reps=3):
         "head_vectors_per_s": n_vec / enc_s,
         "encode_gb_per_s": (fp16 + rows) / enc_s / 1e9,
         "encode_frac": (fp16 + rows) / enc_s / 1e9 / hbm_peak,
+        "encode_frac_of_nominal_8tbs": (fp16 + rows) / enc_s / 1e9 / NOMINAL_HBM_GBS,
         "dequant_gb_per_s": (fp16 + rows) / dq_s / 1e9,
         "dequant_frac": (fp16 + rows) / dq_s / 1e9 / hbm_peak,
+        "dequant_frac_of_nominal_8tbs": (fp16 + rows) / dq_s / 1e9 / NOMINAL_HBM_GBS,
         "ms_per_pass_encode": enc_s * 1e3,
         "ms_per_pass_dequant": dq_s * 1e3,
         "bytes_per_pass": fp16 + rows,
