@@ -28,9 +28,11 @@
 //     all G query heads of the KV head (GQA), so every unpacked code serves G
 //     heads;
 //   - the work per pair is kept to a handful of instructions: a key norm
-//     byte becomes the float 1 + c 2^-15 in one byte permute, and with the
-//     key table holding 2^15 (cos, sin), fma(f, U, -U) is c (cos, sin)
-//     rounded once (no int-to-float conversion); a value norm nibble is
+//     byte becomes the float 1 + c 2^-15 in one byte permute, and with U =
+//     (cos, sin) from the table, fma(f, U, -U) is 2^-15 c (cos, sin)
+//     rounded once (no int-to-float conversion; the exact 2^-15 is undone in
+//     the score scale, and equal K and V codebooks share one table); a value
+//     norm nibble is
 //     or-ed into the mantissa of 1.0 (f = 1 + c/16) and one FMA gives the
 //     exponent LO + c (HI - LO)/15; table bases are folded into the load
 //     address where the tables fit in static shared memory;
@@ -412,10 +414,12 @@ decode_kernel(DecodeArgs A) {
     // table sizes: compile-time for fixed widths (so are the table addresses)
     const int nK = 1 << (BK > 0 ? BK : A.kc.bits), nV = 1 << (BV > 0 ? BV : A.vc.bits);
     unsigned char* dyn = smem + 16 * kMaxStages + 16;
-    // key table: 2^15 (cos, sin) [2^bK][16]; value table: (cos, sin) [2^bV][16]
+    // key table (cos, sin) [2^bK][16], value table (cos, sin) [2^bV][16]
+    // equal codebooks share one dynamic table (the key path uses it unscaled)
+    const bool share = !kStatic && A.kc.L == A.vc.L;
     float2* tabK = kStatic ? s_tab : reinterpret_cast<float2*>(dyn);
-    float2* tabV = tabK + nK * kTabRep;
-    if (!kStatic) dyn += sizeof(float2) * kTabRep * (size_t)(nK + nV);
+    float2* tabV = share ? tabK : tabK + nK * kTabRep;
+    if (!kStatic) dyn += sizeof(float2) * kTabRep * (size_t)(share ? nK : nK + nV);
     float* qs = reinterpret_cast<float*>(dyn);                    // [G][D]
     uint32_t* encst = reinterpret_cast<uint32_t*>(qs + G * D);    // [2][kEncStageWords]
     float* pbuf_all = reinterpret_cast<float*>(encst + 2 * kEncStageWords);  // [WARPS][PBUF]
@@ -546,25 +550,24 @@ decode_kernel(DecodeArgs A) {
     }
 
     // ---- tables and q' (overlap the first copies and the append) -------------
-    // tabV follows tabK, so both tables are one array of nK + nV entries of
-    // kTabRep replicas.  Each bin centre is computed once, into replica 0;
-    // the other replicas are then copied by consecutive threads writing
-    // consecutive addresses (no bank conflicts).
+    // tabV follows tabK (or is tabK), so the tables are one array of nTab
+    // entries of kTabRep replicas.  Each bin centre is computed once, into
+    // replica 0; the other replicas are then copied by consecutive threads
+    // writing consecutive addresses (no bank conflicts).
     if (warp >= w0) {
         const int nthr = CONSUMERS - 32 * w0, t = tid - 32 * w0;
+        const int nTab = tabV == tabK ? nK : nK + nV;
 #pragma unroll 1
-        for (int e = t; e < nK + nV; e += nthr) {
+        for (int e = t; e < nTab; e += nthr) {
             const bool isK = e < nK;
             const int a = isK ? e : e - nK;
             float s, c;
             sincospif((float)(2 * a + 1) / (float)(isK ? A.kc.L : A.vc.L) - 1.f, &s, &c);
-            // key entries scaled by 2^15 (exact): see the norm decoding below
-            const float sc = isK ? 32768.f : 1.f;
-            tabK[e * kTabRep] = make_float2(c * sc, s * sc);
+            tabK[e * kTabRep] = make_float2(c, s);
         }
         named_barrier(2, nthr);
 #pragma unroll 1
-        for (int idx = t; idx < (nK + nV) * kTabRep; idx += nthr)
+        for (int idx = t; idx < nTab * kTabRep; idx += nthr)
             if (idx % kTabRep) tabK[idx] = tabK[idx - idx % kTabRep];
         if (!pending) griddep_wait();
         ctx_in = A.ctx_len[b];
@@ -706,9 +709,10 @@ decode_kernel(DecodeArgs A) {
 #pragma unroll
                     for (int k = 0; k < PP; k++) {
                         // norm byte c -> f = 1 + c 2^-15 (bytes 0x3F 0x80 c 0x00);
-                        // the key table holds U = 2^15 (cos, sin), so
-                        // fma(f, U, -U) = (f - 1) U = c (cos, sin), rounded once;
-                        // the first pair starts the accumulators (no zeroing)
+                        // with U = (cos, sin) from the table, fma(f, U, -U) =
+                        // (f - 1) U = 2^-15 c (cos, sin), rounded once (the
+                        // 2^-15 is exact and undone in the score scale); the
+                        // first pair starts the accumulators (no zeroing)
                         const float f = __uint_as_float(
                             __byte_perm(nw[k / 4], 0x3F800000u, 0x7604u | ((k % 4) << 4)));
                         const float2 U = kTabC ? tab_f2(tabK, off[k]) : lds_f2(off[k]);
@@ -728,7 +732,8 @@ decode_kernel(DecodeArgs A) {
                 for (int e = 0; e < VF; e++) {
                     const int t = blk * TW + ((M + e) / G) * GPW + grp;
                     const float Mk = half_bits_to_float((uint16_t)lds_u16(sKp + 2u * (uint32_t)t));
-                    float sv = part[e] * (Mk * (1.f / 255.f)) * A.scale_log2;
+                    // M/255, times 2^15 for the key products' 2^-15
+                    float sv = part[e] * (Mk * (32768.f / 255.f)) * A.scale_log2;
                     sv = t < ntok ? sv : -INFINITY;
                     part[e] = sv;
                     need |= sv > mh[e] + kLazyThr;
@@ -1105,8 +1110,9 @@ template <int D, int G, int BK, int BV, int CTAS, int TT>
 inline size_t decode_smem_plan(DecodeArgs& a, size_t avail, int min_stages) {
     using Cfg = DecCfg<D, G, CTAS, TT>;
     size_t off = 16 * kMaxStages + 16;
-    if (!decode_static_tables(BK, BV))
-        off += sizeof(float2) * kTabRep * (size_t)((1 << a.kc.bits) + (1 << a.vc.bits));
+    if (!decode_static_tables(BK, BV))  // one table when the codebooks are equal
+        off += sizeof(float2) * kTabRep *
+               (size_t)(a.kc.L == a.vc.L ? (1 << a.kc.bits) : (1 << a.kc.bits) + (1 << a.vc.bits));
     off += sizeof(float) * G * D + sizeof(uint32_t) * 2 * kEncStageWords +
            sizeof(float) * Cfg::WARPS * Cfg::PBUF;
     off = (off + 15) / 16 * 16;
