@@ -199,14 +199,16 @@ dequant_fast_kernel(DqArgs A) {
     extern __shared__ float2 tab[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int grp = lane / NL, lg = lane % NL;
+    // 2^B entries, so that any B-bit pattern indexes inside the table (codes
+    // of a valid cache are below L)
     const int L = A.c.L;
-    for (int j = threadIdx.x; j < L; j += blockDim.x) {
+    for (int j = threadIdx.x; j < (1 << B); j += blockDim.x) {
         float sn, cs;
         sincospif((float)(2 * j + 1) / (float)L - 1.f, &sn, &cs);
         tab[j * 16] = make_float2(cs + sn, cs - sn);
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < L * 16; i += blockDim.x)
+    for (int i = threadIdx.x; i < (16 << B); i += blockDim.x)
         if (i & 15) tab[i] = tab[i & ~15];
     uint32_t m[16];  // fp16 sign bits of D for this lane's element pairs
 #pragma unroll
@@ -317,7 +319,7 @@ static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStre
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     const dim3 g((unsigned)blocks), b(kDqWarps * 32);
-    const size_t smem = (size_t)a.c.L * 16 * sizeof(float2);  // at most 32 KB
+    const size_t smem = ((size_t)16 << a.c.bits) * sizeof(float2);  // at most 32 KB
     switch (a.c.bits) {
         case 1: dequant_fast_kernel<D, 1><<<g, b, smem, stream>>>(a); break;
         case 2: dequant_fast_kernel<D, 2><<<g, b, smem, stream>>>(a); break;
