@@ -80,9 +80,11 @@ __device__ __forceinline__ float gen_norm(const CodecDev& c, const uint8_t* norm
     return exp2f(fmaf(code, prm.y, prm.x));
 }
 
-// Bin centre of code a: (cos, sin) of -pi + (a + 1/2) 2 pi / L.
+// Bin centre of code a: (cos, sin) of -pi + (a + 1/2) 2 pi / L.  A code of
+// L or more (never written by the encoder; KVQ_DEBUG reports it) reads entry
+// 0 rather than past the table.
 __device__ __forceinline__ float2 gen_centre(const float2* tab, uint32_t a, int L) {
-    if (L <= kGenTabMax) return tab[a];
+    if (L <= kGenTabMax) return tab[a < (uint32_t)L ? a : 0u];
     float s, c;
     sincospif((float)(2 * (int)a + 1) / (float)L - 1.f, &s, &c);
     return make_float2(c, s);
