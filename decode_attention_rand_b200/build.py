@@ -24,7 +24,7 @@ ROOT = os.path.dirname(HERE)
 OUT = os.path.join(HERE, "libkvq.so")
 BUILD = os.path.join(ROOT, "_build")
 SOURCES = ["kvq_abi.cu", "kvq_encode.cu", "kvq_dequant.cu", "kvq_decode.cu", "kvq_noalloc.cu",
-           "kvq_decode_generic.cu", "kvq_debug.cu"] + [
+           "kvq_decode_generic.cu", "kvq_debug.cu", "kvq_shard.cu"] + [
     f"kvq_decode_d{d}_g{g}.cu" for d in (64, 128) for g in (1, 2, 4, 8)]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -352,7 +352,7 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
                 float softmax_scale, int32_t num_splits, void* workspace, int64_t ws_bytes,
                 int32_t* err_word, void* out, int32_t out_dtype, void* stream,
                 const kvq_paged_plane* PK = nullptr, const kvq_paged_plane* PV = nullptr,
-                const HostIO* hio = nullptr) {
+                const HostIO* hio = nullptr, bool partials = false) {
     char wk[64], wv[64];
     snprintf(wk, sizeof(wk), "%s (K)", what);
     snprintf(wv, sizeof(wv), "%s (V)", what);
@@ -389,7 +389,7 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
         return fail(KVQ_EINVAL, "%s: workspace of %lld bytes is below the %lld needed", what,
                     (long long)ws_bytes, (long long)need);
     if (!aligned16(workspace)) return fail(KVQ_EINVAL, "%s: workspace not 16-byte aligned", what);
-    if (!q || !signs_k || !signs_v || !ctx_len || !out)
+    if (!q || !signs_k || !signs_v || !ctx_len || (!out && !partials))
         return fail(KVQ_EINVAL, "%s: NULL q, signs, ctx_len or out", what);
     a.q = static_cast<const __half*>(q);
     a.signs_k = signs_k;
@@ -415,6 +415,7 @@ int decode_impl(const char* what, const void* q, const void* k_new, const void* 
     a.err_word = err_word;
     a.out = out;
     a.out_dtype = out_dtype;
+    a.partials_only = partials ? 1 : 0;
     a.k_new = static_cast<const __half*>(k_new);
     a.v_new = static_cast<const __half*>(v_new);
     if (k_new) {
@@ -455,6 +456,47 @@ int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc, con
     return decode_impl("kvq_decode_attn", q, nullptr, nullptr, kc, vc, signs_k, signs_v, K, V,
                        ctx_len, B, H_q, H_kv, max_ctx, softmax_scale, num_splits, workspace,
                        ws_bytes, err_word, out, out_dtype, stream);
+}
+
+int kvq_decode_attn_partials(const void* q, const kvq_codec* kc, const kvq_codec* vc,
+                             const int8_t* signs_k, const int8_t* signs_v, const kvq_plane* K,
+                             const kvq_plane* V, const int32_t* ctx_len, int32_t B, int32_t H_q,
+                             int32_t H_kv, int64_t max_ctx, float softmax_scale,
+                             int32_t num_splits, void* workspace, int64_t ws_bytes,
+                             int32_t* err_word, void* stream) {
+    return decode_impl("kvq_decode_attn_partials", q, nullptr, nullptr, kc, vc, signs_k, signs_v,
+                       K, V, ctx_len, B, H_q, H_kv, max_ctx, softmax_scale, num_splits,
+                       workspace, ws_bytes, err_word, nullptr, 1, stream, nullptr, nullptr,
+                       nullptr, true);
+}
+
+int kvq_decode_merge_partials(const void* parts, int32_t n_parts, int32_t B, int32_t H_q,
+                              int32_t head_dim, int32_t num_splits, const int8_t* signs_v,
+                              void* out, int32_t out_dtype, void* stream) {
+    const char* what = "kvq_decode_merge_partials";
+    if (n_parts < 1 || n_parts > 4096)
+        return fail(KVQ_EINVAL, "%s: n_parts %d outside 1..4096", what, n_parts);
+    if (B < 0 || H_q < 0) return fail(KVQ_EINVAL, "%s: negative size", what);
+    if (head_dim < 4 || head_dim > 256 || (head_dim & (head_dim - 1)))
+        return fail(KVQ_EINVAL, "%s: head_dim %d is not a power of two in 4..256", what,
+                    head_dim);
+    if (num_splits < 1 || num_splits > 65535)
+        return fail(KVQ_EINVAL, "%s: num_splits %d outside 1..65535", what, num_splits);
+    if ((int64_t)n_parts * num_splits > 16384)
+        return fail(KVQ_EINVAL, "%s: n_parts x num_splits above 16384", what);
+    if (out_dtype != 0 && out_dtype != 1)
+        return fail(KVQ_EINVAL, "%s: out_dtype must be 0 (fp16) or 1 (fp32)", what);
+    if (B == 0 || H_q == 0) return ok();
+    if (!parts || !signs_v || !out) return fail(KVQ_EINVAL, "%s: NULL parts, signs or out", what);
+    if (!aligned16(parts)) return fail(KVQ_EINVAL, "%s: parts not 16-byte aligned", what);
+    const int64_t part_floats = kvq_decode_workspace_bytes(B, H_q, head_dim, num_splits) / 4;
+    if (injected_failure()) return injected(what);
+    kvq::ProfileRange range(what);
+    return cuda_status(kvq::launch_merge_partials(static_cast<const float*>(parts), n_parts,
+                                                  part_floats, B, H_q, head_dim, num_splits,
+                                                  signs_v, out, out_dtype,
+                                                  static_cast<cudaStream_t>(stream)),
+                       what);
 }
 
 int kvq_decode_step(const void* q, const void* k_new, const void* v_new, const kvq_codec* kc,

@@ -294,6 +294,9 @@ decode_generic_kernel(DecodeArgs A, int chunks) {
         }
     }
 
+    // partials only (kvq_decode_attn_partials): the caller merges them
+    if (A.partials_only) return;
+
     // ---- the last CTA of this (b, KV head, chunk) merges the splits ----------
     __threadfence();
     __syncthreads();

@@ -1026,6 +1026,9 @@ decode_kernel(DecodeArgs A) {
         return;
     }
 
+    // partials only (kvq_decode_attn_partials): the caller merges them
+    if (A.partials_only) return;
+
     // ---- the last CTA of this (b, KV head) merges the splits ----------------
     __threadfence();
     __syncthreads();
@@ -1219,7 +1222,8 @@ inline cudaError_t launch_decode_kernel(DecodeArgs a, cudaStream_t stream, int m
     // occupancy calculator rather than count SMs
     const int S = a.num_splits;
     a.cluster = 0;
-    if (S <= kMaxClusterSplits && (int64_t)a.B * a.H_kv * S <= (int64_t)sm_count) {
+    if (S <= kMaxClusterSplits && !a.partials_only &&
+        (int64_t)a.B * a.H_kv * S <= (int64_t)sm_count) {
         int n = -1;
         {
             std::lock_guard<std::mutex> g(cache.lock);

@@ -83,6 +83,9 @@ struct DecodeArgs {
     // reads q and ctx_len at once and waits for the append (griddepcontrol)
     // only before copying in the tile that holds the new row
     int append_pending;
+    // 1 (kvq_decode_attn_partials): stop after the per-split partials are in
+    // the workspace; no combine, no output (cluster is 0)
+    int partials_only;
     const __half* k_new;     // [B][H_kv][d] or NULL (no append)
     const __half* v_new;     // [B][H_kv][d]
     EncArgs enc_k, enc_v;    // codec, signs and constants of the two encodes
@@ -93,6 +96,11 @@ struct DecodeArgs {
 bool decode_fast_supported(int d, int G, int LK, int LV, int mode_k, int mode_v);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+// Merge of the split partials of n_parts workspaces laid out back to back
+// (kvq_decode_merge_partials): out[b][h] from every part's splits.
+cudaError_t launch_merge_partials(const float* parts, int n_parts, int64_t part_floats, int B,
+                                  int H_q, int d, int S, const int8_t* signs_v, void* out,
+                                  int out_dtype, cudaStream_t stream);
 cudaError_t launch_decode_generic(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d64_g1(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_d64_g2(const DecodeArgs& a, cudaStream_t stream);

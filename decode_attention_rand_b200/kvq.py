@@ -109,6 +109,15 @@ _SIGNATURES = {
                                   C.POINTER(kvq_plane), C.c_void_p, C.c_int32, C.c_int32,
                                   C.c_int32, C.c_int64, C.c_float, C.c_int32, C.c_void_p,
                                   C.c_int64, C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p]),
+    "kvq_decode_attn_partials": (C.c_int, [C.c_void_p, C.POINTER(kvq_codec),
+                                           C.POINTER(kvq_codec), C.c_void_p, C.c_void_p,
+                                           C.POINTER(kvq_plane), C.POINTER(kvq_plane),
+                                           C.c_void_p, C.c_int32, C.c_int32, C.c_int32,
+                                           C.c_int64, C.c_float, C.c_int32, C.c_void_p,
+                                           C.c_int64, C.c_void_p, C.c_void_p]),
+    "kvq_decode_merge_partials": (C.c_int, [C.c_void_p, C.c_int32, C.c_int32, C.c_int32,
+                                            C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                                            C.c_int32, C.c_void_p]),
 }
 
 
@@ -300,6 +309,23 @@ def kvq_decode_step_paged(q, k_new, v_new, kc: kvq_codec, vc: kvq_codec, signs_k
                                        C.byref(V), _ptr(ctx_len), B, H_q, H_kv, max_ctx,
                                        softmax_scale, num_splits, _ptr(workspace), ws_bytes,
                                        _ptr(err_word), _ptr(out), out_dtype, _stream(stream)))
+
+
+def kvq_decode_attn_partials(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: kvq_plane,
+                             V: kvq_plane, ctx_len, B: int, H_q: int, H_kv: int, max_ctx: int,
+                             softmax_scale: float, num_splits: int, workspace, ws_bytes: int,
+                             err_word=None, stream=None):
+    _check(lib().kvq_decode_attn_partials(_ptr(q), C.byref(kc), C.byref(vc), _ptr(signs_k),
+                                          _ptr(signs_v), C.byref(K), C.byref(V), _ptr(ctx_len),
+                                          B, H_q, H_kv, max_ctx, softmax_scale, num_splits,
+                                          _ptr(workspace), ws_bytes, _ptr(err_word),
+                                          _stream(stream)))
+
+
+def kvq_decode_merge_partials(parts, n_parts: int, B: int, H_q: int, head_dim: int,
+                              num_splits: int, signs_v, out, out_dtype: int, stream=None):
+    _check(lib().kvq_decode_merge_partials(_ptr(parts), n_parts, B, H_q, head_dim, num_splits,
+                                           _ptr(signs_v), _ptr(out), out_dtype, _stream(stream)))
 
 
 def kvq_decode_attn(q, kc: kvq_codec, vc: kvq_codec, signs_k, signs_v, K: kvq_plane,

@@ -270,6 +270,46 @@ int kvq_decode_attn(const void* q, const kvq_codec* kc, const kvq_codec* vc,
                     int32_t* err_word, void* out, int32_t out_dtype,
                     void* stream);
 
+/* Context-sharded decode, part 1: kvq_decode_attn over the tokens this GPU
+ * holds, stopped before the combine.  When a sequence's cached context is
+ * spread over several GPUs (each plane holding a range of its tokens, its own
+ * ctx_len counting the tokens held here), each GPU runs this call on its
+ * planes; the workspace then holds, at the offsets that
+ * kvq_decode_workspace_bytes describes, per (b, query head, split) the
+ * running maximum m (log2 units: the scores times softmax_scale times log2 e,
+ * -inf for a split with no token), the denominator l = sum 2^(s - m) and the
+ * accumulator sum 2^(s - m) z^_V in the rotated domain.  These are the
+ * partials of the split combine that kvq_decode_attn performs (the softmax
+ * and value formulas of "Decode attention" above); merging them across GPUs
+ * gives the same result.  Arguments and checks as for kvq_decode_attn, with
+ * no output; the completion counters are not touched.  All GPUs of one merge
+ * use the same B, H_q, head_dim and num_splits. */
+int kvq_decode_attn_partials(const void* q, const kvq_codec* kc,
+                             const kvq_codec* vc, const int8_t* signs_k,
+                             const int8_t* signs_v, const kvq_plane* K,
+                             const kvq_plane* V, const int32_t* ctx_len,
+                             int32_t B, int32_t H_q, int32_t H_kv,
+                             int64_t max_ctx, float softmax_scale,
+                             int32_t num_splits, void* workspace,
+                             int64_t ws_bytes, int32_t* err_word,
+                             void* stream);
+
+/* Context-sharded decode, part 2: merge the partials of n_parts workspaces
+ * (each kvq_decode_workspace_bytes(B, H_q, head_dim, num_splits) bytes, laid
+ * out back to back in `parts`, e.g. after an all-gather) into the attention
+ * output: M = max m, L = sum l 2^(m - M), z = sum acc 2^(m - M) / L over
+ * every part and split, then o = D_V H z / sqrt(d), as the single-GPU
+ * combine does.
+ *   parts    device, 16-byte aligned, n_parts x workspace bytes
+ *   signs_v  device int8 [head_dim], the V diagonal
+ *   out      device fp16 or fp32 [B][H_q][head_dim]
+ * head_dim a power of two in 4..256; 1 <= n_parts <= 4096 with n_parts x
+ * num_splits <= 16384; a (b, head) whose parts hold no token gives 0. */
+int kvq_decode_merge_partials(const void* parts, int32_t n_parts, int32_t B,
+                              int32_t H_q, int32_t head_dim,
+                              int32_t num_splits, const int8_t* signs_v,
+                              void* out, int32_t out_dtype, void* stream);
+
 /* One decode step of one layer in one kernel: the append of each sequence's
  * new token fused into kvq_decode_attn.  For every b with 1 <= ctx_len[b]
  * <= min(max_ctx, capacity), the token at position ctx_len[b] - 1 of every
