@@ -216,10 +216,10 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs,
                 int64_t pos0, void* y, void* stream);
 
 /* Split count the library would choose for a decode launch (host logic,
- * deterministic).  One CTA per SM streams tiles of about 128 tokens and
- * pays a fixed cost of about three tiles; the split count minimises
- * waves x (tiles per CTA + 3) over at most eight waves on sm_count SMs,
- * the fewer CTAs on ties.  At least 1, at most ceil(max_ctx / 128). */
+ * deterministic).  Its cost model: one CTA per SM, a CTA's time is its
+ * 128-token units plus a fixed cost of about three units; the split count
+ * minimises waves x (units per CTA + 3) over at most eight waves on sm_count
+ * SMs, the fewer CTAs on ties.  At least 1, at most ceil(max_ctx / 128). */
 int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx,
                               int32_t sm_count);
 
@@ -310,8 +310,8 @@ int kvq_decode_merge_partials(const void* parts, int32_t n_parts, int32_t B,
                               int32_t num_splits, const int8_t* signs_v,
                               void* out, int32_t out_dtype, void* stream);
 
-/* One decode step of one layer in one kernel: the append of each sequence's
- * new token fused into kvq_decode_attn.  For every b with 1 <= ctx_len[b]
+/* One decode step of one layer, normally in one kernel: the append of each
+ * sequence's new token fused into kvq_decode_attn.  For every b with 1 <= ctx_len[b]
  * <= min(max_ctx, capacity), the token at position ctx_len[b] - 1 of every
  * KV head is first written as
  *   kvq_encode_kv(kc, signs_k, k_new[b], K, vc, signs_v, v_new[b], V, ...)
@@ -321,8 +321,9 @@ int kvq_decode_merge_partials(const void* parts, int32_t n_parts, int32_t B,
  * attends from codes; doing both in one launch is this library's choice:
  * the split that holds the new token encodes it while its first tiles are
  * in flight, the other splits never wait for it.  (For codecs the staged
- * kernel does not take, see kvq_decode_attn, the append is its own small
- * launch just before the decode, with the same results.)
+ * kernel does not take, see kvq_decode_attn, and for multi-wave launches on
+ * paged caches, the append is its own small launch just before the decode,
+ * which waits for it only before reading the new row; same results.)
  *   k_new, v_new  device fp16 [B][H_kv][head_dim], 16-byte aligned
  * Everything else as for kvq_decode_attn.  A ctx_len outside the range
  * above appends nothing (and is clipped and reported as there). */
