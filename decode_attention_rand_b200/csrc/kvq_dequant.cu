@@ -188,6 +188,25 @@ struct DqFastCfg {
 
 constexpr int kDqFastBlocksPerSM = 3;  // registers for one tile ahead in flight
 
+// The tail is transposed: after the in-lane butterfly stages, the lanes of a
+// vector exchange their elements through shared memory instead of shuffles,
+// so that the stages over the lane index bits run in registers: lane l then
+// holds, for every original lane index Lh, the run of RL = 32 / NL elements
+// starting at Lh 32 + l RL, and stores it as 16-byte (8-byte for d = 256)
+// words.  The exchange writes 16-byte chunks with a rotation of K = 8 / NL
+// chunks per lane and rows of d / 4 + 1 chunks (one chunk of padding, so a
+// row starts one bank group after the previous one); neither its writes nor
+// its reads then share a bank group within a quarter warp.
+template <int D>
+struct DqTrCfg {
+    static constexpr int NL = D / 32;
+    static constexpr int RL = 32 / NL;       // elements per run after the exchange
+    static constexpr int K = 8 / NL;         // chunk rotation per lane
+    static constexpr int ROWC = D / 4 + 1;   // 16-byte chunks per vector row
+    static constexpr int VPW = 32 / NL;
+    static constexpr int WARP_CHUNKS = VPW * ROWC;
+};
+
 template <int D, int B>
 __global__ void __launch_bounds__(kDqWarps * 32, kDqFastBlocksPerSM)
 dequant_fast_kernel(DqArgs A) {
@@ -210,12 +229,17 @@ dequant_fast_kernel(DqArgs A) {
     __syncthreads();
     for (int i = threadIdx.x; i < (16 << B); i += blockDim.x)
         if (i & 15) tab[i] = tab[i & ~15];
-    uint32_t m[16];  // fp16 sign bits of D for this lane's element pairs
+    uint32_t m[16];  // fp16 sign bits of D for this lane's output element pairs
 #pragma unroll
     for (int w = 0; w < 16; w++) {
-        const int e = lg * 32 + 2 * w;
+        // pair w is pair w % (RL / 2) of run w / (RL / 2)
+        const int e = (w / (DqTrCfg<D>::RL / 2)) * 32 + lg * DqTrCfg<D>::RL +
+                      2 * (w % (DqTrCfg<D>::RL / 2));
         m[w] = (A.signs[e] < 0 ? 0x8000u : 0u) | (A.signs[e + 1] < 0 ? 0x80000000u : 0u);
     }
+    // exchange buffer, after the table: [warp][vector][d / 4 + 1 chunks]
+    uint4* xbuf = reinterpret_cast<uint4*>(tab + (16 << B)) +
+                  (size_t)warp * DqTrCfg<D>::WARP_CHUNKS + (size_t)grp * DqTrCfg<D>::ROWC;
     __syncthreads();
     const float2* tl = tab + (lane & 15);
     const int AW = A.c.angle_words;
@@ -292,7 +316,42 @@ dequant_fast_kernel(DqArgs A) {
             const float2 t = tl[a * 16];
             P[k] = pack2(r[k] * t.x, r[k] * t.y);
         }
-        fwht_pairs<NL>(P, lg);
+        using T = DqTrCfg<D>;
+        fwht_pairs<1>(P, lg);  // the in-lane stages
+        // chunk q of this lane = pairs 2q, 2q + 1 = elements lg 32 + 4q .. + 3
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 8; q++)
+            xbuf[lg * 8 + ((q + T::K * lg) & 7)] =
+                make_uint4((uint32_t)P[2 * q], (uint32_t)(P[2 * q] >> 32),
+                           (uint32_t)P[2 * q + 1], (uint32_t)(P[2 * q + 1] >> 32));
+        __syncwarp();
+        // run Lh: chunks lg RL / 4 + h of the lane Lh that wrote them
+#pragma unroll
+        for (int Lh = 0; Lh < NL; Lh++) {
+#pragma unroll
+            for (int h = 0; h < T::RL / 4; h++) {
+                const int qw = lg * (T::RL / 4) + h;
+                const uint4 c = xbuf[Lh * 8 + ((qw + T::K * Lh) & 7)];
+                P[Lh * (T::RL / 2) + 2 * h] = ((f32x2)c.y << 32) | c.x;
+                P[Lh * (T::RL / 2) + 2 * h + 1] = ((f32x2)c.w << 32) | c.z;
+            }
+        }
+        // the stages over the former lane bits, now in registers
+#pragma unroll
+        for (int st = 1; st < NL; st <<= 1) {
+#pragma unroll
+            for (int Lh = 0; Lh < NL; Lh++) {
+                if ((Lh & st) == 0) {
+#pragma unroll
+                    for (int u = 0; u < T::RL / 2; u++) {
+                        const f32x2 a = P[Lh * (T::RL / 2) + u], b = P[(Lh + st) * (T::RL / 2) + u];
+                        P[Lh * (T::RL / 2) + u] = add2(a, b);
+                        P[(Lh + st) * (T::RL / 2) + u] = sub2(a, b);
+                    }
+                }
+            }
+        }
         if (valid) {
             uint32_t o[16];
 #pragma unroll
@@ -300,10 +359,19 @@ dequant_fast_kernel(DqArgs A) {
                 const __half2 h = __floats2half2_rn(lo2(P[k]), hi2(P[k]));
                 o[k] = *reinterpret_cast<const uint32_t*>(&h) ^ m[k];
             }
-            uint4* dst = reinterpret_cast<uint4*>(A.y + (size_t)v * D + lg * 32);
+            __half* y = A.y + (size_t)v * D + lg * T::RL;
 #pragma unroll
-            for (int q = 0; q < 4; q++)
-                dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            for (int Lh = 0; Lh < NL; Lh++) {
+                const uint32_t* oo = o + Lh * (T::RL / 2);
+                if constexpr (T::RL == 4) {
+                    *reinterpret_cast<uint2*>(y + Lh * 32) = make_uint2(oo[0], oo[1]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < T::RL / 8; c++)
+                        reinterpret_cast<uint4*>(y + Lh * 32)[c] =
+                            make_uint4(oo[4 * c], oo[4 * c + 1], oo[4 * c + 2], oo[4 * c + 3]);
+                }
+            }
         }
     }
 }
@@ -319,18 +387,23 @@ static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStre
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     const dim3 g((unsigned)blocks), b(kDqWarps * 32);
-    const size_t smem = ((size_t)16 << a.c.bits) * sizeof(float2);  // at most 32 KB
+    // table (at most 32 KB) + exchange buffer (33 to 35 KB)
+    const size_t smem = ((size_t)16 << a.c.bits) * sizeof(float2) +
+                        sizeof(uint4) * kDqWarps * DqTrCfg<D>::WARP_CHUNKS;
+#define KVQ_DQ(BB)                                                                          \
+    case BB: {                                                                              \
+        const cudaError_t e = cudaFuncSetAttribute(                                         \
+            dequant_fast_kernel<D, BB>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
+            (int)smem);                                                                     \
+        if (e != cudaSuccess) return e;                                                     \
+        dequant_fast_kernel<D, BB><<<g, b, smem, stream>>>(a);                              \
+        break;                                                                              \
+    }
     switch (a.c.bits) {
-        case 1: dequant_fast_kernel<D, 1><<<g, b, smem, stream>>>(a); break;
-        case 2: dequant_fast_kernel<D, 2><<<g, b, smem, stream>>>(a); break;
-        case 3: dequant_fast_kernel<D, 3><<<g, b, smem, stream>>>(a); break;
-        case 4: dequant_fast_kernel<D, 4><<<g, b, smem, stream>>>(a); break;
-        case 5: dequant_fast_kernel<D, 5><<<g, b, smem, stream>>>(a); break;
-        case 6: dequant_fast_kernel<D, 6><<<g, b, smem, stream>>>(a); break;
-        case 7: dequant_fast_kernel<D, 7><<<g, b, smem, stream>>>(a); break;
-        case 8: dequant_fast_kernel<D, 8><<<g, b, smem, stream>>>(a); break;
+        KVQ_DQ(1) KVQ_DQ(2) KVQ_DQ(3) KVQ_DQ(4) KVQ_DQ(5) KVQ_DQ(6) KVQ_DQ(7) KVQ_DQ(8)
         default: return cudaErrorInvalidValue;
     }
+#undef KVQ_DQ
     return cudaGetLastError();
 }
 
