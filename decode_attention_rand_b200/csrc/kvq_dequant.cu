@@ -193,19 +193,30 @@ constexpr int kDqFastBlocksPerSM = 3;  // registers for one tile ahead in flight
 // so that the stages over the lane index bits run in registers: lane l then
 // holds, for every original lane index Lh, the run of RL = 32 / NL elements
 // starting at Lh 32 + l RL, and stores it as 16-byte (8-byte for d = 256)
-// words.  The exchange writes 16-byte chunks with a rotation of K = 8 / NL
-// chunks per lane and rows of d / 4 + 1 chunks (one chunk of padding, so a
-// row starts one bank group after the previous one); neither its writes nor
-// its reads then share a bank group within a quarter warp.
+// words.  Lane (g, l) of vector g writes its 16-byte chunk q to slot
+// q ^ f(g, l) of its 8-chunk block, f(g, l) = l K + (g mod K) with
+// K = 8 / NL; a quarter warp (K vectors of NL lanes) then covers all eight
+// bank groups, on the writes and on the reads (chunk l K + h of the block of
+// lane Lh sits in slot (l ^ Lh) K + (h ^ (g mod K))).  On a 128-byte aligned
+// block both addresses are a per-lane base XOR a constant.
 template <int D>
 struct DqTrCfg {
     static constexpr int NL = D / 32;
     static constexpr int RL = 32 / NL;       // elements per run after the exchange
-    static constexpr int K = 8 / NL;         // chunk rotation per lane
-    static constexpr int ROWC = D / 4 + 1;   // 16-byte chunks per vector row
-    static constexpr int VPW = 32 / NL;
-    static constexpr int WARP_CHUNKS = VPW * ROWC;
+    static constexpr int K = 8 / NL;         // runs of 16 bytes a lane reads per block
+    static constexpr int WARP_BYTES = 32 * 8 * 16;
 };
+
+// One 16-byte chunk of the exchange, moved as a single 128-bit shared-memory
+// access: two 64-bit loads would each be served per half warp, where the
+// chunk rotation does not keep the banks apart.  The "memory" clobbers keep
+// the accesses on their side of the __syncwarp()s around the exchange.
+__device__ __forceinline__ void xch_store(uint32_t addr, f32x2 a, f32x2 b) {
+    asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(addr), "l"(a), "l"(b) : "memory");
+}
+__device__ __forceinline__ void xch_load(uint32_t addr, f32x2& a, f32x2& b) {
+    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr) : "memory");
+}
 
 template <int D, int B>
 __global__ void __launch_bounds__(kDqWarps * 32, kDqFastBlocksPerSM)
@@ -237,9 +248,14 @@ dequant_fast_kernel(DqArgs A) {
                       2 * (w % (DqTrCfg<D>::RL / 2));
         m[w] = (A.signs[e] < 0 ? 0x8000u : 0u) | (A.signs[e + 1] < 0 ? 0x80000000u : 0u);
     }
-    // exchange buffer, after the table: [warp][vector][d / 4 + 1 chunks]
-    uint4* xbuf = reinterpret_cast<uint4*>(tab + (16 << B)) +
-                  (size_t)warp * DqTrCfg<D>::WARP_CHUNKS + (size_t)grp * DqTrCfg<D>::ROWC;
+    // exchange buffer after the table, 128-byte aligned: [warp][vector][lane][8 chunks]
+    using T = DqTrCfg<D>;
+    const uint32_t xrow =
+        (((uint32_t)__cvta_generic_to_shared(tab + (16 << B)) + 127u) & ~127u) +
+        (uint32_t)(warp * T::WARP_BYTES + grp * D * 4);
+    const uint32_t xsw = (uint32_t)(lg * T::K + grp % T::K) << 4;
+    const uint32_t xw = xrow + lg * 128 + xsw;  // chunk q goes to xw ^ (q << 4)
+    const uint32_t xr = xrow | xsw;             // run Lh, chunk h: (xr ^ ((Lh K + h) << 4)) + Lh 128
     __syncthreads();
     const float2* tl = tab + (lane & 15);
     const int AW = A.c.angle_words;
@@ -316,25 +332,20 @@ dequant_fast_kernel(DqArgs A) {
             const float2 t = tl[a * 16];
             P[k] = pack2(r[k] * t.x, r[k] * t.y);
         }
-        using T = DqTrCfg<D>;
         fwht_pairs<1>(P, lg);  // the in-lane stages
         // chunk q of this lane = pairs 2q, 2q + 1 = elements lg 32 + 4q .. + 3
         __syncwarp();
 #pragma unroll
         for (int q = 0; q < 8; q++)
-            xbuf[lg * 8 + ((q + T::K * lg) & 7)] =
-                make_uint4((uint32_t)P[2 * q], (uint32_t)(P[2 * q] >> 32),
-                           (uint32_t)P[2 * q + 1], (uint32_t)(P[2 * q + 1] >> 32));
+            xch_store(xw ^ (q << 4), P[2 * q], P[2 * q + 1]);
         __syncwarp();
-        // run Lh: chunks lg RL / 4 + h of the lane Lh that wrote them
+        // run Lh: chunks lg K + h of the block of lane Lh
 #pragma unroll
         for (int Lh = 0; Lh < NL; Lh++) {
 #pragma unroll
             for (int h = 0; h < T::RL / 4; h++) {
-                const int qw = lg * (T::RL / 4) + h;
-                const uint4 c = xbuf[Lh * 8 + ((qw + T::K * Lh) & 7)];
-                P[Lh * (T::RL / 2) + 2 * h] = ((f32x2)c.y << 32) | c.x;
-                P[Lh * (T::RL / 2) + 2 * h + 1] = ((f32x2)c.w << 32) | c.z;
+                xch_load((xr ^ ((Lh * T::K + h) << 4)) + Lh * 128, P[Lh * (T::RL / 2) + 2 * h],
+                         P[Lh * (T::RL / 2) + 2 * h + 1]);
             }
         }
         // the stages over the former lane bits, now in registers
@@ -387,9 +398,9 @@ static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStre
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     const dim3 g((unsigned)blocks), b(kDqWarps * 32);
-    // table (at most 32 KB) + exchange buffer (33 to 35 KB)
-    const size_t smem = ((size_t)16 << a.c.bits) * sizeof(float2) +
-                        sizeof(uint4) * kDqWarps * DqTrCfg<D>::WARP_CHUNKS;
+    // table (at most 32 KB) + exchange buffer (32 KB) and its alignment
+    const size_t smem = ((size_t)16 << a.c.bits) * sizeof(float2) + 128 +
+                        (size_t)kDqWarps * DqTrCfg<D>::WARP_BYTES;
 #define KVQ_DQ(BB)                                                                          \
     case BB: {                                                                              \
         const cudaError_t e = cudaFuncSetAttribute(                                         \
