@@ -225,8 +225,10 @@ dequant_fast_kernel(DqArgs A) {
     constexpr int NL = Cfg::NL, VPW = Cfg::VPW, S = Cfg::S;
     // r-free (cos + sin, cos - sin) of each bin centre, 16 copies side by side
     // ([code][16]): lane l of a half warp reads copy l, so a lookup never
-    // shares a bank within the half warp
-    extern __shared__ float2 tab[];
+    // shares a bank within the half warp.  A static array: its base is a
+    // compile-time address that the lookups carry in the load's immediate.
+    __shared__ __align__(128) float2 tab[16 << B];
+    extern __shared__ __align__(16) unsigned char xdyn[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int grp = lane / NL, lg = lane % NL;
     // 2^B entries, so that any B-bit pattern indexes inside the table (codes
@@ -251,13 +253,14 @@ dequant_fast_kernel(DqArgs A) {
     // exchange buffer after the table, 128-byte aligned: [warp][vector][lane][8 chunks]
     using T = DqTrCfg<D>;
     const uint32_t xrow =
-        (((uint32_t)__cvta_generic_to_shared(tab + (16 << B)) + 127u) & ~127u) +
+        (((uint32_t)__cvta_generic_to_shared(xdyn) + 127u) & ~127u) +
         (uint32_t)(warp * T::WARP_BYTES + grp * D * 4);
     const uint32_t xsw = (uint32_t)(lg * T::K + grp % T::K) << 4;
     const uint32_t xw = xrow + lg * 128 + xsw;  // chunk q goes to xw ^ (q << 4)
     const uint32_t xr = xrow | xsw;             // run Lh, chunk h: (xr ^ ((Lh K + h) << 4)) + Lh 128
     __syncthreads();
-    const float2* tl = tab + (lane & 15);
+    // byte offset of the lane's replica (code c's entries span 128 bytes)
+    const uint32_t tlo = (uint32_t)(lane & 15) * sizeof(float2);
     const int AW = A.c.angle_words;
     const bool lin8 = A.c.mode == KVQ_NORM_LIN8;
     const float isd = A.inv_sqrt_d;
@@ -326,10 +329,15 @@ dequant_fast_kernel(DqArgs A) {
         f32x2 P[16];
 #pragma unroll
         for (int k = 0; k < 16; k++) {
-            constexpr uint32_t mask = (1u << B) - 1u;
+            // code k moved to bits 7 .. 7 + B - 1 (times 128 bytes), the
+            // replica offset or-ed in below them
+            constexpr uint32_t mask = ((1u << B) - 1u) << 7;
             const int pos = k * B, wi = pos >> 5, bi = pos & 31;
-            const uint32_t a = (bi + B <= 32 ? (W[wi] >> bi) : __funnelshift_r(W[wi], W[wi + 1], bi)) & mask;
-            const float2 t = tl[a * 16];
+            const uint32_t x = bi + B > 32 ? __funnelshift_r(W[wi], W[wi + 1], bi - 7)
+                               : bi >= 7   ? W[wi] >> (bi - 7)
+                                           : W[wi] << (7 - bi);
+            const float2 t =
+                *reinterpret_cast<const float2*>(reinterpret_cast<const char*>(tab) + ((x & mask) | tlo));
             P[k] = pack2(r[k] * t.x, r[k] * t.y);
         }
         fwht_pairs<1>(P, lg);  // the in-lane stages
@@ -398,9 +406,9 @@ static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStre
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     const dim3 g((unsigned)blocks), b(kDqWarps * 32);
-    // table (at most 32 KB) + exchange buffer (32 KB) and its alignment
-    const size_t smem = ((size_t)16 << a.c.bits) * sizeof(float2) + 128 +
-                        (size_t)kDqWarps * DqTrCfg<D>::WARP_BYTES;
+    // the exchange buffer (32 KB) and its alignment; the table (at most
+    // 32 KB) is static
+    const size_t smem = 128 + (size_t)kDqWarps * DqTrCfg<D>::WARP_BYTES;
 #define KVQ_DQ(BB)                                                                          \
     case BB: {                                                                              \
         const cudaError_t e = cudaFuncSetAttribute(                                         \
