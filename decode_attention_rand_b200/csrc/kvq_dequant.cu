@@ -314,16 +314,19 @@ dequant_fast_kernel(DqArgs A) {
             for (int k = 0; k < 16; k++)
                 r[k] = (float)((nw[k >> 2] >> (8 * (k & 3))) & 0xFFu) * sc;
         } else {
-            const uint2 nq = make_uint2(cur.nq.x, cur.nq.y);
-            const uint32_t pr = cur.pr;
-            const float LO = half_bits_to_float((uint16_t)(pr & 0xFFFF));
-            const float step = (half_bits_to_float((uint16_t)(pr >> 16)) - LO) * (1.f / 15.f);
-            // 2^(LO + c step) / sqrt(d) = 2^(LO - S/2 + c step)
-            const float base = LO - 0.5f * (float)S;
+            // log2(r / sqrt(d)) = LO - S / 2 + c (HI - LO) / 15 = f A + B with
+            // f = 1 + c / 16 (the nibble as mantissa bits, no conversion),
+            // A = 16 (HI - LO) / 15, B = LO - S / 2 - A
+            const float LO = half_bits_to_float((uint16_t)(cur.pr & 0xFFFF));
+            const float A16 = (half_bits_to_float((uint16_t)(cur.pr >> 16)) - LO) * (16.f / 15.f);
+            const float B16 = LO - 0.5f * (float)S - A16;
 #pragma unroll
             for (int k = 0; k < 16; k++) {
-                const uint32_t c = ((k < 8 ? nq.x : nq.y) >> (4 * (k & 7))) & 0xFu;
-                r[k] = exp2f(fmaf((float)c, step, base));
+                const int sh4 = 4 * (k & 7);
+                const uint32_t w = k < 8 ? cur.nq.x : cur.nq.y;
+                const uint32_t mant = sh4 <= 19 ? (w << (19 - sh4)) : (w >> (sh4 - 19));
+                const float f = __uint_as_float((mant & 0x00780000u) | 0x3F800000u);
+                asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r[k]) : "f"(fmaf(f, A16, B16)));
             }
         }
         f32x2 P[16];
