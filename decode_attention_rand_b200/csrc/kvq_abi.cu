@@ -298,10 +298,11 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs, const kvq_plane* in
 }
 
 int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx, int32_t sm_count) {
-    // One CTA runs per SM, streaming tiles of about 128 tokens, and every CTA
-    // pays a fixed cost (prologue, merge, combine) of about three tiles.  The
-    // launch takes waves x (tiles per CTA + 3) tile times; pick the split
-    // count that minimises it, the fewer CTAs on ties.
+    // One CTA runs per SM; a CTA's time is its tokens (the block loop skips
+    // what is past its split) plus a fixed cost (prologue, the first tile's
+    // copy, merge, combine) of about 512 tokens' worth.  The launch takes
+    // waves x (tokens per CTA + 512); pick the split count that minimises it,
+    // the fewer CTAs on ties.  Splits are at least 128 tokens long.
     if (B <= 0 || H_kv <= 0 || max_ctx <= 0 || sm_count <= 0) return 1;
     const int64_t units = (int64_t)B * H_kv;
     const int64_t tiles = (max_ctx + 127) / 128;
@@ -313,8 +314,8 @@ int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx, int32_t 
     int64_t best = 1, best_cost = -1;
     for (int64_t s = 1; s <= max_s; s++) {
         const int64_t waves = (units * s + sm_count - 1) / sm_count;
-        const int64_t per_cta = (tiles + s - 1) / s;
-        const int64_t cost = waves * (per_cta + 3);
+        const int64_t per_cta = (max_ctx + s - 1) / s;
+        const int64_t cost = waves * (per_cta + 512);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best = s;

@@ -217,9 +217,10 @@ int kvq_dequant(const kvq_codec* codec, const int8_t* signs,
 
 /* Split count the library would choose for a decode launch (host logic,
  * deterministic).  Its cost model: one CTA per SM, a CTA's time is its
- * 128-token units plus a fixed cost of about three units; the split count
- * minimises waves x (units per CTA + 3) over at most eight waves on sm_count
- * SMs, the fewer CTAs on ties.  At least 1, at most ceil(max_ctx / 128). */
+ * ceil(max_ctx / splits) tokens plus a fixed cost of about 512 tokens'
+ * worth (prologue, first copy, merge, combine); the split count minimises
+ * waves x (tokens per CTA + 512) over at most eight waves on sm_count SMs,
+ * the fewer CTAs on ties.  At least 1, at most ceil(max_ctx / 128). */
 int32_t kvq_decode_num_splits(int32_t B, int32_t H_kv, int64_t max_ctx,
                               int32_t sm_count);
 

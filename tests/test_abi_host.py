@@ -66,18 +66,18 @@ def test_split_heuristic():
         assert 1 <= s <= max(1, (ctx + 127) // 128)
         assert s == kvq.kvq_decode_num_splits(B, H, ctx, sm)
         assert B * H * s <= 8 * sm + B * H
-    # the model: waves x (128-token tiles per CTA + 3), minimised, fewer CTAs on ties
+    # the model: waves x (tokens per CTA + 512), minimised, fewer CTAs on ties
     def cost(B, H, ctx, s, sm=148):
-        tiles = -(-ctx // 128)
-        return -(-(B * H * s) // sm) * (-(-tiles // s) + 3)
+        return -(-(B * H * s) // sm) * (-(-ctx // s) + 512)
     for B, H, ctx in [(8, 8, 32768), (4, 4, 65536), (1, 8, 4096), (2, 8, 4096), (16, 8, 8192)]:
         s = kvq.kvq_decode_num_splits(B, H, ctx, 148)
         best = min(cost(B, H, ctx, t) for t in range(1, -(-ctx // 128) + 1)
                    if B * H * t <= 8 * 148 + B * H)
         assert cost(B, H, ctx, s) == best, (B, H, ctx, s)
-    # the decode workloads: one wave of 128 CTAs of two tiles each for the
-    # Llama-shaped layer, about four waves for the two long-context ones
-    assert kvq.kvq_decode_num_splits(1, 8, 4096, 148) == 16
+    # the decode workloads: one wave of 144 CTAs of 228 tokens each for the
+    # Llama-shaped layer (16 splits ran 8 % slower), about four waves for the
+    # Mistral-shaped one, one wave of 144 for the TinyLlama-shaped one
+    assert kvq.kvq_decode_num_splits(1, 8, 4096, 148) == 18
     assert kvq.kvq_decode_num_splits(8, 8, 32768, 148) == 9
     assert kvq.kvq_decode_num_splits(4, 4, 65536, 148) == 9
     assert kvq.kvq_decode_num_splits(0, 8, 100, 148) == 1

@@ -62,6 +62,8 @@ def _noalloc(w, kc, vc, skd, svd, Kp, Vp, q, ctx, tau, S, err, like):
 
 @pytest.mark.parametrize("name,ctx_lens,splits", [
     # 16 splits of 8 KV heads: one cluster per KV head, partials in shared memory
+    ("llama7b_layer_b1_hq32_hkv8_d128_ctx4096", None, 16),
+    # the default split count (18 here: last-CTA combine)
     ("llama7b_layer_b1_hq32_hkv8_d128_ctx4096", None, None),
     # 20 splits (more than a cluster takes): partials and completion counters
     # in the built-in scratch array, merged by the last CTA of each KV head
