@@ -39,13 +39,15 @@ def _signs(rng, d):
     return np.where(rng.integers(0, 2, d) == 0, 1, -1).astype(np.int8)
 
 
-@pytest.mark.parametrize("splits,base", [(3, 300), (16, 4090), (40, 4090)])
+@pytest.mark.parametrize("splits,base", [(3, 300), (16, 4090), (40, 4090), (2, 1500)])
 def test_graph_of_chained_steps_matches_oracle(dev, splits, base):
     """3 layers x 4 steps, B 2, 2 KV heads, G 4, d 128; the first case
     splits 300..303 tokens three ways (last-CTA combine), the second takes
     16 splits (one cluster per KV head) over 4090..4093 tokens, the third 40
-    splits (160 CTAs, more than one wave; 256-token tiles for layers 1 and
-    2, 128-token tiles for layer 0's 8-bit codes)."""
+    splits (160 CTAs, more than one wave), all three with 128-token tiles
+    (splits of at most 256 tokens); the fourth two splits of about 750
+    tokens (256-token tiles for layers 1 and 2, 128-token tiles for layer
+    0's 8-bit codes)."""
     layers, steps, B, H_kv, G, d = 3, 4, 2, 2, 4, 128
     H_q = G * H_kv
     cap = (base + steps + 15) // 16 * 16

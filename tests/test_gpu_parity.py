@@ -320,10 +320,11 @@ def test_decode_every_codec(dev, d, G, LK, LV, mk, mv):
 def test_decode_multi_wave(dev, G, LK, LV):
     """Launches of more than one wave of CTAs (here 8 x 4 x 6 = 192 > 148)
     with G up to 4 and 5..7-bit codes: the one-CTA instance with 256-token
-    tiles on this contiguous cache (the two-CTAs-per-SM instance serves paged
-    caches: test_paged); against the oracle."""
+    tiles on this contiguous cache (splits of 336 tokens; the two-CTAs-per-SM
+    instance serves paged caches: test_paged); against the oracle."""
     B, H_kv = 8, 4
-    got, want, err = run_decode_case(B, G * H_kv, H_kv, 128, [700, 1, 129, 513, 0, 640, 64, 333],
+    got, want, err = run_decode_case(B, G * H_kv, H_kv, 128,
+                                     [2000, 1, 129, 1500, 0, 1800, 64, 333],
                                      LK, LV, seed=G + LK, splits=6)
     assert err == 0
     e = rel_l2(got, want)

@@ -133,7 +133,7 @@ def _signs(rng, d):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("d,G,LK,LV,N,S", [
-    (128, 4, 128, 64, 3, 4),    # the staged kernel, 256-token tiles
+    (128, 4, 128, 64, 3, 4),    # the staged kernel, one CTA per SM
     (64, 8, 256, 256, 2, 3),    # staged, one shared table
     (32, 2, 1000, 24, 3, 2),    # the runtime-width kernel
 ])
