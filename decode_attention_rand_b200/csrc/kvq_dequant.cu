@@ -7,10 +7,14 @@
 // D H / sqrt(d) (H symmetric, H H = d I).  r^ = c M / 255 (8-bit linear) or
 // 2^(LO + c (HI - LO) / 15) (4-bit log space).
 //
-// Work layout mirrors the encode kernel: one vector per group of NL lanes,
-// EPL elements per lane, FWHT in registers plus shuffles, 128-bit stores.
-// cos/sin of the L bin centres come from a shared-memory table (L <= 4096)
-// or from sincospif for larger codebooks.
+// Two kernels.  The fast one (d = 64, 128, 256 and L <= 256) keeps 32
+// elements per lane, looks the bin centres up in a static shared-memory
+// table and runs the butterfly stages over the lane index bits in registers
+// after one exchange through shared memory (see dequant_fast_kernel).  The
+// general one (any d and L) mirrors the encode kernel: one vector per group
+// of NL lanes, EPL elements per lane, FWHT in registers plus shuffles,
+// 128-bit stores; cos/sin of the L bin centres come from a shared-memory
+// table (L <= 4096) or from sincospif for larger codebooks.
 #include "kvq_internal.h"
 
 namespace kvq {
