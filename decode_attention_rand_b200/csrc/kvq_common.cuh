@@ -271,6 +271,90 @@ __device__ __forceinline__ void fwht_pairs(f32x2 (&P)[16], int lg) {
     }
 }
 
+// ------------------------------------------- lane slices <-> runs ----
+// A vector of d = 32 NL elements held 32 per lane (lane l of its group: the
+// slice l 32 .. l 32 + 31, as 16 packed pairs) is transposed through shared
+// memory so that lane l holds, for every slice Lh, the run of RL = 32 / NL
+// elements starting at Lh 32 + l RL (P[Lh RL/2 .. Lh RL/2 + RL/2 - 1]).  The
+// butterfly stages over the slice index then run in registers (fwht_runs)
+// instead of through shuffles.  Lane (g, l) writes its 16-byte chunk q to
+// slot q ^ f(g, l) of its 8-chunk block, f(g, l) = l K + (g mod K) with
+// K = 8 / NL; a quarter warp (K vectors of NL lanes) then covers all eight
+// bank groups on the writes and on the reads (chunk l K + h of the block of
+// lane Lh sits in slot (l ^ Lh) K + (h ^ (g mod K))), and on a 128-byte
+// aligned block both addresses are a per-lane base XOR a constant.  Chunks
+// move as single 128-bit accesses: two 64-bit ones would each be served per
+// half warp, where the slot pattern does not keep the banks apart.  The
+// "memory" clobbers keep them on their side of the __syncwarp()s.
+__device__ __forceinline__ void xch_store(uint32_t addr, f32x2 a, f32x2 b) {
+    asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(addr), "l"(a), "l"(b) : "memory");
+}
+__device__ __forceinline__ void xch_load(uint32_t addr, f32x2& a, f32x2& b) {
+    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr) : "memory");
+}
+
+template <int NL>
+struct LaneRuns {
+    static constexpr int RL = 32 / NL;              // elements per run
+    static constexpr int K = 8 / NL;                // chunks a lane reads from each block
+    static constexpr int WARP_BYTES = 32 * 8 * 16;  // exchange bytes of one warp
+    uint32_t xw, xr;  // chunk q: xw ^ (q << 4); run Lh, chunk h: (xr ^ ((Lh K + h) << 4)) + Lh 128
+    // warp_base: shared-window address of the warp's WARP_BYTES, 128-byte aligned
+    __device__ __forceinline__ LaneRuns(uint32_t warp_base, int grp, int lg) {
+        const uint32_t row = warp_base + (uint32_t)grp * (NL * 128);
+        const uint32_t sw = (uint32_t)(lg * K + grp % K) << 4;
+        xw = row + (uint32_t)lg * 128 + sw;
+        xr = row | sw;
+    }
+    // slices -> runs (the whole warp takes part)
+    __device__ __forceinline__ void to_runs(f32x2 (&P)[16]) const {
+        __syncwarp();  // earlier readers of the buffer are done
+#pragma unroll
+        for (int q = 0; q < 8; q++) xch_store(xw ^ (q << 4), P[2 * q], P[2 * q + 1]);
+        __syncwarp();
+#pragma unroll
+        for (int Lh = 0; Lh < NL; Lh++)
+#pragma unroll
+            for (int h = 0; h < K; h++)
+                xch_load((xr ^ ((Lh * K + h) << 4)) + Lh * 128, P[Lh * (RL / 2) + 2 * h],
+                         P[Lh * (RL / 2) + 2 * h + 1]);
+    }
+    // runs -> slices
+    __device__ __forceinline__ void from_runs(f32x2 (&P)[16]) const {
+        __syncwarp();
+#pragma unroll
+        for (int Lh = 0; Lh < NL; Lh++)
+#pragma unroll
+            for (int h = 0; h < K; h++)
+                xch_store((xr ^ ((Lh * K + h) << 4)) + Lh * 128, P[Lh * (RL / 2) + 2 * h],
+                          P[Lh * (RL / 2) + 2 * h + 1]);
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 8; q++) xch_load(xw ^ (q << 4), P[2 * q], P[2 * q + 1]);
+    }
+};
+
+// Butterflies over the slice index of a vector held as runs (LaneRuns):
+// the stages fwht_pairs<NL> runs across lanes, here in registers.
+template <int NL>
+__device__ __forceinline__ void fwht_runs(f32x2 (&P)[16]) {
+    constexpr int H = 16 / NL;  // pairs per run
+#pragma unroll
+    for (int st = 1; st < NL; st <<= 1) {
+#pragma unroll
+        for (int Lh = 0; Lh < NL; Lh++) {
+            if ((Lh & st) == 0) {
+#pragma unroll
+                for (int u = 0; u < H; u++) {
+                    const f32x2 a = P[Lh * H + u], b = P[(Lh + st) * H + u];
+                    P[Lh * H + u] = add2(a, b);
+                    P[(Lh + st) * H + u] = sub2(a, b);
+                }
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------ device errors ----
 
 __device__ __forceinline__ void report(int32_t* err_word, int bits) {

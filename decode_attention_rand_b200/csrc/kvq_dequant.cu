@@ -192,35 +192,11 @@ struct DqFastCfg {
 
 constexpr int kDqFastBlocksPerSM = 3;  // registers for one tile ahead in flight
 
-// The tail is transposed: after the in-lane butterfly stages, the lanes of a
-// vector exchange their elements through shared memory instead of shuffles,
-// so that the stages over the lane index bits run in registers: lane l then
-// holds, for every original lane index Lh, the run of RL = 32 / NL elements
+// The butterfly stages over the lane index bits run in registers after a
+// transposition of each vector through shared memory (LaneRuns): lane l then
+// holds, for every former lane index Lh, the run of RL = 32 / NL elements
 // starting at Lh 32 + l RL, and stores it as 16-byte (8-byte for d = 256)
-// words.  Lane (g, l) of vector g writes its 16-byte chunk q to slot
-// q ^ f(g, l) of its 8-chunk block, f(g, l) = l K + (g mod K) with
-// K = 8 / NL; a quarter warp (K vectors of NL lanes) then covers all eight
-// bank groups, on the writes and on the reads (chunk l K + h of the block of
-// lane Lh sits in slot (l ^ Lh) K + (h ^ (g mod K))).  On a 128-byte aligned
-// block both addresses are a per-lane base XOR a constant.
-template <int D>
-struct DqTrCfg {
-    static constexpr int NL = D / 32;
-    static constexpr int RL = 32 / NL;       // elements per run after the exchange
-    static constexpr int K = 8 / NL;         // runs of 16 bytes a lane reads per block
-    static constexpr int WARP_BYTES = 32 * 8 * 16;
-};
-
-// One 16-byte chunk of the exchange, moved as a single 128-bit shared-memory
-// access: two 64-bit loads would each be served per half warp, where the
-// chunk rotation does not keep the banks apart.  The "memory" clobbers keep
-// the accesses on their side of the __syncwarp()s around the exchange.
-__device__ __forceinline__ void xch_store(uint32_t addr, f32x2 a, f32x2 b) {
-    asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(addr), "l"(a), "l"(b) : "memory");
-}
-__device__ __forceinline__ void xch_load(uint32_t addr, f32x2& a, f32x2& b) {
-    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr) : "memory");
-}
+// words.
 
 template <int D, int B>
 __global__ void __launch_bounds__(kDqWarps * 32, kDqFastBlocksPerSM)
@@ -250,18 +226,15 @@ dequant_fast_kernel(DqArgs A) {
 #pragma unroll
     for (int w = 0; w < 16; w++) {
         // pair w is pair w % (RL / 2) of run w / (RL / 2)
-        const int e = (w / (DqTrCfg<D>::RL / 2)) * 32 + lg * DqTrCfg<D>::RL +
-                      2 * (w % (DqTrCfg<D>::RL / 2));
+        constexpr int RL = LaneRuns<NL>::RL;
+        const int e = (w / (RL / 2)) * 32 + lg * RL + 2 * (w % (RL / 2));
         m[w] = (A.signs[e] < 0 ? 0x8000u : 0u) | (A.signs[e + 1] < 0 ? 0x80000000u : 0u);
     }
-    // exchange buffer after the table, 128-byte aligned: [warp][vector][lane][8 chunks]
-    using T = DqTrCfg<D>;
-    const uint32_t xrow =
-        (((uint32_t)__cvta_generic_to_shared(xdyn) + 127u) & ~127u) +
-        (uint32_t)(warp * T::WARP_BYTES + grp * D * 4);
-    const uint32_t xsw = (uint32_t)(lg * T::K + grp % T::K) << 4;
-    const uint32_t xw = xrow + lg * 128 + xsw;  // chunk q goes to xw ^ (q << 4)
-    const uint32_t xr = xrow | xsw;             // run Lh, chunk h: (xr ^ ((Lh K + h) << 4)) + Lh 128
+    // exchange buffer, 128-byte aligned: [warp][vector][lane][8 chunks]
+    using T = LaneRuns<NL>;
+    const T runs((((uint32_t)__cvta_generic_to_shared(xdyn) + 127u) & ~127u) +
+                     (uint32_t)(warp * T::WARP_BYTES),
+                 grp, lg);
     __syncthreads();
     // byte offset of the lane's replica (code c's entries span 128 bytes)
     const uint32_t tlo = (uint32_t)(lane & 15) * sizeof(float2);
@@ -348,36 +321,8 @@ dequant_fast_kernel(DqArgs A) {
             P[k] = pack2(r[k] * t.x, r[k] * t.y);
         }
         fwht_pairs<1>(P, lg);  // the in-lane stages
-        // chunk q of this lane = pairs 2q, 2q + 1 = elements lg 32 + 4q .. + 3
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < 8; q++)
-            xch_store(xw ^ (q << 4), P[2 * q], P[2 * q + 1]);
-        __syncwarp();
-        // run Lh: chunks lg K + h of the block of lane Lh
-#pragma unroll
-        for (int Lh = 0; Lh < NL; Lh++) {
-#pragma unroll
-            for (int h = 0; h < T::RL / 4; h++) {
-                xch_load((xr ^ ((Lh * T::K + h) << 4)) + Lh * 128, P[Lh * (T::RL / 2) + 2 * h],
-                         P[Lh * (T::RL / 2) + 2 * h + 1]);
-            }
-        }
-        // the stages over the former lane bits, now in registers
-#pragma unroll
-        for (int st = 1; st < NL; st <<= 1) {
-#pragma unroll
-            for (int Lh = 0; Lh < NL; Lh++) {
-                if ((Lh & st) == 0) {
-#pragma unroll
-                    for (int u = 0; u < T::RL / 2; u++) {
-                        const f32x2 a = P[Lh * (T::RL / 2) + u], b = P[(Lh + st) * (T::RL / 2) + u];
-                        P[Lh * (T::RL / 2) + u] = add2(a, b);
-                        P[(Lh + st) * (T::RL / 2) + u] = sub2(a, b);
-                    }
-                }
-            }
-        }
+        runs.to_runs(P);
+        fwht_runs<NL>(P);      // the stages over the former lane bits
         if (valid) {
             uint32_t o[16];
 #pragma unroll
@@ -415,7 +360,7 @@ static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStre
     const dim3 g((unsigned)blocks), b(kDqWarps * 32);
     // the exchange buffer (32 KB) and its alignment; the table (at most
     // 32 KB) is static
-    const size_t smem = 128 + (size_t)kDqWarps * DqTrCfg<D>::WARP_BYTES;
+    const size_t smem = 128 + (size_t)kDqWarps * LaneRuns<D / 32>::WARP_BYTES;
 #define KVQ_DQ(BB)                                                                          \
     case BB: {                                                                              \
         const cudaError_t e = cudaFuncSetAttribute(                                         \
