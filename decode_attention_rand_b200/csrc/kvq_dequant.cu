@@ -246,7 +246,9 @@ dequant_fast_kernel(DqArgs A) {
     const uint32_t n_tiles = (uint32_t)((A.n_vec + VPW - 1) / VPW);
     const uint32_t stride = gridDim.x * kDqWarps;
     // The code rows of a warp tile are loaded one iteration ahead: the loads
-    // of tile wt + stride are in flight while tile wt is transformed.
+    // of tile wt + stride are in flight while tile wt is transformed.  Codes
+    // are read once and the fp16 vectors written once: both carry the
+    // evict-first hint (.cs).
     struct Rows {
         uint32_t w[5];   // angle words from the lane's first one
         uint4 nq;        // norm bytes (LIN8: 16, LOG4: 8 in .x/.y)
@@ -260,12 +262,12 @@ dequant_fast_kernel(DqArgs A) {
             (int64_t)vt * A.in.capacity + A.pos0 + (int64_t)(vv - vt * (uint32_t)A.T);
         const uint32_t* ar = reinterpret_cast<const uint32_t*>(A.in.angles) + row * AW;
 #pragma unroll
-        for (int j = 0; j < 5; j++) R.w[j] = wbase + j < AW ? ar[wbase + j] : 0u;
+        for (int j = 0; j < 5; j++) R.w[j] = wbase + j < AW ? __ldcs(ar + wbase + j) : 0u;
         if (lin8) {
-            R.nq = *reinterpret_cast<const uint4*>(A.in.norms + row * (D / 2) + lg * 16);
+            R.nq = __ldcs(reinterpret_cast<const uint4*>(A.in.norms + row * (D / 2) + lg * 16));
             R.pr = reinterpret_cast<const uint16_t*>(A.in.params)[row];
         } else {
-            const uint2 q2 = *reinterpret_cast<const uint2*>(A.in.norms + row * (D / 4) + lg * 8);
+            const uint2 q2 = __ldcs(reinterpret_cast<const uint2*>(A.in.norms + row * (D / 4) + lg * 8));
             R.nq = make_uint4(q2.x, q2.y, 0u, 0u);
             R.pr = reinterpret_cast<const uint32_t*>(A.in.params)[row];
         }
@@ -335,12 +337,12 @@ dequant_fast_kernel(DqArgs A) {
             for (int Lh = 0; Lh < NL; Lh++) {
                 const uint32_t* oo = o + Lh * (T::RL / 2);
                 if constexpr (T::RL == 4) {
-                    *reinterpret_cast<uint2*>(y + Lh * 32) = make_uint2(oo[0], oo[1]);
+                    __stcs(reinterpret_cast<uint2*>(y + Lh * 32), make_uint2(oo[0], oo[1]));
                 } else {
 #pragma unroll
                     for (int c = 0; c < T::RL / 8; c++)
-                        reinterpret_cast<uint4*>(y + Lh * 32)[c] =
-                            make_uint4(oo[4 * c], oo[4 * c + 1], oo[4 * c + 2], oo[4 * c + 3]);
+                        __stcs(reinterpret_cast<uint4*>(y + Lh * 32) + c,
+                               make_uint4(oo[4 * c], oo[4 * c + 1], oo[4 * c + 2], oo[4 * c + 3]));
                 }
             }
         }
