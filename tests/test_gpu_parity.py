@@ -241,6 +241,34 @@ def test_dequant_sweep(dev, d, L):
         assert err.max() <= REL_L2_TOL, (mode, err.max())
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("B,H,T,pos0", [(1, 1, 3, 0), (1, 3, 7, 5), (3, 2, 13, 1), (2, 5, 101, 17)])
+def test_dequant_fast_ragged_tiles(dev, d, B, H, T, pos0):
+    """The fast dequant (32 elements per lane, d/32 lanes per vector, 32*32/d
+    vectors per warp tile, the lane-bit butterflies after a transposition
+    through shared memory) on vector counts that leave the last warp tile
+    partly filled, fewer vectors than one tile included, with rows read from
+    an offset position of each (b, KV head) run."""
+    s = _signs(d + B * 7 + T, d)
+    x = _rand_x(B, H, T, d, seed=d * 3 + T)
+    n = B * H * T
+    for L, mode in ((128, O.MODE_LIN8), (64, O.MODE_LOG4), (256, O.MODE_LIN8), (16, O.MODE_LOG4)):
+        oc = O.encode(x, s, L, mode)
+        c = kvq.codec(d, L, mode)
+        plane = kvq.alloc_plane(c, B, H, (pos0 + T + 15) // 16 * 16 + 16)
+        k = 0
+        for b in range(B):
+            for h in range(H):
+                put_rows(plane, oc.take(slice(k, k + T)), b, h, pos0)
+                k += T
+        y = kvq.dequant(c, _dev_signs(s), plane, T, pos0=pos0)
+        torch.cuda.synchronize()
+        got = y.cpu().numpy().astype(np.float64).reshape(-1, d)
+        assert got.shape[0] == n
+        err = rel_l2(got, O.dequant(oc, s))
+        assert err.max() <= REL_L2_TOL, (L, mode, err.max())
+
+
 # ------------------------------------------------------------------ decode --
 
 def run_decode_case(B, H_q, H_kv, d, ctx_lens, LK, LV, seed=0, splits=None, cap=None,
