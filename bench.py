@@ -90,11 +90,16 @@ def parse():
     p.add_argument("--no-extra", action="store_true",
                    help="headline workload only (no TinyLlama / Llama-layer steps, no prefill)")
     p.add_argument("--case", default=None,
-                   choices=["decode_layer", "step_layer", "encode_layer", "dequant_layer"],
+                   choices=["decode_layer", "step_layer", "encode_layer", "dequant_layer",
+                            "shard_layer"],
                    help="run one kernel case only (for profiler captures): the decode (or the "
                         "append + decode step) of --layer of --workload, or the prefill encode "
                         "(or dequant) of 8 batch entries of one layer; --steps launches after 3 "
-                        "warm-up launches")
+                        "warm-up launches.  shard_layer: the context-sharded decode of --layer "
+                        "with --parts ranks emulated on this GPU (each holding 1/parts of every "
+                        "sequence: its split partials, then the merge of all parts)")
+    p.add_argument("--parts", type=int, default=2,
+                   help="shard_layer case: ranks the context is spread over")
     p.add_argument("--L", type=int, default=None,
                    help="with --case: codebook size for K and V instead of the workload's "
                         "(sizes outside the fast kernels' set select the general kernels)")
@@ -620,6 +625,51 @@ def run_case(args):
             what = f"append + decode step {w.name} layer {layer}, {S} splits"
         if args.L:
             what += f", L_K = L_V = {args.L}"
+    elif args.case == "shard_layer":
+        # context-sharded decode with the ranks emulated one after another on
+        # this GPU: part r holds tokens [r ctx / N, (r + 1) ctx / N) of every
+        # sequence in planes of its own and writes its split partials into
+        # row r of the stacked buffer the merge reads
+        w = synth.WORKLOADS[args.workload]
+        layer, N = args.layer, max(1, args.parts)
+        sk, sv = synth.layer_signs(w, layer)
+        skd, svd = torch.from_numpy(sk).to(device), torch.from_numpy(sv).to(device)
+        kc = kvq.codec(w.d, args.L or w.L_K[layer], w.mode_K)
+        vc = kvq.codec(w.d, args.L or w.L_V[layer], w.mode_V)
+        bounds = [(r * w.ctx // N, (r + 1) * w.ctx // N) for r in range(N)]
+        planes = []
+        for lo, hi in bounds:
+            cap = max(16, (hi - lo + 15) // 16 * 16)
+            pr = []
+            for kind, c, sg in ((synth.KIND_K, kc, skd), (synth.KIND_V, vc, svd)):
+                pl = kvq.alloc_plane(c, w.B, w.H_kv, cap, device)
+                x = synth.kv(w, layer, kind, device=device)[:, :, lo:hi].contiguous()
+                kvq.encode(c, sg, x, pl, 0)
+                del x
+                pr.append(pl)
+            planes.append(pr)
+        torch.cuda.empty_cache()
+        q = synth.queries(w, layer, device=device)
+        out = torch.empty((w.B, w.H_q, w.d), dtype=torch.float16, device=device)
+        sm = torch.cuda.get_device_properties(device).multi_processor_count
+        max_part = max(hi - lo for lo, hi in bounds)
+        S = kvq.kvq_decode_num_splits(w.B, w.H_kv, max_part, sm)
+        nbytes = kvq.kvq_decode_workspace_bytes(w.B, w.H_q, w.d, S)
+        parts = torch.zeros((N, nbytes), dtype=torch.uint8, device=device)
+        ctxs = [torch.full((w.B,), hi - lo, dtype=torch.int32, device=device) for lo, hi in bounds]
+        tau = 1.0 / math.sqrt(w.d)
+
+        def merge():
+            kvq.kvq_decode_merge_partials(parts, N, w.B, w.H_q, w.d, S, svd, out, kvq.OUT_FP16)
+
+        def run():
+            for r, (lo, hi) in enumerate(bounds):
+                kvq.kvq_decode_attn_partials(q, kc, vc, skd, svd, planes[r][0].c(),
+                                             planes[r][1].c(), ctxs[r], w.B, w.H_q, w.H_kv,
+                                             hi - lo, tau, S, parts[r], nbytes)
+            merge()
+        what = (f"context-sharded decode {w.name} layer {layer}: {N} parts of {max_part} tokens, "
+                f"{S} splits each, then the merge")
     else:
         w = synth.WORKLOADS[PREFILL]
         sk, sv = synth.layer_signs(w, 0)
@@ -651,7 +701,25 @@ def run_case(args):
         run()
     e1.record()
     torch.cuda.synchronize()
-    print(json.dumps({"case": what, "us_per_launch": e0.elapsed_time(e1) * 1e3 / steps}), flush=True)
+    res = {"case": what, "us_per_launch": e0.elapsed_time(e1) * 1e3 / steps}
+    if args.case == "shard_layer":
+        # the merge alone, replayed from a CUDA graph (a launch of a few
+        # microseconds would otherwise be timed at the host's call rate), and
+        # the bytes it reads (every part's partials) and writes
+        graph, side = torch.cuda.CUDAGraph(), torch.cuda.Stream()
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(steps):
+                merge()
+        graph.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        res["merge_us"] = e0.elapsed_time(e1) * 1e3 / steps
+        del graph
+        res["merge_bytes"] = N * nbytes + out.numel() * out.element_size()
+    print(json.dumps(res), flush=True)
     return 0
 
 
