@@ -201,6 +201,11 @@ constexpr int kDqFastBlocksPerSM = 3;  // registers for one tile ahead in flight
 template <int D, int B>
 __global__ void __launch_bounds__(kDqWarps * 32, kDqFastBlocksPerSM)
 dequant_fast_kernel(DqArgs A) {
+    // Launched as a programmatic dependent of the previous kernel on the
+    // stream: the next kernel may start its own setup now, and this one builds
+    // its table (from its arguments alone) while the previous one drains; no
+    // global memory is read or written before griddepcontrol.wait.
+    asm volatile("griddepcontrol.launch_dependents;");
     using Cfg = DqFastCfg<D>;
     constexpr int NL = Cfg::NL, VPW = Cfg::VPW, S = Cfg::S;
     // r-free (cos + sin, cos - sin) of each bin centre, 16 copies side by side
@@ -222,6 +227,7 @@ dequant_fast_kernel(DqArgs A) {
     __syncthreads();
     for (int i = threadIdx.x; i < (16 << B); i += blockDim.x)
         if (i & 15) tab[i] = tab[i & ~15];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     uint32_t m[16];  // fp16 sign bits of D for this lane's output element pairs
 #pragma unroll
     for (int w = 0; w < 16; w++) {
@@ -363,13 +369,25 @@ static cudaError_t launch_dequant_fast_d(const DqArgs& a, int sm_count, cudaStre
     // the exchange buffer (32 KB) and its alignment; the table (at most
     // 32 KB) is static
     const size_t smem = 128 + (size_t)kDqWarps * LaneRuns<D / 32>::WARP_BYTES;
+    // programmatic dependent launch (see the kernel)
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = g;
+    cfg.blockDim = b;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
 #define KVQ_DQ(BB)                                                                          \
     case BB: {                                                                              \
         const cudaError_t e = cudaFuncSetAttribute(                                         \
             dequant_fast_kernel<D, BB>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
             (int)smem);                                                                     \
         if (e != cudaSuccess) return e;                                                     \
-        dequant_fast_kernel<D, BB><<<g, b, smem, stream>>>(a);                              \
+        const cudaError_t l = cudaLaunchKernelEx(&cfg, dequant_fast_kernel<D, BB>, a);      \
+        if (l != cudaSuccess) return l;                                                     \
         break;                                                                              \
     }
     switch (a.c.bits) {
