@@ -217,3 +217,21 @@ def test_merge_of_empty_parts_is_zero(dev):
     out = shard.merge_partials(parts, B, H_q, d, S, signs)
     torch.cuda.synchronize()
     assert bool((out == 0).all())
+
+
+@pytest.mark.gpu
+def test_bench_shard_case_runs(dev):
+    """bench.py's context-sharded case (ranks emulated on this GPU) on the
+    Llama-shaped layer split three ways: one JSON line with the whole step's
+    and the merge's times and the bytes the merge moves."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--case", "shard_layer",
+                        "--workload", "llama7b_layer_b1_hq32_hkv8_d128_ctx4096", "--parts", "3",
+                        "--steps", "2"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    assert "3 parts" in res["case"]
+    assert res["us_per_launch"] > 0 and res["merge_us"] > 0
+    S = int(res["case"].split(" splits")[0].split()[-1])
+    assert res["merge_bytes"] == 3 * kvq.kvq_decode_workspace_bytes(1, 32, 128, S) + 32 * 128 * 2
